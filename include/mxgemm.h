@@ -1,0 +1,169 @@
+/*
+ * mxgemm.h -- C ABI of the B200 (sm_100a) MX block-scaled matrix multiply.
+ *
+ * Operation (all entry points below serve it):
+ *
+ *     C[m][n] = sum_k  dec(A[m][k]) * 2^(SA[m][k/32]-127)
+ *                    * dec(B[n][k]) * 2^(SB[n][k/32]-127)
+ *
+ * accumulated in FP32 and stored as BF16.  This is the "MXFP scaled GEMM" of
+ * the 5ulink.com page "PyTorch 接上 FlyDSL" (support-matrix table: A
+ * row-major, B column-major i.e. NT, K a multiple of 128; note under the
+ * table: one E8M0 scale per 32 values "BlockWise1x32", FP32 accumulation,
+ * FP16/BF16 output -- this library writes BF16).  The devotd.net page, section
+ * 2, reports the MXFP8 and MXFP4 NT suites this operation is measured on.
+ *
+ * Formats (OCP Microscaling v1.0 encodings; the pages only name them):
+ *   MXGEMM_FMT_MXFP8: elements FP8 E4M3 (max 448, S.1111.111 = NaN), one byte
+ *                     each; a row of K elements is K bytes.
+ *   MXGEMM_FMT_MXFP4: elements FP4 E2M1, two per byte, element 2j in the low
+ *                     nibble of byte j; a row of K elements is K/2 bytes.
+ *   scales:           E8M0 bytes, value 2^(e-127), 0xFF = NaN, one per 32
+ *                     consecutive K elements.
+ *
+ * Canonical layouts (caller-owned, dense, row-major, device memory unless an
+ * entry point says "host"):
+ *   A        [M][row_bytes(K)]   row_bytes = K (MXFP8) or K/2 (MXFP4)
+ *   A_scales [M][K/32]           uint8
+ *   B        [N][row_bytes(K)]   (B stored as N rows of K: "column-major K x N")
+ *   B_scales [N][K/32]           uint8
+ *   C        [M][N]              bfloat16 bits (uint16)
+ *
+ * Requirements checked before any launch: K > 0 and K % 128 == 0; M, N >= 1;
+ * every pointer non-NULL and 16-byte aligned; fmt one of the two formats.
+ * Violations return an error status and launch nothing.  The calls are
+ * stream-ordered and do not synchronise the host unless stated.  A handle is
+ * not thread-safe: use one handle per host thread / stream.
+ */
+#ifndef MXGEMM_H
+#define MXGEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MXGEMM_API __attribute__((visibility("default")))
+#else
+#define MXGEMM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct mxgemm_ctx *mxgemm_handle;
+
+/* Element formats. */
+enum {
+    MXGEMM_FMT_MXFP8_E4M3 = 0,
+    MXGEMM_FMT_MXFP4_E2M1 = 1
+};
+
+/* Status codes.  Every entry point returns one of these. */
+enum {
+    MXGEMM_OK = 0,
+    MXGEMM_ERR_INVALID_ARG = 1,        /* bad size, format, NULL pointer or handle */
+    MXGEMM_ERR_ALIGNMENT = 2,          /* a pointer is not 16-byte aligned */
+    MXGEMM_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not compute capability 10.0 */
+    MXGEMM_ERR_OOM = 4,                /* workspace allocation failed */
+    MXGEMM_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+    MXGEMM_ERR_TIMEOUT = 6             /* a kernel gave up on a bounded wait */
+};
+
+/* Schedules for the GEMM's persistent tile scheduler (mxgemm_set_schedule). */
+enum {
+    MXGEMM_SCHED_AUTO = 0,     /* pick per shape (default) */
+    MXGEMM_SCHED_DP = 1,       /* one whole output tile per work unit */
+    MXGEMM_SCHED_SPLITK = 2,   /* each tile split into `splits` equal K ranges */
+    MXGEMM_SCHED_STREAMK = 3   /* K iterations of all tiles split evenly over the SMs */
+};
+
+/* Create a handle bound to the current CUDA device.  The device must be an
+ * sm_100 part (B200).  The handle owns a lazily grown device workspace
+ * (repacked scales, split-K partials and tile counters).
+ * out: receives the handle (host pointer, not NULL). */
+MXGEMM_API int mxgemm_create(mxgemm_handle *out);
+
+/* Free the handle and its workspace (synchronises the device first).
+ * NULL is accepted and ignored. */
+MXGEMM_API int mxgemm_destroy(mxgemm_handle h);
+
+/* Full hot path on `stream`: repack A_scales and B_scales from the canonical
+ * row-major layout into the tensor-core scale layout (in the handle's
+ * workspace), then run the block-scaled GEMM writing C.  Two kernel launches,
+ * no host synchronisation.  All buffers are device memory.  `stream` is a
+ * cudaStream_t (NULL = legacy default stream). */
+MXGEMM_API int mxgemm_run(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
+               const void *A, const uint8_t *A_scales,
+               const void *B, const uint8_t *B_scales,
+               void *C, void *stream);
+
+/* The first half of mxgemm_run on its own: the scale repack into the
+ * handle's workspace.  Sizes as for mxgemm_run. */
+MXGEMM_API int mxgemm_repack(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
+                  const uint8_t *A_scales, const uint8_t *B_scales, void *stream);
+
+/* The second half of mxgemm_run on its own: the GEMM, reading the scales the
+ * last mxgemm_repack on this handle (same fmt, M, N, K) left in the
+ * workspace.  Returns MXGEMM_ERR_INVALID_ARG if the shape differs from the
+ * last repack. */
+MXGEMM_API int mxgemm_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
+                const void *A, const void *B, void *C, void *stream);
+
+/* mxgemm_run with HOST buffers (pinned or pageable): copies the operands and
+ * scales to device staging buffers owned by the handle, runs the hot path and
+ * copies C back to the host buffer C_host, all on `stream`, then synchronises
+ * the stream.  Host buffers use the canonical layouts above. */
+MXGEMM_API int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
+                    const void *A_host, const uint8_t *A_scales_host,
+                    const void *B_host, const uint8_t *B_scales_host,
+                    void *C_host, void *stream);
+
+/* OCP MX quantisation (the input generator; not part of the timed path).
+ * X: FP32 [R][K] device.  Q: codes [R][row_bytes(K)] device.  scales: E8M0
+ * [R][K/32] device.  Per 32-element block: amax = max|x|, scale exponent
+ * s = floor(log2 amax) - emax (emax 8 for E4M3, 2 for E2M1) clamped to
+ * [-127, 127] (all-zero block: s = -127), elements x / 2^s rounded to nearest
+ * even with saturation at +-448 / +-6, the sign of a zero kept.  A block that
+ * holds a NaN or an infinity gets scale 0xFF and zero codes.  K % 32 == 0. */
+MXGEMM_API int mxgemm_quantize(int fmt, int64_t R, int64_t K, const float *X,
+                    void *Q, uint8_t *scales, void *stream);
+
+/* Force a schedule for later mxgemm_run / mxgemm_gemm calls on this handle.
+ * splits is used by MXGEMM_SCHED_SPLITK (>= 1); workers by
+ * MXGEMM_SCHED_STREAMK (0 = number of SMs). */
+MXGEMM_API int mxgemm_set_schedule(mxgemm_handle h, int schedule, int splits, int workers);
+
+/* Describe the plan mxgemm_gemm would use for a shape: writes up to `cap`
+ * bytes of a NUL-terminated text such as
+ * "fmt=1 swap=1 BN=32 stages=10 tiles=112 kt=16 workers=148 grid=148 sched=streamk". */
+MXGEMM_API int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
+                         char *buf, size_t cap);
+
+/* Read and clear the device error word that kernels set when a bounded wait
+ * runs out.  Synchronises the device.  *code receives 0 if no kernel gave
+ * up, else a nonzero site code; the return value is MXGEMM_ERR_TIMEOUT in
+ * that case, else MXGEMM_OK. */
+MXGEMM_API int mxgemm_check_device_error(mxgemm_handle h, int *code);
+
+/* Set the per-wait time limit of the kernels' bounded waits in nanoseconds
+ * (default 2e9).  0 restores the default. */
+MXGEMM_API int mxgemm_set_wait_limit(mxgemm_handle h, uint64_t ns);
+
+/* Test hook: when `mode` is 1 the next GEMM launch on this handle arms no
+ * TMA load for its first pipeline stage, so the consumer's bounded wait runs
+ * out and the kernel reports MXGEMM_ERR_TIMEOUT through
+ * mxgemm_check_device_error.  The hook disarms itself after one launch. */
+MXGEMM_API int mxgemm_debug_inject(mxgemm_handle h, int mode);
+
+/* Static description of a status code. */
+MXGEMM_API const char *mxgemm_status_string(int status);
+
+/* Library version as "major.minor.patch". */
+MXGEMM_API const char *mxgemm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXGEMM_H */

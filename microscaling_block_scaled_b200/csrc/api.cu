@@ -1,0 +1,397 @@
+// api.cu -- the C ABI declared in include/mxgemm.h.
+//
+// Host-side responsibilities only: argument validation (before any launch),
+// the workspace the handle owns, the scheduling plan, and the order of the
+// two launches of the hot path (scale repack, then the GEMM) on the caller's
+// stream.  Every step of the arithmetic runs in the CUDA kernels of
+// repack.cu, gemm.cu and quant.cu; there is no host fallback.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "../../include/mxgemm.h"
+#include "mx_internal.h"
+
+struct mxgemm_ctx {
+    int device = 0;
+    int num_sms = 0;
+    // scale workspace: repacked A scales then repacked B scales
+    uint8_t *sf = nullptr;
+    size_t sf_cap = 0;
+    int64_t sf_offB = 0;
+    // split partials and per-tile counters (counters kept zero between launches)
+    float *partials = nullptr;
+    size_t partials_cap = 0;
+    uint32_t *counters = nullptr;
+    size_t counters_cap = 0;
+    int *err = nullptr;
+    // device staging of mxgemm_run_host
+    uint8_t *stage = nullptr;
+    size_t stage_cap = 0;
+    // schedule override
+    int sched = MXGEMM_SCHED_AUTO;
+    int splits = 1;
+    int workers = 0;
+    uint64_t limit_ns = 2000000000ull;
+    int inject = 0;
+    // shape of the last repack
+    int last_fmt = -1;
+    int64_t last_M = 0, last_N = 0, last_K = 0;
+};
+
+namespace {
+
+constexpr uint64_t kDefaultLimitNs = 2000000000ull;
+constexpr int64_t kMaxDim = int64_t(1) << 24;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int fmt, int64_t M, int64_t N, int64_t K)
+{
+    if (fmt != MXGEMM_FMT_MXFP8_E4M3 && fmt != MXGEMM_FMT_MXFP4_E2M1)
+        return MXGEMM_ERR_INVALID_ARG;
+    if (M < 1 || N < 1 || K < 128 || K % 128 != 0)
+        return MXGEMM_ERR_INVALID_ARG;
+    if (M > kMaxDim || N > kMaxDim || K > kMaxDim)
+        return MXGEMM_ERR_INVALID_ARG;
+    return MXGEMM_OK;
+}
+
+int check_ptrs(std::initializer_list<const void *> ptrs)
+{
+    for (const void *p : ptrs)
+        if (p == nullptr)
+            return MXGEMM_ERR_INVALID_ARG;
+    for (const void *p : ptrs)
+        if (!aligned16(p))
+            return MXGEMM_ERR_ALIGNMENT;
+    return MXGEMM_OK;
+}
+
+template <typename T>
+int grow(T **buf, size_t *cap, size_t need, bool zero)
+{
+    if (need <= *cap)
+        return MXGEMM_OK;
+    if (*buf) {
+        cudaFree(*buf);
+        *buf = nullptr;
+        *cap = 0;
+    }
+    size_t want = need + need / 4;
+    if (cudaMalloc(reinterpret_cast<void **>(buf), want) != cudaSuccess) {
+        cudaGetLastError();
+        *buf = nullptr;
+        return MXGEMM_ERR_OOM;
+    }
+    if (zero && cudaMemset(*buf, 0, want) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    *cap = want;
+    return MXGEMM_OK;
+}
+
+int enter_device(mxgemm_handle h)
+{
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    if (cur != h->device && cudaSetDevice(h->device) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    return MXGEMM_OK;
+}
+
+int do_repack(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const uint8_t *sa, const uint8_t *sb,
+              cudaStream_t st)
+{
+    const int64_t ba = mxg::sf_repacked_bytes(fmt, M, K);
+    const int64_t bb = mxg::sf_repacked_bytes(fmt, N, K);
+    int rc = grow(&h->sf, &h->sf_cap, static_cast<size_t>(ba + bb), false);
+    if (rc != MXGEMM_OK)
+        return rc;
+    h->sf_offB = ba;
+    if (mxg::launch_repack(fmt, M, N, K, sa, sb, h->sf, h->sf + ba, st) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    h->last_fmt = fmt;
+    h->last_M = M;
+    h->last_N = N;
+    h->last_K = K;
+    return MXGEMM_OK;
+}
+
+int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const void *B, void *C,
+            cudaStream_t st)
+{
+    if (h->last_fmt != fmt || h->last_M != M || h->last_N != N || h->last_K != K)
+        return MXGEMM_ERR_INVALID_ARG;
+    const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers);
+    int rc = grow(&h->partials, &h->partials_cap, static_cast<size_t>(pl.partial_bytes > 0 ? pl.partial_bytes : 16),
+                  false);
+    if (rc != MXGEMM_OK)
+        return rc;
+    rc = grow(&h->counters, &h->counters_cap, static_cast<size_t>(pl.counter_bytes), true);
+    if (rc != MXGEMM_OK)
+        return rc;
+    mxg::GemmBuffers b;
+    b.A = A;
+    b.B = B;
+    b.sfA = h->sf;
+    b.sfB = h->sf + h->sf_offB;
+    b.C = C;
+    b.partials = h->partials;
+    b.counters = h->counters;
+    b.error = h->err;
+    const int inject = h->inject;
+    h->inject = 0;
+    if (mxg::launch_gemm(pl, b, h->limit_ns, inject, st) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    return MXGEMM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *mxgemm_version(void) { return "0.1.0"; }
+
+const char *mxgemm_status_string(int status)
+{
+    switch (status) {
+    case MXGEMM_OK: return "ok";
+    case MXGEMM_ERR_INVALID_ARG: return "invalid argument";
+    case MXGEMM_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case MXGEMM_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100 (B200)";
+    case MXGEMM_ERR_OOM: return "workspace allocation failed";
+    case MXGEMM_ERR_CUDA: return "CUDA call failed";
+    case MXGEMM_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    default: return "unknown status";
+    }
+}
+
+int mxgemm_create(mxgemm_handle *out)
+{
+    if (!out)
+        return MXGEMM_ERR_INVALID_ARG;
+    *out = nullptr;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MXGEMM_ERR_UNSUPPORTED_DEVICE;
+    }
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MXGEMM_ERR_CUDA;
+    }
+    if (prop.major != 10 || prop.minor != 0)
+        return MXGEMM_ERR_UNSUPPORTED_DEVICE;
+    if (mxg::prepare_gemm_kernels() != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    mxgemm_ctx *h = new (std::nothrow) mxgemm_ctx();
+    if (!h)
+        return MXGEMM_ERR_OOM;
+    h->device = dev;
+    h->num_sms = prop.multiProcessorCount;
+    if (cudaMalloc(reinterpret_cast<void **>(&h->err), 16) != cudaSuccess ||
+        cudaMemset(h->err, 0, 16) != cudaSuccess) {
+        cudaGetLastError();
+        delete h;
+        return MXGEMM_ERR_OOM;
+    }
+    *out = h;
+    return MXGEMM_OK;
+}
+
+int mxgemm_destroy(mxgemm_handle h)
+{
+    if (!h)
+        return MXGEMM_OK;
+    int rc = enter_device(h);
+    cudaDeviceSynchronize();
+    cudaFree(h->sf);
+    cudaFree(h->partials);
+    cudaFree(h->counters);
+    cudaFree(h->err);
+    cudaFree(h->stage);
+    delete h;
+    return rc;
+}
+
+int mxgemm_repack(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const uint8_t *A_scales,
+                  const uint8_t *B_scales, void *stream)
+{
+    if (!h)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = check_shape(fmt, M, N, K);
+    if (rc == MXGEMM_OK)
+        rc = check_ptrs({A_scales, B_scales});
+    if (rc == MXGEMM_OK)
+        rc = enter_device(h);
+    if (rc != MXGEMM_OK)
+        return rc;
+    return do_repack(h, fmt, M, N, K, A_scales, B_scales, static_cast<cudaStream_t>(stream));
+}
+
+int mxgemm_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const void *B, void *C,
+                void *stream)
+{
+    if (!h)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = check_shape(fmt, M, N, K);
+    if (rc == MXGEMM_OK)
+        rc = check_ptrs({A, B, C});
+    if (rc == MXGEMM_OK)
+        rc = enter_device(h);
+    if (rc != MXGEMM_OK)
+        return rc;
+    return do_gemm(h, fmt, M, N, K, A, B, C, static_cast<cudaStream_t>(stream));
+}
+
+int mxgemm_run(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const uint8_t *A_scales,
+               const void *B, const uint8_t *B_scales, void *C, void *stream)
+{
+    if (!h)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = check_shape(fmt, M, N, K);
+    if (rc == MXGEMM_OK)
+        rc = check_ptrs({A, A_scales, B, B_scales, C});
+    if (rc == MXGEMM_OK)
+        rc = enter_device(h);
+    if (rc != MXGEMM_OK)
+        return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = do_repack(h, fmt, M, N, K, A_scales, B_scales, st);
+    if (rc != MXGEMM_OK)
+        return rc;
+    return do_gemm(h, fmt, M, N, K, A, B, C, st);
+}
+
+int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A_host,
+                    const uint8_t *A_scales_host, const void *B_host, const uint8_t *B_scales_host, void *C_host,
+                    void *stream)
+{
+    if (!h)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = check_shape(fmt, M, N, K);
+    if (rc == MXGEMM_OK && (!A_host || !A_scales_host || !B_host || !B_scales_host || !C_host))
+        rc = MXGEMM_ERR_INVALID_ARG;
+    if (rc == MXGEMM_OK)
+        rc = enter_device(h);
+    if (rc != MXGEMM_OK)
+        return rc;
+    auto up16 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    const size_t rbytes = static_cast<size_t>(mxg::row_bytes(fmt, K));
+    const size_t nA = static_cast<size_t>(M) * rbytes, nB = static_cast<size_t>(N) * rbytes;
+    const size_t nSA = static_cast<size_t>(M) * static_cast<size_t>(K / 32);
+    const size_t nSB = static_cast<size_t>(N) * static_cast<size_t>(K / 32);
+    const size_t nC = static_cast<size_t>(M) * static_cast<size_t>(N) * 2;
+    const size_t oA = 0, oSA = oA + up16(nA), oB = oSA + up16(nSA), oSB = oB + up16(nB), oC = oSB + up16(nSB);
+    rc = grow(&h->stage, &h->stage_cap, oC + up16(nC), false);
+    if (rc != MXGEMM_OK)
+        return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *d = h->stage;
+    if (cudaMemcpyAsync(d + oA, A_host, nA, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(d + oSA, A_scales_host, nSA, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(d + oB, B_host, nB, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(d + oSB, B_scales_host, nSB, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    rc = do_repack(h, fmt, M, N, K, d + oSA, d + oSB, st);
+    if (rc != MXGEMM_OK)
+        return rc;
+    rc = do_gemm(h, fmt, M, N, K, d + oA, d + oB, d + oC, st);
+    if (rc != MXGEMM_OK)
+        return rc;
+    if (cudaMemcpyAsync(C_host, d + oC, nC, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    return MXGEMM_OK;
+}
+
+int mxgemm_quantize(int fmt, int64_t R, int64_t K, const float *X, void *Q, uint8_t *scales, void *stream)
+{
+    if (fmt != MXGEMM_FMT_MXFP8_E4M3 && fmt != MXGEMM_FMT_MXFP4_E2M1)
+        return MXGEMM_ERR_INVALID_ARG;
+    if (R < 1 || K < 32 || K % 32 != 0 || R > kMaxDim || K > kMaxDim)
+        return MXGEMM_ERR_INVALID_ARG;
+    if (!X || !Q || !scales)
+        return MXGEMM_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(Q) || !aligned16(scales))
+        return MXGEMM_ERR_ALIGNMENT;
+    if (mxg::launch_quantize(fmt, R, K, X, static_cast<uint8_t *>(Q), scales, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    return MXGEMM_OK;
+}
+
+int mxgemm_set_schedule(mxgemm_handle h, int schedule, int splits, int workers)
+{
+    if (!h || schedule < MXGEMM_SCHED_AUTO || schedule > MXGEMM_SCHED_STREAMK || splits < 1 || workers < 0)
+        return MXGEMM_ERR_INVALID_ARG;
+    h->sched = schedule;
+    h->splits = splits;
+    h->workers = workers;
+    return MXGEMM_OK;
+}
+
+int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, char *buf, size_t cap)
+{
+    if (!h || !buf || cap == 0)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = check_shape(fmt, M, N, K);
+    if (rc != MXGEMM_OK)
+        return rc;
+    const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers);
+    static const char *names[] = {"auto", "dp", "splitk", "streamk"};
+    snprintf(buf, cap,
+             "fmt=%d swap=%d BN=%d stages=%d tiles=%lld kt=%lld workers=%lld grid=%d sched=%s partial_bytes=%lld",
+             pl.fmt, pl.swap, pl.bn, pl.stages, static_cast<long long>(pl.tiles), static_cast<long long>(pl.kt),
+             static_cast<long long>(pl.workers), pl.grid, names[pl.sched & 3],
+             static_cast<long long>(pl.partial_bytes));
+    return MXGEMM_OK;
+}
+
+int mxgemm_check_device_error(mxgemm_handle h, int *code)
+{
+    if (!h || !code)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = enter_device(h);
+    if (rc != MXGEMM_OK)
+        return rc;
+    int v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess || cudaMemcpy(&v, h->err, sizeof(int), cudaMemcpyDeviceToHost) !=
+                                                      cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    *code = v;
+    if (v != 0) {
+        // A CTA that gave up may have left split counters behind: clear them.
+        if (cudaMemset(h->err, 0, sizeof(int)) != cudaSuccess ||
+            (h->counters && cudaMemset(h->counters, 0, h->counters_cap) != cudaSuccess) ||
+            cudaDeviceSynchronize() != cudaSuccess)
+            return MXGEMM_ERR_CUDA;
+        return MXGEMM_ERR_TIMEOUT;
+    }
+    return MXGEMM_OK;
+}
+
+int mxgemm_set_wait_limit(mxgemm_handle h, uint64_t ns)
+{
+    if (!h)
+        return MXGEMM_ERR_INVALID_ARG;
+    h->limit_ns = ns == 0 ? kDefaultLimitNs : ns;
+    return MXGEMM_OK;
+}
+
+int mxgemm_debug_inject(mxgemm_handle h, int mode)
+{
+    if (!h || mode < 0 || mode > 1)
+        return MXGEMM_ERR_INVALID_ARG;
+    h->inject = mode;
+    return MXGEMM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,82 @@
+// mx_internal.h -- declarations shared by the library's translation units
+// (not part of the public C ABI, which is include/mxgemm.h).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mxg {
+
+constexpr int kFmtMXFP8 = 0;
+constexpr int kFmtMXFP4 = 1;
+
+// Bytes of one operand row of K elements.
+inline int64_t row_bytes(int fmt, int64_t K) { return fmt == kFmtMXFP8 ? K : K / 2; }
+
+// 512-byte scale atoms per 128-row block per pipeline stage (a stage spans
+// 128 bytes of K: 128 E4M3 elements = 4 scale blocks, or 256 E2M1 elements
+// = 8 scale blocks).
+inline int atoms_per_stage(int fmt) { return fmt == kFmtMXFP8 ? 1 : 2; }
+
+// Repacked scale layout of one operand with R rows: [ceil(R/256)*2][ka][512]
+// (row blocks of 128, padded to an even count so a 256-row tile never reads
+// past the end), ka = atoms per 128-row block (K/128 rounded up to whole
+// stages).  Inside a
+// 512-byte atom the scale of row r (0..127) and block j (0..3) sits at byte
+// (r % 32) * 16 + (r / 32) * 4 + j: the layout tcgen05.cp .32x128b.warpx4
+// expects for block-scale factors.
+inline int64_t sf_atoms_per_rowblock(int fmt, int64_t K)
+{
+    const int64_t a = K / 128, s = atoms_per_stage(fmt);
+    return (a + s - 1) / s * s;
+}
+inline int64_t sf_repacked_bytes(int fmt, int64_t R, int64_t K)
+{
+    return (R + 255) / 256 * 2 * sf_atoms_per_rowblock(fmt, K) * 512;
+}
+
+// Launch the repack of both operands' scales (one kernel launch).
+cudaError_t launch_repack(int fmt, int64_t M, int64_t N, int64_t K, const uint8_t *sa, const uint8_t *sb,
+                          uint8_t *sa_out, uint8_t *sb_out, cudaStream_t stream);
+
+// Launch the OCP MX quantiser.
+cudaError_t launch_quantize(int fmt, int64_t R, int64_t K, const float *X, uint8_t *Q, uint8_t *S,
+                            cudaStream_t stream);
+
+// Scheduling plan of one GEMM.
+struct GemmPlan {
+    int fmt = 0;
+    int swap = 0;          // 1: MMA rows come from B (C^T = B * A^T)
+    int bn = 0;            // MMA N (columns of one output tile)
+    int stages = 0;
+    int64_t M = 0, N = 0, K = 0;
+    int64_t P = 0, Q = 0;  // rows of the MMA's row operand / column operand
+    int64_t tilesP = 0, tilesQ = 0, kt = 0, tiles = 0, iters = 0;
+    int64_t workers = 0;
+    int grid = 0;
+    int sched = 0;         // resolved schedule (MXGEMM_SCHED_*)
+    int64_t kaP = 0, kaQ = 0;
+    int64_t partial_bytes = 0;  // workspace for split partials
+    int64_t counter_bytes = 0;
+};
+
+// Build the plan for a shape.  sched/splits/workers as mxgemm_set_schedule.
+GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sched, int splits,
+                   int workers);
+
+// Launch the GEMM kernel for `plan`.
+struct GemmBuffers {
+    const void *A, *B;
+    const uint8_t *sfA, *sfB;   // repacked scales of A and of B
+    void *C;
+    float *partials;
+    uint32_t *counters;
+    int *error;
+};
+cudaError_t launch_gemm(const GemmPlan &plan, const GemmBuffers &buf, uint64_t wait_limit_ns, int inject,
+                        cudaStream_t stream);
+
+// Per-(fmt, BN) kernel attribute setup; returns cudaSuccess once done.
+cudaError_t prepare_gemm_kernels();
+
+}  // namespace mxg

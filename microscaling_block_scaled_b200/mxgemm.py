@@ -1,0 +1,227 @@
+"""Python binding of ``libmxgemm.so`` (ctypes; argument marshalling only).
+
+Every function named ``mxgemm_*`` here calls the C entry point of the same
+name declared in ``include/mxgemm.h``; the ``Handle`` class and the
+``quantize`` / ``run`` helpers only turn torch tensors into pointers, sizes
+and the current CUDA stream.  There is no fallback: if the shared library is
+missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmxgemm.so")
+
+FMT_MXFP8 = 0
+FMT_MXFP4 = 1
+FMT_NAMES = {"mxfp8": FMT_MXFP8, "mxfp4": FMT_MXFP4}
+
+SCHED_AUTO, SCHED_DP, SCHED_SPLITK, SCHED_STREAMK = 0, 1, 2, 3
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_ALIGNMENT = 2
+ERR_UNSUPPORTED_DEVICE = 3
+ERR_OOM = 4
+ERR_CUDA = 5
+ERR_TIMEOUT = 6
+
+# Entry points and their C signatures (restype, argtypes).
+_i64 = ctypes.c_int64
+_vp = ctypes.c_void_p
+SIGNATURES = {
+    "mxgemm_create": (ctypes.c_int, [ctypes.POINTER(_vp)]),
+    "mxgemm_destroy": (ctypes.c_int, [_vp]),
+    "mxgemm_run": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "mxgemm_repack": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "mxgemm_gemm": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "mxgemm_run_host": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "mxgemm_quantize": (ctypes.c_int, [ctypes.c_int, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "mxgemm_set_schedule": (ctypes.c_int, [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "mxgemm_describe_plan": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, ctypes.c_char_p, ctypes.c_size_t]),
+    "mxgemm_check_device_error": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_int)]),
+    "mxgemm_set_wait_limit": (ctypes.c_int, [_vp, ctypes.c_uint64]),
+    "mxgemm_debug_inject": (ctypes.c_int, [_vp, ctypes.c_int]),
+    "mxgemm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "mxgemm_version": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+class MXGemmError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__("%s failed: %s (status %d)" % (fn, status_string(status), status))
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError("libmxgemm.so not found at %s: run `python -m microscaling_block_scaled_b200.build`"
+                               % path)
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().mxgemm_status_string(status).decode()
+
+
+def version() -> str:
+    return load().mxgemm_version().decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != OK:
+        raise MXGemmError(fn, status)
+
+
+def row_bytes(fmt: int, K: int) -> int:
+    return K if fmt == FMT_MXFP8 else K // 2
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _ptr(t) -> int:
+    return int(t.data_ptr())
+
+
+# ------------------------------------------------------------- raw calls
+
+def mxgemm_create() -> int:
+    h = _vp()
+    _check("mxgemm_create", load().mxgemm_create(ctypes.byref(h)))
+    return h.value
+
+
+def mxgemm_destroy(h: int) -> None:
+    _check("mxgemm_destroy", load().mxgemm_destroy(h))
+
+
+def mxgemm_run(h, fmt, M, N, K, A, SA, B, SB, C, stream) -> int:
+    return load().mxgemm_run(h, fmt, M, N, K, A, SA, B, SB, C, stream)
+
+
+def mxgemm_repack(h, fmt, M, N, K, SA, SB, stream) -> int:
+    return load().mxgemm_repack(h, fmt, M, N, K, SA, SB, stream)
+
+
+def mxgemm_gemm(h, fmt, M, N, K, A, B, C, stream) -> int:
+    return load().mxgemm_gemm(h, fmt, M, N, K, A, B, C, stream)
+
+
+def mxgemm_run_host(h, fmt, M, N, K, A, SA, B, SB, C, stream) -> int:
+    return load().mxgemm_run_host(h, fmt, M, N, K, A, SA, B, SB, C, stream)
+
+
+def mxgemm_quantize(fmt, R, K, X, Q, S, stream) -> int:
+    return load().mxgemm_quantize(fmt, R, K, X, Q, S, stream)
+
+
+def mxgemm_set_schedule(h, schedule, splits=1, workers=0) -> int:
+    return load().mxgemm_set_schedule(h, schedule, splits, workers)
+
+
+def mxgemm_describe_plan(h, fmt, M, N, K) -> str:
+    buf = ctypes.create_string_buffer(256)
+    _check("mxgemm_describe_plan", load().mxgemm_describe_plan(h, fmt, M, N, K, buf, 256))
+    return buf.value.decode()
+
+
+def mxgemm_check_device_error(h) -> tuple[int, int]:
+    code = ctypes.c_int(0)
+    st = load().mxgemm_check_device_error(h, ctypes.byref(code))
+    return st, code.value
+
+
+def mxgemm_set_wait_limit(h, ns: int) -> int:
+    return load().mxgemm_set_wait_limit(h, ns)
+
+
+def mxgemm_debug_inject(h, mode: int) -> int:
+    return load().mxgemm_debug_inject(h, mode)
+
+
+# ------------------------------------------------------- torch helpers
+
+def quantize(fmt: int, X, stream=None):
+    """OCP MX quantisation of an FP32 CUDA tensor [R][K] on the device.
+    Returns (codes uint8 [R][row_bytes], scales uint8 [R][K/32])."""
+    import torch
+    assert X.is_cuda and X.dtype == torch.float32 and X.is_contiguous()
+    R, K = X.shape
+    Q = torch.empty((R, row_bytes(fmt, K)), dtype=torch.uint8, device=X.device)
+    S = torch.empty((R, K // 32), dtype=torch.uint8, device=X.device)
+    _check("mxgemm_quantize", mxgemm_quantize(fmt, R, K, _ptr(X), _ptr(Q), _ptr(S), _stream_ptr(stream)))
+    return Q, S
+
+
+class Handle:
+    """Owns one ``mxgemm_handle`` (workspace, schedule) on the current device."""
+
+    def __init__(self):
+        self.h = mxgemm_create()
+
+    def close(self):
+        if self.h:
+            mxgemm_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def set_schedule(self, schedule: int, splits: int = 1, workers: int = 0):
+        _check("mxgemm_set_schedule", mxgemm_set_schedule(self.h, schedule, splits, workers))
+
+    def describe(self, fmt, M, N, K) -> str:
+        return mxgemm_describe_plan(self.h, fmt, M, N, K)
+
+    def run(self, fmt, A, SA, B, SB, C=None, K=None, stream=None):
+        """C = A * B^T for MX operands on the device; returns C (bfloat16 [M][N])."""
+        import torch
+        M, N = A.shape[0], B.shape[0]
+        if K is None:
+            K = SA.shape[1] * 32
+        if C is None:
+            C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+        _check("mxgemm_run", mxgemm_run(self.h, fmt, M, N, K, _ptr(A), _ptr(SA), _ptr(B), _ptr(SB), _ptr(C),
+                                        _stream_ptr(stream)))
+        return C
+
+    def repack(self, fmt, M, N, K, SA, SB, stream=None):
+        _check("mxgemm_repack", mxgemm_repack(self.h, fmt, M, N, K, _ptr(SA), _ptr(SB), _stream_ptr(stream)))
+
+    def gemm(self, fmt, M, N, K, A, B, C, stream=None):
+        _check("mxgemm_gemm", mxgemm_gemm(self.h, fmt, M, N, K, _ptr(A), _ptr(B), _ptr(C), _stream_ptr(stream)))
+
+    def run_host(self, fmt, M, N, K, A, SA, B, SB, C, stream=None):
+        """Host (CPU, ideally pinned) tensors in, C written to the host tensor ``C``."""
+        _check("mxgemm_run_host", mxgemm_run_host(self.h, fmt, M, N, K, _ptr(A), _ptr(SA), _ptr(B), _ptr(SB),
+                                                  _ptr(C), _stream_ptr(stream)))
+
+    def check_device_error(self) -> tuple[int, int]:
+        return mxgemm_check_device_error(self.h)
+
+    def set_wait_limit(self, ns: int):
+        _check("mxgemm_set_wait_limit", mxgemm_set_wait_limit(self.h, ns))
+
+    def debug_inject(self, mode: int):
+        _check("mxgemm_debug_inject", mxgemm_debug_inject(self.h, mode))

@@ -1,0 +1,251 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Pass rule per element: |C_gpu - C_ref| <= 1 BF16 ulp(C_ref) + 2^-18 * sum_k |a_k b_k|
+with identical NaN / +-Inf positions; quantised codes and scales must agree
+bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from microscaling_block_scaled_b200 import mxgemm, synth
+
+from gpu_util import assert_parity, bits, full_case, handle, sampled_case
+
+pytestmark = pytest.mark.gpu
+
+F8, F4 = mxgemm.FMT_MXFP8, mxgemm.FMT_MXFP4
+
+
+# ------------------------------------------------------------- quantiser
+
+@pytest.mark.parametrize("fmt", [F8, F4])
+@pytest.mark.parametrize("kind", ["normal", "heavy"])
+def test_quantiser_bit_exact(fmt, kind):
+    A32, _ = synth.operands(96, 1, 2048, seed=21, kind=kind)
+    q, s = mxgemm.quantize(fmt, A32.cuda())
+    oq, os_ = oracle.quantize(fmt, A32.numpy())
+    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(q.cpu().numpy(), oq)
+
+
+@pytest.mark.parametrize("fmt", [F8, F4])
+def test_quantiser_edge_blocks_bit_exact(fmt):
+    emax = 8 if fmt == F8 else 2
+    rows = []
+    r = np.zeros(32 * 12, dtype=np.float32)
+    r[32:64] = -0.0                                  # negative zeros
+    r[64] = np.float32(2.0 ** -140)                  # FP32 subnormal amax
+    r[65] = -np.float32(2.0 ** -145)
+    r[96:128] = np.nan                               # NaN block
+    r[128] = np.inf                                  # Inf block
+    r[160] = 1000.0                                  # saturation
+    r[161] = -930.0
+    # ties in the scaled domain (scale 2^0 when amax is in [2^emax, 2^(emax+1)))
+    r[192] = 2.0 ** emax
+    if fmt == F8:
+        r[193:200] = [1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10, 15.5 * 2.0 ** -7, -1.0625, 460.0 / 2]
+    else:
+        r[193:200] = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, -5.0]
+    r[224] = np.float32(3.0e38)                      # near FP32 max
+    r[225] = np.float32(-1.0e-38)
+    r[256] = np.float32(2.0 ** -126) * 1.5           # smallest normal binade amax
+    r[288:320] = np.linspace(-7.0, 7.0, 32, dtype=np.float32)
+    r[320:352] = np.float32(2.0 ** -149)             # smallest subnormal
+    rows.append(r)
+    X = np.stack(rows + [np.random.default_rng(3).standard_normal(r.shape).astype(np.float32)])
+    q, s = mxgemm.quantize(fmt, torch.from_numpy(X).cuda())
+    oq, os_ = oracle.quantize(fmt, X)
+    assert np.array_equal(s.cpu().numpy(), os_), (s.cpu().numpy(), os_)
+    assert np.array_equal(q.cpu().numpy(), oq), np.argwhere(q.cpu().numpy() != oq)[:8]
+
+
+# ------------------------------------------------------ full comparisons
+
+SMALL = [
+    (1, 8, 128), (16, 256, 128), (32, 256, 512), (33, 100, 384), (48, 200, 256), (64, 136, 256),
+    (65, 128, 128), (100, 300, 256), (128, 128, 512), (200, 264, 640), (256, 512, 256), (130, 1000, 1152),
+]
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("M,N,K", SMALL)
+def test_gemm_small_full(fmt, M, N, K):
+    full_case(fmt, M, N, K, seed=M * 7 + N + K)
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("M,N,K", [(32, 512, 1024), (300, 384, 768)])
+def test_gemm_heavy_tails_full(fmt, M, N, K):
+    full_case(fmt, M, N, K, seed=4, kind="heavy")
+
+
+def test_config_mxfp8_32x256x512_full():
+    full_case(F8, 32, 256, 512, seed=0)
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("sched", [
+    (mxgemm.SCHED_DP, 1, 0), (mxgemm.SCHED_SPLITK, 3, 0), (mxgemm.SCHED_SPLITK, 8, 0),
+    (mxgemm.SCHED_STREAMK, 1, 0), (mxgemm.SCHED_STREAMK, 1, 7), (mxgemm.SCHED_STREAMK, 1, 37),
+])
+@pytest.mark.parametrize("M,N,K", [(64, 1024, 2048), (200, 640, 1536)])
+def test_gemm_forced_schedules(fmt, sched, M, N, K):
+    full_case(fmt, M, N, K, seed=9, schedule=sched)
+
+
+# ----------------------------------------------------------- edge cases
+
+def _codes_case(fmt, A, SA, B, SB, K):
+    h = handle()
+    ta = torch.from_numpy(A).cuda()
+    tb = torch.from_numpy(B).cuda()
+    tsa = torch.from_numpy(SA).cuda()
+    tsb = torch.from_numpy(SB).cuda()
+    C = h.run(fmt, ta, tsa, tb, tsb, K=K)
+    torch.cuda.synchronize()
+    ref, _, mag = oracle.gemm(fmt, K, A, SA, B, SB)
+    return bits(C), ref, mag
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+def test_gemm_nan_scales_and_zero_blocks(fmt):
+    rng = np.random.default_rng(17)
+    M, N, K = 70, 160, 384
+    rb = oracle.row_bytes(fmt, K)
+    A = rng.integers(0, 256, (M, rb), dtype=np.uint8)
+    B = rng.integers(0, 256, (N, rb), dtype=np.uint8)
+    if fmt == F8:
+        A[(A & 0x7F) == 0x7F] = 0x35
+        B[(B & 0x7F) == 0x7F] = 0x4A
+    SA = rng.integers(110, 140, (M, K // 32), dtype=np.uint8)
+    SB = rng.integers(110, 140, (N, K // 32), dtype=np.uint8)
+    SA[3, 5] = 0xFF                        # NaN scale in A: row 3 all NaN
+    SB[7, 0] = 0xFF                        # NaN scale in B: column 7 all NaN
+    blk = 32 * rb // K
+    A[10, 2 * blk:3 * blk] = 0             # an all-zero block
+    B[20, :] = 0                           # an all-zero column
+    got, ref, mag = _codes_case(fmt, A, SA, B, SB, K)
+    assert_parity(got, ref, mag, "nan scales")
+    gv = oracle.bf16_bits_to_f64(got)
+    assert np.isnan(gv[3]).all() and np.isnan(gv[:, 7]).all()
+    assert (gv[np.arange(M) != 3, 20] == 0).all()
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+def test_gemm_overflow_and_underflow_scales(fmt):
+    """Positive elements (no cancellation) with extreme scales: 2^127 * 2^127
+    overflows BF16 to +Inf, 2^-95 * 2^-95 underflows to 0, mixed pairs give
+    normal results."""
+    rng = np.random.default_rng(23)
+    M, N, K = 130, 140, 256
+    if fmt == F8:
+        A = rng.integers(0x08, 0x7F, (M, K), dtype=np.uint8)
+        B = rng.integers(0x08, 0x7F, (N, K), dtype=np.uint8)
+    else:
+        na = rng.integers(1, 8, (M, K), dtype=np.uint8)
+        nb = rng.integers(1, 8, (N, K), dtype=np.uint8)
+        A = (na[:, 0::2] | (na[:, 1::2] << 4)).astype(np.uint8)
+        B = (nb[:, 0::2] | (nb[:, 1::2] << 4)).astype(np.uint8)
+    SA = np.full((M, K // 32), 0x7F, np.uint8)
+    SB = np.full((N, K // 32), 0x7F, np.uint8)
+    SA[5, :] = 0xFE
+    SA[6, :] = 0x20
+    SB[9, :] = 0xFE
+    SB[10, :] = 0x20
+    got, ref, mag = _codes_case(fmt, A, SA, B, SB, K)
+    assert_parity(got, ref, mag, "extreme scales")
+    gv = oracle.bf16_bits_to_f64(got)
+    assert np.isposinf(gv[5, 9]) and np.isposinf(gv[5, 0]) and gv[6, 10] == 0.0
+    assert np.isfinite(gv[5, 10]) and gv[5, 10] > 0
+
+
+def test_gemm_nan_elements_e4m3():
+    rng = np.random.default_rng(5)
+    M, N, K = 40, 72, 256
+    A = rng.integers(0, 0x70, (M, K), dtype=np.uint8)
+    B = rng.integers(0, 0x70, (N, K), dtype=np.uint8)
+    A[5, 17] = 0x7F                        # E4M3 NaN element
+    B[9, 200] = 0xFF
+    SA = np.full((M, K // 32), 0x7F, np.uint8)
+    SB = np.full((N, K // 32), 0x7F, np.uint8)
+    got, ref, mag = _codes_case(F8, A, SA, B, SB, K)
+    assert_parity(got, ref, mag, "nan elements")
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+def test_gemm_integer_exact(fmt):
+    """All scales 1 and small integer elements: every output is an exact
+    integer (a textbook integer matmul) and must match exactly."""
+    rng = np.random.default_rng(8)
+    M, N, K = 96, 200, 512
+    vals = np.arange(-16, 17) if fmt == F8 else np.array([0, 1, 2, 3, 4, 6, -1, -2, -3, -4, -6])
+    ai = rng.choice(vals, (M, K))
+    bi = rng.choice(vals, (N, K))
+    enc = oracle.encode_e4m3 if fmt == F8 else oracle.encode_e2m1
+    table = {int(v): enc(float(v)) for v in vals}
+    ea = np.vectorize(table.get)(ai).astype(np.uint8)
+    eb = np.vectorize(table.get)(bi).astype(np.uint8)
+    if fmt == F4:
+        ea = (ea[:, 0::2] | (ea[:, 1::2] << 4)).astype(np.uint8)
+        eb = (eb[:, 0::2] | (eb[:, 1::2] << 4)).astype(np.uint8)
+    S1 = np.full((M, K // 32), 0x7F, np.uint8)
+    S2 = np.full((N, K // 32), 0x7F, np.uint8)
+    got, ref, mag = _codes_case(fmt, ea, S1, eb, S2, K)
+    exact = ai.astype(np.int64) @ bi.astype(np.int64).T
+    small = np.abs(exact) <= 256           # exactly representable in BF16
+    assert np.array_equal(oracle.bf16_bits_to_f64(got)[small], exact[small].astype(np.float64))
+    assert_parity(got, ref, mag, "integer")
+
+
+# -------------------------------------------------------- entry points
+
+def test_repack_then_gemm_equals_run_and_host_path():
+    fmt, M, N, K = F4, 48, 512, 1024
+    A32, B32 = synth.operands(M, N, K, seed=31)
+    qa, sa = mxgemm.quantize(fmt, A32.cuda())
+    qb, sb = mxgemm.quantize(fmt, B32.cuda())
+    h = handle()
+    C1 = h.run(fmt, qa, sa, qb, sb, K=K)
+    C2 = torch.empty_like(C1)
+    h.repack(fmt, M, N, K, sa, sb)
+    h.gemm(fmt, M, N, K, qa, qb, C2)
+    C3 = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    h.run_host(fmt, M, N, K, qa.cpu().pin_memory(), sa.cpu().pin_memory(), qb.cpu().pin_memory(),
+               sb.cpu().pin_memory(), C3)
+    torch.cuda.synchronize()
+    assert torch.equal(C1.view(torch.int16), C2.view(torch.int16))
+    assert torch.equal(C1.view(torch.int16).cpu(), C3.view(torch.int16))
+
+
+def test_gemm_rejects_shape_not_repacked():
+    h = handle()
+    t = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    st = mxgemm.mxgemm_repack(h.h, F8, 4, 4, 128, t.data_ptr(), t.data_ptr(), 0)
+    assert st == mxgemm.OK
+    st = mxgemm.mxgemm_gemm(h.h, F8, 4, 8, 128, t.data_ptr(), t.data_ptr(), t.data_ptr(), 0)
+    assert st == mxgemm.ERR_INVALID_ARG
+    st = mxgemm.mxgemm_run(h.h, F8, 4, 4, 100, t.data_ptr(), t.data_ptr(), t.data_ptr(), t.data_ptr(),
+                           t.data_ptr(), 0)
+    assert st == mxgemm.ERR_INVALID_ARG
+    st = mxgemm.mxgemm_run(h.h, F8, 4, 4, 128, t.data_ptr() + 8, t.data_ptr(), t.data_ptr(), t.data_ptr(),
+                           t.data_ptr(), 0)
+    assert st == mxgemm.ERR_ALIGNMENT
+
+
+# ----------------------------------------------- the pages' workloads
+
+@pytest.mark.parametrize("fmt,M,N,K,seed", [
+    (F4, 32, 14336, 4096, 1),
+    (F8, 64, 4096, 4096, 2),
+    (F4, 64, 4096, 4096, 2),
+])
+def test_decode_workloads_sampled(fmt, M, N, K, seed):
+    sampled_case(fmt, M, N, K, seed, n_rows=M, n_cols=1024)
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("M,N,K", [(2048, 28672, 8192), (8192, 8192, 8192), (4096, 4096, 14336)])
+def test_prefill_workloads_sampled(fmt, M, N, K):
+    sampled_case(fmt, M, N, K, seed=3, n_rows=96, n_cols=96)

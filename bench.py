@@ -1,0 +1,439 @@
+"""Benchmark of the MX block-scaled GEMM hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the hot path over one batch of pre-quantised inputs:
+the scale repack and the block-scaled GEMM (``mxgemm_run``: two kernel
+launches).  Quantisation is input generation and stays outside the timed
+region, as in the pages' methodology (devotd.net section 2: measurements
+start from already-quantised inputs).
+
+Timing: W eager warm-up steps, then the K timed steps are replayed from one
+CUDA graph bracketed by a barrier + synchronize and CUDA events on the launch
+stream.  Inputs rotate over enough copies that the bytes touched between two
+uses of a copy exceed twice the L2 size, so every step streams from HBM.
+Multi-GPU runs are replicas (the workload does not shard): every rank runs
+the full workload, time is the max over ranks and ``value`` the total work of
+all ranks divided by it.
+
+The ``reference`` arm times the CPU oracle (test infrastructure) on a bounded
+sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MX scaled-GEMM TFLOPS (MXFP8/MXFP4, NT) and % of roofline on 1 B200"
+DEFAULT_WORKLOAD = "mxfp4_32x14336x4096"
+KERNEL_SOURCES = ["microscaling_block_scaled_b200/csrc/gemm.cu", "microscaling_block_scaled_b200/csrc/sm100_ptx.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    return ap.parse_args()
+
+
+def workload(name):
+    from microscaling_block_scaled_b200 import synth
+    if name not in synth.WORKLOADS:
+        raise SystemExit("unknown workload %s; one of %s" % (name, sorted(synth.WORKLOADS)))
+    fmt_name, M, N, K, seed, kind = synth.WORKLOADS[name]
+    return fmt_name, M, N, K, seed, kind
+
+
+def flops(M, N, K):
+    return 2.0 * M * N * K
+
+
+def algorithmic_bytes(fmt, M, N, K):
+    """A + B + both scale arrays read once, C written once (BF16)."""
+    rb = K if fmt == 0 else K // 2
+    return M * rb + N * rb + (M + N) * (K // 32) + 2 * M * N
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
+    taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload_name)
+    if not e or e.get("kernel_hash") != kernel_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML in a thread."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index, period=0.002):
+        self.samples = []
+        self.period = period
+        self.active = False
+        self._stop = False
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self.t = threading.Thread(target=self._loop, daemon=True)
+
+    def _loop(self):
+        while not self._stop:
+            if self.active and self.ok:
+                try:
+                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                    rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((mhz, rs))
+                except Exception:
+                    pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop = True
+        self.t.join(timeout=1)
+
+    def summary(self):
+        if not self.samples:
+            if self.ok:   # region too short for the thread: one sample right now
+                try:
+                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                    rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((mhz, rs))
+                except Exception:
+                    pass
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = set()
+        for _, rs in self.samples:
+            for k, bit in self.REASONS.items():
+                if rs & bit and k != "gpu_idle":
+                    reasons.add(k)
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- CPU arm
+
+class OracleSampler:
+    """Times the CPU oracle (as it stands) on a bounded sample of C: a block of
+    sampled rows of A against a block of sampled rows of B, sized so one call
+    takes about ``target_s`` seconds.  The sampled operand rows are quantised by
+    the oracle's own quantiser once, outside the timing."""
+
+    def __init__(self, fmt, M, N, K, A32, B32, seed=99):
+        import numpy as np
+        import torch
+
+        import oracle
+        self.oracle = oracle
+        self.fmt, self.M, self.N, self.K = fmt, M, N, K
+        rng = np.random.default_rng(seed)
+        self.nm = min(M, 16)
+        rm = np.sort(rng.choice(M, self.nm, replace=False))
+        a = A32[torch.from_numpy(rm).to(A32.device)].float().cpu().numpy()
+        self.oa, self.osa = oracle.quantize(fmt, a)
+        self.pool = min(N, 4096)
+        rn = np.sort(rng.choice(N, self.pool, replace=False))
+        b = B32[torch.from_numpy(rn).to(B32.device)].float().cpu().numpy()
+        self.ob, self.osb = oracle.quantize(fmt, b)
+        t0 = time.perf_counter()
+        nn0 = min(self.pool, 32)
+        oracle.gemm(fmt, K, self.oa, self.osa, self.ob[:nn0], self.osb[:nn0])
+        self.sec_per_col = max(time.perf_counter() - t0, 1e-5) / nn0
+
+    def run(self, target_s):
+        nn = int(min(self.pool, max(8, target_s / self.sec_per_col)))
+        t0 = time.perf_counter()
+        self.oracle.gemm(self.fmt, self.K, self.oa, self.osa, self.ob[:nn], self.osb[:nn])
+        dt = time.perf_counter() - t0
+        tflops = flops(self.nm, nn, self.K) / dt / 1e12
+        desc = "C[%d sampled rows][%d sampled cols] of the %dx%dx%d product (%.3g GFLOP)" % (
+            self.nm, nn, self.M, self.N, self.K, flops(self.nm, nn, self.K) / 1e9)
+        return tflops, dt, self.oracle.num_threads(), desc
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from microscaling_block_scaled_b200 import synth
+    fmt_name, M, N, K, seed, kind = workload(args.workload)
+    fmt = 0 if fmt_name == "mxfp8" else 1
+    # the whole run stays within a few minutes: split the budget over the steps
+    per_step = max(0.05, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
+    A32, B32 = synth.operands(M, N, K, seed=seed, kind=kind, device="cpu")
+    sampler = OracleSampler(fmt, M, N, K, A32, B32)
+    times, vals = [], []
+    desc = cores = None
+    for i in range(args.warmup + args.steps):
+        v, dt, cores, desc = sampler.run(per_step)
+        if i >= args.warmup:
+            times.append(dt)
+            vals.append(v)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(times) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": fmt_name,
+        "data": "synthetic",
+        "config": {"workload": args.workload, "fmt": fmt_name, "M": M, "N": N, "K": K, "seed": seed,
+                   "inputs": kind},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from microscaling_block_scaled_b200 import mxgemm, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    fmt_name, M, N, K, seed, kind = workload(args.workload)
+    fmt = mxgemm.FMT_NAMES[fmt_name]
+    A32, B32 = synth.operands(M, N, K, seed=seed, kind=kind, device=dev)
+    qa, sa = mxgemm.quantize(fmt, A32)
+    qb, sb = mxgemm.quantize(fmt, B32)
+    torch.cuda.synchronize()
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    set_bytes = algorithmic_bytes(fmt, M, N, K)
+    nsets = max(2, math.ceil(2 * l2 / set_bytes) + 1)
+    sets = [(qa.clone(), sa.clone(), qb.clone(), sb.clone(), torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+            for _ in range(nsets)]
+    h = mxgemm.Handle()
+    plan = h.describe(fmt, M, N, K)
+
+    def step(i, stream=None):
+        a, s_a, b, s_b, c = sets[i % nsets]
+        h.run(fmt, a, s_a, b, s_b, C=c, K=K, stream=stream)
+
+    def gemm_only(i, stream=None):
+        a, _, b, _, c = sets[i % nsets]
+        h.gemm(fmt, M, N, K, a, b, c, stream=stream)
+
+    def repack_only(i, stream=None):
+        _, s_a, _, s_b, _ = sets[i % nsets]
+        h.repack(fmt, M, N, K, s_a, s_b, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    def capture(fn, n):
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            fn(0, s)                     # one eager call on the capture stream
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            for i in range(n):
+                fn(i, s)
+        torch.cuda.synchronize()
+        return g, s
+
+    def timed(g, s):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        launch = torch.cuda.current_stream()      # replay() launches on the current stream
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(launch)
+        g.replay()
+        e1.record(launch)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return e0.elapsed_time(e1)
+
+    g_step, s_step = capture(step, args.steps)
+    g_step.replay()                      # untimed replay (graph upload)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        clk.active = True
+        ms = timed(g_step, s_step)
+        clk.active = False
+    clocks = clk.summary()
+    g_gemm, s_gemm = capture(gemm_only, args.steps)
+    g_gemm.replay()
+    ms_gemm = timed(g_gemm, s_gemm)
+    g_rep, s_rep = capture(repack_only, args.steps)
+    g_rep.replay()
+    ms_rep = timed(g_rep, s_rep)
+    # graphs go before the process group
+    del g_step, g_gemm, g_rep
+    torch.cuda.synchronize()
+
+    if world > 1:
+        t = torch.tensor([ms, ms_gemm, ms_rep], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, ms_gemm, ms_rep = (float(x) for x in t.tolist())
+
+    ms_per_step = ms / args.steps
+    value = flops(M, N, K) * world * args.steps / (ms * 1e-3) / 1e12
+    gemm_us = ms_gemm / args.steps * 1e3
+    rep_us = ms_rep / args.steps * 1e3
+
+    # roofline of the dominant kernel (the GEMM)
+    peaks, peak_src = measured_peaks()
+    tc_peak = peaks["bf16_tflops"] * (2.0 if fmt == 0 else 4.0)      # dense MXFP8 = 2x, MXFP4 = 4x bf16
+    hbm = peaks["hbm_gbs"]
+    t_tc = flops(M, N, K) / (tc_peak * 1e12)
+    t_hbm = algorithmic_bytes(fmt, M, N, K) / (hbm * 1e9)
+    if t_hbm >= t_tc:
+        achieved = algorithmic_bytes(fmt, M, N, K) / (gemm_us * 1e-6) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm}
+    else:
+        achieved = flops(M, N, K) / (gemm_us * 1e-6) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": achieved / tc_peak}
+    tr = recorded_traffic(args.workload)
+    roof["traffic"] = tr
+    roof["peak_source"] = "%s (%s)" % (peak_src, "hbm_gbs" if roof["bound"] == "hbm" else
+                                       "bf16_tflops x %d (nominal MX/bf16 ratio)" % (2 if fmt == 0 else 4))
+    roof["kernel"] = "mx_gemm_kernel"
+    roof["algorithmic_bytes"] = algorithmic_bytes(fmt, M, N, K)
+    roof["flops"] = flops(M, N, K)
+
+    # end to end through the public host-buffer API
+    pa = qa.cpu().pin_memory()
+    psa = sa.cpu().pin_memory()
+    pb = qb.cpu().pin_memory()
+    psb = sb.cpu().pin_memory()
+    pc = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    st = torch.cuda.current_stream()
+    h.run_host(fmt, M, N, K, pa, psa, pb, psb, pc)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.e2e_steps):
+        h.run_host(fmt, M, N, K, pa, psa, pb, psb, pc)
+    e1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = flops(M, N, K) * world * args.e2e_steps / (e2e_ms * 1e-3) / 1e12
+    h2d = pa.numel() + psa.numel() + pb.numel() + psb.numel()
+    d2h = pc.numel() * 2
+
+    st_err, code = h.check_device_error()
+    if st_err != mxgemm.OK:
+        raise SystemExit("device error word set: %d" % code)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, cores, desc = OracleSampler(fmt, M, N, K, A32, B32).run(args.cpu_seconds)
+        cpu = {"value": v, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": desc, "seconds": dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": fmt_name, "data": "synthetic",
+            "config": {"workload": args.workload, "fmt": fmt_name, "M": M, "N": N, "K": K, "seed": seed,
+                       "inputs": "%s FP32 from torch CUDA generator, quantised on device (OCP MX), untimed" % kind,
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "l2": "inputs rotate over %d copies (%.1f MB each, %.0f MB > 2x L2 %.0f MB)" % (
+                           nsets, set_bytes / 1e6, nsets * set_bytes / 1e6, l2 / 1e6),
+                       "timing": "CUDA graph of K steps, CUDA events on the launch stream",
+                       "plan": plan, "gemm_us": gemm_us, "repack_us": rep_us,
+                       "gemm_tflops": flops(M, N, K) / (gemm_us * 1e-6) / 1e12},
+            "clocks": clocks,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "api": "mxgemm_run_host (pinned host buffers)", "steps": args.e2e_steps},
+            "gpu_launches": 2 * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -123,11 +123,13 @@ int do_repack(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const u
 }
 
 int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const void *B, void *C,
-            cudaStream_t st)
+            cudaStream_t st, int pdl)
 {
     if (h->last_fmt != fmt || h->last_M != M || h->last_N != N || h->last_K != K)
         return MXGEMM_ERR_INVALID_ARG;
     const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers);
+    if (!pl.valid)
+        return MXGEMM_ERR_INVALID_ARG;
     int rc = grow(&h->partials, &h->partials_cap, static_cast<size_t>(pl.partial_bytes > 0 ? pl.partial_bytes : 16),
                   false);
     if (rc != MXGEMM_OK)
@@ -146,7 +148,7 @@ int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const voi
     b.error = h->err;
     const int inject = h->inject;
     h->inject = 0;
-    if (mxg::launch_gemm(pl, b, h->limit_ns, inject, st) != cudaSuccess)
+    if (mxg::launch_gemm(pl, b, h->limit_ns, inject, pdl, st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
     return MXGEMM_OK;
 }
@@ -247,7 +249,7 @@ int mxgemm_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const
         rc = enter_device(h);
     if (rc != MXGEMM_OK)
         return rc;
-    return do_gemm(h, fmt, M, N, K, A, B, C, static_cast<cudaStream_t>(stream));
+    return do_gemm(h, fmt, M, N, K, A, B, C, static_cast<cudaStream_t>(stream), 0);
 }
 
 int mxgemm_run(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const uint8_t *A_scales,
@@ -266,7 +268,7 @@ int mxgemm_run(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const 
     rc = do_repack(h, fmt, M, N, K, A_scales, B_scales, st);
     if (rc != MXGEMM_OK)
         return rc;
-    return do_gemm(h, fmt, M, N, K, A, B, C, st);
+    return do_gemm(h, fmt, M, N, K, A, B, C, st, 1);
 }
 
 int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A_host,
@@ -302,7 +304,7 @@ int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
     rc = do_repack(h, fmt, M, N, K, d + oSA, d + oSB, st);
     if (rc != MXGEMM_OK)
         return rc;
-    rc = do_gemm(h, fmt, M, N, K, d + oA, d + oB, d + oC, st);
+    rc = do_gemm(h, fmt, M, N, K, d + oA, d + oB, d + oC, st, 1);
     if (rc != MXGEMM_OK)
         return rc;
     if (cudaMemcpyAsync(C_host, d + oC, nC, cudaMemcpyDeviceToHost, st) != cudaSuccess)

@@ -60,7 +60,9 @@ struct Cfg {
     static constexpr int kSFABytes = kAtoms * 512;
     static constexpr int kSFBBytes = kRBQ * kAtoms * 512;
     static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
-    static constexpr int kSmemBudget = 227 * 1024 - 2048;
+    static constexpr int kCW = BN < 32 ? BN : 32;             // accumulator columns per epilogue chunk
+    static constexpr int kOutBytes = 128 * kCW * 2;           // one BF16 output chunk
+    static constexpr int kSmemBudget = 227 * 1024 - 2048 - 2 * kOutBytes;
     static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
     static constexpr int kSFACols = kAtoms * 4;
@@ -76,7 +78,8 @@ struct Cfg {
     static constexpr int kOffB = kOffA + kStages * kABytes;
     static constexpr int kOffSFA = kOffB + kStages * kBBytes;
     static constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
-    static constexpr int kOffBar = kOffSFB + kStages * kSFBBytes;
+    static constexpr int kOffOut = (kOffSFB + kStages * kSFBBytes + 1023) / 1024 * 1024;
+    static constexpr int kOffBar = kOffOut + 2 * kOutBytes;
     static constexpr int kNumBars = 2 * kStages + 2 * kNumAcc + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 64 + 1024;   // + alignment slack
@@ -111,11 +114,13 @@ struct KParams {
     int *error;
     int64_t P, Q;          // valid rows of the two MMA operands
     int64_t ldc;           // = N
-    int64_t tilesP, kt, iters, workers;
+    uint32_t tilesP, kt, iters, workers;   // host guarantees iters * workers < 2^32
+    int dp;                // workers == tiles: worker w is exactly tile w
     int64_t kaP, kaQ;      // scale atoms per 128-row block
     uint64_t limit_ns;
     int swap;
     int inject;
+    int tma_store;         // 1: epilogue stores C through shared memory with TMA
 };
 
 // Error site codes written to the device error word.
@@ -133,13 +138,82 @@ __device__ __forceinline__ void record_error(int *err, int code, volatile int *a
     *abort_flag = 1;
 }
 
-// Which worker owns K-iteration i (largest g with floor(g*I/W) <= i).
-__device__ __forceinline__ int64_t worker_of(int64_t i, int64_t I, int64_t W)
-{
-    return ((i + 1) * W - 1) / I;
-}
+// Work decomposition shared by the three roles.  All index arithmetic is
+// 32-bit (64-bit integer division is a long software sequence on the GPU and
+// sat on the critical path of every hand-off); whole-tile schedules take a
+// division-free path.
+struct Sched {
+    uint32_t I, W, KT, tilesP;
+    bool dp;
+    // first K-iteration of worker g: floor(g * I / W)
+    __device__ __forceinline__ uint32_t begin(uint32_t g) const { return dp ? g * KT : (g * I) / W; }
+    // worker owning K-iteration i: the largest g with begin(g) <= i
+    __device__ __forceinline__ uint32_t owner(uint32_t i) const { return dp ? i / KT : ((i + 1) * W - 1) / I; }
+};
 
-__device__ __forceinline__ int64_t worker_begin(int64_t g, int64_t I, int64_t W) { return g * I / W; }
+// Walks the K-iterations of the workers a CTA owns (blockIdx.x, +gridDim.x,
+// ...) in order, tracking the tile and its K step incrementally.
+struct IterCursor {
+    Sched sc;
+    uint32_t w, step;
+    uint32_t it, end, tile, k;
+    __device__ __forceinline__ IterCursor(const Sched &sc_, uint32_t first, uint32_t step_)
+        : sc(sc_), w(first), step(step_), it(0), end(0), tile(0), k(0)
+    {
+        enter();
+    }
+    __device__ __forceinline__ void enter()
+    {
+        while (w < sc.W) {
+            it = sc.begin(w);
+            end = sc.begin(w + 1);
+            if (it < end)
+                break;
+            w += step;
+        }
+        if (w < sc.W) {
+            tile = sc.dp ? w : it / sc.KT;
+            k = it - tile * sc.KT;
+        }
+    }
+    __device__ __forceinline__ bool valid() const { return w < sc.W; }
+    __device__ __forceinline__ void advance()
+    {
+        ++it;
+        if (it >= end) {
+            w += step;
+            enter();
+            return;
+        }
+        if (++k == sc.KT) {
+            k = 0;
+            ++tile;
+        }
+    }
+    __device__ __forceinline__ uint32_t total() const
+    {
+        uint32_t n = 0;
+        for (uint32_t g = w; g < sc.W; g += step)
+            n += sc.begin(g + 1) - sc.begin(g);
+        return n;
+    }
+};
+
+// One maximal run of a worker's K-iterations inside one tile.
+struct Segment {
+    uint32_t tile, kb, ke, tp, tq;
+};
+
+__device__ __forceinline__ Segment segment_at(const Sched &sc, uint32_t it, uint32_t end)
+{
+    Segment g;
+    g.tile = it / sc.KT;
+    g.kb = it - g.tile * sc.KT;
+    g.ke = (g.kb + (end - it) < sc.KT) ? g.kb + (end - it) : sc.KT;
+    g.tq = g.tile / sc.tilesP;
+    g.tp = g.tile - g.tq * sc.tilesP;
+    return g;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
@@ -150,14 +224,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 // Store CW FP32 values as BF16 into C.  Non-swapped: thread's row p = C row,
 // values are C[p][q0 .. q0+CW).  Swapped: thread's row p = C column, values
 // are C[q0 .. q0+CW)[p].
+struct OutView {
+    __nv_bfloat16 *C;
+    int64_t ldc, P, Q;
+    int swap;
+};
+
 template <int CW>
-__device__ __forceinline__ void store_bf16(const KParams &kp, int64_t p, int64_t q0, const float (&v)[CW])
+__device__ __forceinline__ void store_bf16(const OutView o, int64_t p, int64_t q0, const float (&v)[CW])
 {
-    if (p >= kp.P)
+    if (p >= o.P)
         return;
-    if (!kp.swap) {
-        __nv_bfloat16 *dst = kp.C + p * kp.ldc + q0;
-        const int64_t nvalid = kp.Q - q0;
+    if (!o.swap) {
+        __nv_bfloat16 *dst = o.C + p * o.ldc + q0;
+        const int64_t nvalid = o.Q - q0;
         if (nvalid >= CW && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
 #pragma unroll
             for (int j = 0; j < CW / 8; ++j) {
@@ -178,8 +258,8 @@ __device__ __forceinline__ void store_bf16(const KParams &kp, int64_t p, int64_t
 #pragma unroll
         for (int j = 0; j < CW; ++j) {
             const int64_t q = q0 + j;
-            if (q < kp.Q)
-                kp.C[q * kp.ldc + p] = __float2bfloat16_rn(v[j]);
+            if (q < o.Q)
+                o.C[q * o.ldc + p] = __float2bfloat16_rn(v[j]);
         }
     }
 }
@@ -187,10 +267,17 @@ __device__ __forceinline__ void store_bf16(const KParams &kp, int64_t p, int64_t
 template <int FMT, int BN>
 __global__ void __launch_bounds__(192, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
-                   const KParams kp)
+                   const __grid_constant__ CUtensorMap tmC, const KParams kp_in)
 {
     using C_ = Cfg<FMT, BN>;
     constexpr int S = C_::kStages;
+    constexpr int CW = C_::kCW;
+
+    // Work on a register copy of the parameters: the inline-asm memory
+    // clobbers of the pipeline would otherwise force reloads from parameter
+    // space after each TMA / MMA / barrier instruction.
+    const KParams kp = kp_in;
+    const OutView out{kp.C, kp.ldc, kp.P, kp.Q, kp.swap};
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -210,6 +297,9 @@ __global__ void __launch_bounds__(192, 1)
     const int lane = threadIdx.x % 32;
 
     if (threadIdx.x == 0) {
+        tma_prefetch_desc(&tmP);
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmC);
         for (int s = 0; s < S; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
@@ -233,79 +323,91 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
 
-    const int64_t I = kp.iters, W = kp.workers, KT = kp.kt;
+    const Sched sc{kp.iters, kp.workers, kp.kt, kp.tilesP, kp.dp != 0};
+    const uint32_t W = sc.W;
+
+    // Everything except the producer's first operand loads may depend on the
+    // preceding kernel in the stream (the scale repack, or the previous GEMM
+    // that used the same workspace): wait for it here.  Without a
+    // programmatic launch this returns at once.
+    if (warp != 0)
+        grid_dependency_wait();
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            tma_prefetch_desc(&tmP);
-            tma_prefetch_desc(&tmQ);
-        }
         const uint64_t pol_stream = policy_evict_first();
-        int s = 0;
-        uint32_t ph = 0;
-        int64_t armed = 0;          // loads armed so far (round-robin over stages)
+        uint32_t armed = 0;         // stages armed so far (round-robin over the ring)
         int skipped_stage = -1;
         bool inject = kp.inject == 1;
         bool ok = true;
-        for (int64_t w = blockIdx.x; w < W && ok; w += gridDim.x) {
-            int64_t it = worker_begin(w, I, W);
-            const int64_t end = worker_begin(w + 1, I, W);
-            while (it < end && ok) {
-                const int64_t tile = it / KT;
-                const int64_t kb = it - tile * KT;
-                const int64_t ke = (kb + (end - it) < KT) ? kb + (end - it) : KT;
-                const int64_t tp = tile % kp.tilesP, tq = tile / kp.tilesP;
-                for (int64_t k = kb; k < ke; ++k) {
-                    int good = 1;
-                    if (lane == 0)
-                        good = mbar_wait_bounded(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns);
-                    good = __shfl_sync(0xffffffffu, good, 0);
-                    if (!good) {
-                        if (lane == 0)
-                            record_error(kp.error, kErrProducerEmpty, s_abort);
-                        ok = false;
-                        break;
-                    }
-                    if (lane == 0) {
-                        if (inject) {
-                            inject = false;          // leave this stage unarmed
-                            skipped_stage = s;
-                        } else {
-                            const uint32_t fb = full_bar(s);
-                            mbar_arrive_expect_tx(fb, C_::kTxBytes);
-                            const int32_t x = static_cast<int32_t>(k * C_::kStageKBytes);
-                            tma_load_2d(sbase + C_::kOffA + s * C_::kABytes, &tmP, x,
-                                        static_cast<int32_t>(tp * 128), fb, pol_stream);
-                            tma_load_2d(sbase + C_::kOffB + s * C_::kBBytes, &tmQ, x,
-                                        static_cast<int32_t>(tq * BN), fb, pol_stream);
-                            const uint8_t *sfa = kp.sfP + (tp * kp.kaP + k * C_::kAtoms) * 512;
-                            bulk_load(sbase + C_::kOffSFA + s * C_::kSFABytes, sfa, C_::kSFABytes, fb);
-                            const int64_t rb0 = (tq * BN) / 128;
+        auto load_operands = [&](int s, uint32_t tile, uint32_t k) {
+            const uint32_t tq = tile / sc.tilesP, tp = tile - tq * sc.tilesP;
+            const uint32_t fb = full_bar(s);
+            const int32_t x = static_cast<int32_t>(k * C_::kStageKBytes);
+            tma_load_2d(sbase + C_::kOffA + s * C_::kABytes, &tmP, x, static_cast<int32_t>(tp) * 128, fb,
+                        pol_stream);
+            tma_load_2d(sbase + C_::kOffB + s * C_::kBBytes, &tmQ, x, static_cast<int32_t>(tq) * BN, fb,
+                        pol_stream);
+        };
+        auto load_scales = [&](int s, uint32_t tile, uint32_t k) {
+            const uint32_t tq = tile / sc.tilesP, tp = tile - tq * sc.tilesP;
+            const uint32_t fb = full_bar(s);
+            const uint8_t *sfa = kp.sfP + (static_cast<int64_t>(tp) * kp.kaP + k * C_::kAtoms) * 512;
+            bulk_load(sbase + C_::kOffSFA + s * C_::kSFABytes, sfa, C_::kSFABytes, fb);
+            const int64_t rb0 = (static_cast<int64_t>(tq) * BN) / 128;
 #pragma unroll
-                            for (int rb = 0; rb < C_::kRBQ; ++rb) {
-                                const uint8_t *sfb = kp.sfQ + ((rb0 + rb) * kp.kaQ + k * C_::kAtoms) * 512;
-                                bulk_load(sbase + C_::kOffSFB + s * C_::kSFBBytes + rb * C_::kAtoms * 512, sfb,
-                                          C_::kAtoms * 512, fb);
-                            }
-                        }
-                        ++armed;
-                    }
-                    __syncwarp();
-                    if (++s == S) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
-                }
-                it += ke - kb;
+            for (int rb = 0; rb < C_::kRBQ; ++rb) {
+                const uint8_t *sfb = kp.sfQ + ((rb0 + rb) * kp.kaQ + k * C_::kAtoms) * 512;
+                bulk_load(sbase + C_::kOffSFB + s * C_::kSFBBytes + rb * C_::kAtoms * 512, sfb, C_::kAtoms * 512,
+                          fb);
             }
-        }
-        // Let every armed copy land before the CTA can exit: wait for the
-        // latest armed phase of each stage (already complete on the normal
-        // path, where the MMA warp consumed every stage).
+        };
         if (lane == 0) {
+            IterCursor cur(sc, blockIdx.x, gridDim.x);
+            const uint32_t n_total = cur.total();
+            const uint32_t n_pre = n_total < static_cast<uint32_t>(S) ? n_total : static_cast<uint32_t>(S);
+            // Pass 1: operand tiles of the first ring's worth of stages (the
+            // ring is empty, no wait needed); they do not depend on the
+            // preceding kernel.
+            for (uint32_t n = 0; n < n_pre; ++n, cur.advance()) {
+                const int s = static_cast<int>(n);
+                if (inject && n == 0) {
+                    skipped_stage = s;          // test hook: leave this stage unarmed
+                } else {
+                    mbar_arrive_expect_tx(full_bar(s), C_::kTxBytes);
+                    load_operands(s, cur.tile, cur.k);
+                }
+                ++armed;
+            }
+            grid_dependency_wait();
+            // Pass 2: the scales of those stages.
+            IterCursor cur2(sc, blockIdx.x, gridDim.x);
+            for (uint32_t n = 0; n < n_pre; ++n, cur2.advance())
+                if (static_cast<int>(n) != skipped_stage)
+                    load_scales(static_cast<int>(n), cur2.tile, cur2.k);
+            // Pass 3: the rest, one ring slot at a time.
+            int s = static_cast<int>(n_pre % S);
+            uint32_t ph = n_pre == static_cast<uint32_t>(S) ? 1u : 0u;
+            for (uint32_t n = n_pre; n < n_total; ++n, cur.advance()) {
+                if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns)) {
+                    record_error(kp.error, kErrProducerEmpty, s_abort);
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(full_bar(s), C_::kTxBytes);
+                load_operands(s, cur.tile, cur.k);
+                load_scales(s, cur.tile, cur.k);
+                ++armed;
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            // Let every armed copy land before the CTA can exit: wait for the
+            // latest armed phase of each stage (already complete on the normal
+            // path, where the MMA warp consumed every stage).
             for (int st = 0; st < S; ++st) {
-                const int64_t n = armed / S + (st < armed % S ? 1 : 0);
+                const uint32_t n = armed / S + (static_cast<uint32_t>(st) < armed % S ? 1u : 0u);
                 if (n == 0 || (st == skipped_stage && n == 1))
                     continue;
                 const uint32_t parity = static_cast<uint32_t>((n - 1) & 1);
@@ -313,6 +415,7 @@ __global__ void __launch_bounds__(192, 1)
                 if (!mbar_wait_bounded(full_bar(st), parity, &dummy_abort, kp.limit_ns))
                     atomicCAS(kp.error, 0, kErrDrain);
             }
+            (void)ok;
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -325,13 +428,12 @@ __global__ void __launch_bounds__(192, 1)
         int acc = 0;
         uint32_t acc_ph = 0;
         bool ok = true;
-        for (int64_t w = blockIdx.x; w < W && ok; w += gridDim.x) {
-            int64_t it = worker_begin(w, I, W);
-            const int64_t end = worker_begin(w + 1, I, W);
+        for (uint32_t w = blockIdx.x; w < W && ok; w += gridDim.x) {
+            uint32_t it = sc.begin(w);
+            const uint32_t end = sc.begin(w + 1);
             while (it < end && ok) {
-                const int64_t tile = it / KT;
-                const int64_t kb = it - tile * KT;
-                const int64_t ke = (kb + (end - it) < KT) ? kb + (end - it) : KT;
+                const Segment sg = segment_at(sc, it, end);
+                const uint32_t kb = sg.kb, ke = sg.ke;
                 int good = 1;
                 if (lane == 0)
                     good = mbar_wait_bounded(acce_bar(acc), acc_ph ^ 1u, s_abort, kp.limit_ns);
@@ -344,7 +446,7 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 tc_fence_after();
                 const uint32_t t_acc = tmem + acc * BN;
-                for (int64_t k = kb; k < ke; ++k) {
+                for (uint32_t k = kb; k < ke; ++k) {
                     good = 1;
                     if (lane == 0)
                         good = mbar_wait_bounded(full_bar(s), ph, s_abort, kp.limit_ns);
@@ -418,22 +520,65 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------------- epilogue
-        constexpr int CW = BN < 32 ? BN : 32;  // accumulator columns per tcgen05.ld
         const int quad = warp & 3;             // TMEM lanes 32*quad .. +31
         const int row = quad * 32 + lane;      // accumulator row = MMA row in tile
         const int etid = threadIdx.x - 64;     // 0..127
         int acc = 0;
         uint32_t acc_ph = 0;
+        uint32_t out_chunks = 0;               // BF16 chunks staged so far (buffer = parity)
         bool stop = false;
-        for (int64_t w = blockIdx.x; w < W && !stop; w += gridDim.x) {
-            int64_t it = worker_begin(w, I, W);
-            const int64_t end = worker_begin(w + 1, I, W);
+
+        // Convert one CW-column chunk of the tile (this thread's row) to BF16
+        // and write it to C: through shared memory and a TMA store when the
+        // output layout allows, else with predicated global stores.
+        auto emit = [&](const float (&v)[CW], int64_t tp, int64_t qcol) {
+            const int64_t p = tp * 128 + row;
+            if (!kp.tma_store) {
+                store_bf16<CW>(out, p, qcol, v);
+                return;
+            }
+            const int b = static_cast<int>(out_chunks & 1u);
+            uint8_t *buf = smem + C_::kOffOut + b * C_::kOutBytes;
+            if (etid == 0)
+                bulk_wait_group_read<1>();      // the store that last read this buffer is done
+            named_bar_sync(1, 128);
+            if (!kp.swap) {                     // [128 rows][CW] row-major, this thread's row
+                uint4 *dst = reinterpret_cast<uint4 *>(buf + row * CW * 2);
+#pragma unroll
+                for (int j = 0; j < CW / 8; ++j) {
+                    uint4 w;
+                    w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+                    w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+                    w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+                    w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+                    dst[j] = w;
+                }
+            } else {                            // [CW rows of C][128 columns of C]
+                __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(buf) + row;
+#pragma unroll
+                for (int j = 0; j < CW; ++j)
+                    dst[j * 128] = __float2bfloat16_rn(v[j]);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (etid == 0) {
+                if (!kp.swap)
+                    tma_store_2d(&tmC, smem_u32(buf), static_cast<int32_t>(qcol), static_cast<int32_t>(tp * 128));
+                else
+                    tma_store_2d(&tmC, smem_u32(buf), static_cast<int32_t>(tp * 128), static_cast<int32_t>(qcol));
+                bulk_commit_group();
+            }
+            ++out_chunks;
+        };
+
+        for (uint32_t w = blockIdx.x; w < W && !stop; w += gridDim.x) {
+            uint32_t it = sc.begin(w);
+            const uint32_t end = sc.begin(w + 1);
             bool first = true;
             while (it < end) {
-                const int64_t tile = it / KT;
-                const int64_t kb = it - tile * KT;
-                const int64_t ke = (kb + (end - it) < KT) ? kb + (end - it) : KT;
-                const int64_t tp = tile % kp.tilesP, tq = tile / kp.tilesP;
+                const Segment sg = segment_at(sc, it, end);
+                const uint32_t tile = sg.tile, kb = sg.kb, ke = sg.ke;
+                const int64_t tp = sg.tp, tq = sg.tq;
                 int good = 1;
                 if (lane == 0)
                     good = mbar_wait_bounded(accf_bar(acc), acc_ph, s_abort, kp.limit_ns);
@@ -447,9 +592,8 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 tc_fence_after();
                 const uint32_t t_acc = tmem + acc * BN + (static_cast<uint32_t>(quad * 32) << 16);
-                const int64_t p = tp * 128 + row;
-                const int64_t g_first = worker_of(tile * KT, I, W);
-                const int64_t g_last = worker_of(tile * KT + KT - 1, I, W);
+                const uint32_t g_first = sc.dp ? tile : sc.owner(tile * sc.KT);
+                const uint32_t g_last = sc.dp ? tile : sc.owner(tile * sc.KT + sc.KT - 1);
                 if (g_first == g_last) {
 #pragma unroll 1
                     for (int c = 0; c < BN; c += CW) {
@@ -460,10 +604,10 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                         for (int j = 0; j < CW; ++j)
                             v[j] = __uint_as_float(r[j]);
-                        store_bf16<CW>(kp, p, tq * BN + c, v);
+                        emit(v, tp, tq * BN + c);
                     }
                 } else {
-                    const int64_t slot = 2 * w + (first ? 0 : 1);
+                    const int64_t slot = 2 * static_cast<int64_t>(w) + (first ? 0 : 1);
                     float *mine = kp.partials + (slot * 128 + row) * BN;
 #pragma unroll 1
                     for (int c = 0; c < BN; c += CW) {
@@ -478,9 +622,9 @@ __global__ void __launch_bounds__(192, 1)
                     __threadfence();
                     named_bar_sync(1, 128);
                     if (etid == 0) {
-                        const int64_t nseg = g_last - g_first + 1;
+                        const uint32_t nseg = g_last - g_first + 1;
                         const uint32_t old = atomicAdd(kp.counters + tile, 1u);
-                        const int last = (static_cast<int64_t>(old) == nseg - 1) ? 1 : 0;
+                        const int last = (old == nseg - 1) ? 1 : 0;
                         if (last)
                             kp.counters[tile] = 0u;
                         *s_last = last;
@@ -497,14 +641,14 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                             for (int j = 0; j < CW; ++j)
                                 v[j] = 0.0f;
-                            for (int64_t g = g_first; g <= g_last; ++g) {
+                            for (uint32_t g = g_first; g <= g_last; ++g) {
                                 if (g == w) {
 #pragma unroll
                                     for (int j = 0; j < CW; ++j)
                                         v[j] += __uint_as_float(r[j]);
                                 } else {
                                     const int64_t gslot =
-                                        2 * g + ((worker_begin(g, I, W) / KT == tile) ? 0 : 1);
+                                        2 * static_cast<int64_t>(g) + ((sc.begin(g) / sc.KT == tile) ? 0 : 1);
                                     const float4 *src = reinterpret_cast<const float4 *>(
                                         kp.partials + (gslot * 128 + row) * BN + c);
 #pragma unroll
@@ -517,7 +661,7 @@ __global__ void __launch_bounds__(192, 1)
                                     }
                                 }
                             }
-                            store_bf16<CW>(kp, p, tq * BN + c, v);
+                            emit(v, tp, tq * BN + c);
                         }
                     }
                 }
@@ -533,6 +677,9 @@ __global__ void __launch_bounds__(192, 1)
                 it += ke - kb;
             }
         }
+        // Output stores must finish reading shared memory before the CTA exits.
+        if (etid == 0)
+            bulk_wait_group<0>();
     }
 
     tc_fence_before();
@@ -588,15 +735,41 @@ cudaError_t set_attrs()
                                 Cfg<FMT, BN>::kSmemBytes);
 }
 
+// 2-D BF16 map over C [M][N] with a box of box_x (inner, along N) x box_y
+// rows, no swizzle; used by the epilogue's TMA stores.
+bool make_output_map(CUtensorMap *map, void *C, int64_t M, int64_t N, int box_x, int box_y)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_x), static_cast<cuuint32_t>(box_y)};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int FMT, int BN>
-cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, cudaStream_t st)
+cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
+                     cudaStream_t st)
 {
     using C_ = Cfg<FMT, BN>;
     const int64_t rbytes = row_bytes(FMT, pl.K);
     const void *Pptr = pl.swap ? b.B : b.A;
     const void *Qptr = pl.swap ? b.A : b.B;
-    CUtensorMap tmP, tmQ;
+    CUtensorMap tmP, tmQ, tmC;
     if (!make_operand_map(&tmP, Pptr, pl.P, rbytes, 128) || !make_operand_map(&tmQ, Qptr, pl.Q, rbytes, BN))
+        return cudaErrorInvalidValue;
+    // TMA stores need 16-byte row pitch; other widths take the predicated
+    // store path (the map is then a never-used placeholder over C).
+    const int tma_store = (pl.N % 8 == 0) ? 1 : 0;
+    const bool okC = tma_store ? (pl.swap ? make_output_map(&tmC, b.C, pl.M, pl.N, 128, C_::kCW)
+                                          : make_output_map(&tmC, b.C, pl.M, pl.N, C_::kCW, 128))
+                               : make_output_map(&tmC, b.C, 1, 8, 8, 1);
+    if (!okC)
         return cudaErrorInvalidValue;
     KParams kp;
     kp.sfP = pl.swap ? b.sfB : b.sfA;
@@ -608,28 +781,40 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     kp.P = pl.P;
     kp.Q = pl.Q;
     kp.ldc = pl.N;
-    kp.tilesP = pl.tilesP;
-    kp.kt = pl.kt;
-    kp.iters = pl.iters;
-    kp.workers = pl.workers;
+    kp.tilesP = static_cast<uint32_t>(pl.tilesP);
+    kp.kt = static_cast<uint32_t>(pl.kt);
+    kp.iters = static_cast<uint32_t>(pl.iters);
+    kp.workers = static_cast<uint32_t>(pl.workers);
+    kp.dp = pl.workers == pl.tiles ? 1 : 0;
     kp.kaP = pl.kaP;
     kp.kaQ = pl.kaQ;
     kp.limit_ns = limit_ns;
     kp.swap = pl.swap;
     kp.inject = inject;
-    mx_gemm_kernel<FMT, BN><<<pl.grid, 192, C_::kSmemBytes, st>>>(tmP, tmQ, kp);
-    return cudaGetLastError();
+    kp.tma_store = tma_store;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = C_::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, mx_gemm_kernel<FMT, BN>, tmP, tmQ, tmC, kp);
 }
 
 template <int FMT>
-cudaError_t dispatch_bn(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, cudaStream_t st)
+cudaError_t dispatch_bn(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
+                        cudaStream_t st)
 {
     switch (pl.bn) {
-    case 16: return launch_t<FMT, 16>(pl, b, limit_ns, inject, st);
-    case 32: return launch_t<FMT, 32>(pl, b, limit_ns, inject, st);
-    case 64: return launch_t<FMT, 64>(pl, b, limit_ns, inject, st);
-    case 128: return launch_t<FMT, 128>(pl, b, limit_ns, inject, st);
-    case 256: return launch_t<FMT, 256>(pl, b, limit_ns, inject, st);
+    case 16: return launch_t<FMT, 16>(pl, b, limit_ns, inject, pdl, st);
+    case 32: return launch_t<FMT, 32>(pl, b, limit_ns, inject, pdl, st);
+    case 64: return launch_t<FMT, 64>(pl, b, limit_ns, inject, pdl, st);
+    case 128: return launch_t<FMT, 128>(pl, b, limit_ns, inject, pdl, st);
+    case 256: return launch_t<FMT, 256>(pl, b, limit_ns, inject, pdl, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -686,8 +871,21 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
     pl.iters = pl.tiles * pl.kt;
     const int64_t sms = num_sms > 0 ? num_sms : 1;
     int s = sched;
-    if (s == 0)   // auto
-        s = pl.tiles >= sms ? 1 : 3;
+    int auto_splits = 1;
+    if (s == 0) {
+        // auto: whole tiles unless the tiles fill at most half the GPU and
+        // each tile has enough K steps to amortise a two-way split's fixup
+        // (measured on B200 for the decode shapes: the split's partial
+        // write, atomic and reduction cost ~2 us per tile).
+        if (pl.tiles * 2 <= sms && pl.kt >= 16) {
+            s = 2;
+            auto_splits = 2;
+        } else {
+            s = 1;
+        }
+    }
+    if (sched == 0 && s == 2)
+        splits = auto_splits;
     pl.sched = s;
     if (s == 1) {
         pl.workers = pl.tiles;
@@ -704,6 +902,16 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
     }
     if (pl.workers < 1)
         pl.workers = 1;
+    // the kernel's scheduler arithmetic is 32-bit: iters * workers < 2^32
+    // unless whole tiles are scheduled (which needs no products)
+    const int64_t lim = (int64_t(1) << 32) - 1;
+    if (pl.workers != pl.tiles && pl.iters * pl.workers > lim) {
+        const int64_t w = lim / pl.iters;
+        pl.workers = w > pl.tiles ? w : pl.tiles;
+        if (pl.workers != pl.tiles && pl.iters * pl.workers > lim)
+            pl.workers = pl.tiles;
+    }
+    pl.valid = pl.iters < (int64_t(1) << 31) && pl.tiles < (int64_t(1) << 31);
     pl.grid = static_cast<int>(pl.workers < sms ? pl.workers : sms);
     pl.kaP = sf_atoms_per_rowblock(fmt, K);
     pl.kaQ = pl.kaP;
@@ -712,12 +920,12 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
     return pl;
 }
 
-cudaError_t launch_gemm(const GemmPlan &plan, const GemmBuffers &buf, uint64_t wait_limit_ns, int inject,
+cudaError_t launch_gemm(const GemmPlan &plan, const GemmBuffers &buf, uint64_t wait_limit_ns, int inject, int pdl,
                         cudaStream_t stream)
 {
     if (plan.fmt == kFmtMXFP8)
-        return dispatch_bn<0>(plan, buf, wait_limit_ns, inject, stream);
-    return dispatch_bn<1>(plan, buf, wait_limit_ns, inject, stream);
+        return dispatch_bn<0>(plan, buf, wait_limit_ns, inject, pdl, stream);
+    return dispatch_bn<1>(plan, buf, wait_limit_ns, inject, pdl, stream);
 }
 
 }  // namespace mxg

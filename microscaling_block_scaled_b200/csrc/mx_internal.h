@@ -57,6 +57,7 @@ struct GemmPlan {
     int sched = 0;         // resolved schedule (MXGEMM_SCHED_*)
     int64_t kaP = 0, kaQ = 0;
     int64_t partial_bytes = 0;  // workspace for split partials
+    bool valid = true;          // false: the shape exceeds the kernel's 32-bit scheduler range
     int64_t counter_bytes = 0;
 };
 
@@ -73,7 +74,10 @@ struct GemmBuffers {
     uint32_t *counters;
     int *error;
 };
-cudaError_t launch_gemm(const GemmPlan &plan, const GemmBuffers &buf, uint64_t wait_limit_ns, int inject,
+// pdl: launch as a programmatic dependent of the preceding kernel (the
+// scale repack of mxgemm_run), letting the prologue and the first operand
+// loads overlap it; the kernel waits for it before touching the scales.
+cudaError_t launch_gemm(const GemmPlan &plan, const GemmBuffers &buf, uint64_t wait_limit_ns, int inject, int pdl,
                         cudaStream_t stream);
 
 // Per-(fmt, BN) kernel attribute setup; returns cudaSuccess once done.

@@ -134,9 +134,14 @@ MXGEMM_API int mxgemm_quantize(int fmt, int64_t R, int64_t K, const float *X,
  * MXGEMM_SCHED_STREAMK (0 = number of SMs). */
 MXGEMM_API int mxgemm_set_schedule(mxgemm_handle h, int schedule, int splits, int workers);
 
+/* Force the number of 128-byte K chunks each pipeline stage of later GEMMs
+ * on this handle loads: 1 or 2 (2 applies only when an operand row is a
+ * whole number of 128-byte chunks), 0 = automatic (the default). */
+MXGEMM_API int mxgemm_set_kchunks(mxgemm_handle h, int kc);
+
 /* Describe the plan mxgemm_gemm would use for a shape: writes up to `cap`
  * bytes of a NUL-terminated text such as
- * "fmt=1 swap=1 BN=32 stages=10 tiles=112 kt=16 workers=148 grid=148 sched=streamk". */
+ * "fmt=1 swap=1 BN=32 kc=2 stages=4 tiles=112 kt=8 workers=112 grid=112 sched=dp partial_bytes=0". */
 MXGEMM_API int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
                          char *buf, size_t cap);
 

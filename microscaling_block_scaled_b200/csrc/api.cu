@@ -36,6 +36,7 @@ struct mxgemm_ctx {
     int sched = MXGEMM_SCHED_AUTO;
     int splits = 1;
     int workers = 0;
+    int kchunks = 0;        // 0 = auto
     uint64_t limit_ns = 2000000000ull;
     int inject = 0;
     // shape of the last repack
@@ -127,7 +128,7 @@ int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const voi
 {
     if (h->last_fmt != fmt || h->last_M != M || h->last_N != N || h->last_K != K)
         return MXGEMM_ERR_INVALID_ARG;
-    const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers);
+    const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks);
     if (!pl.valid)
         return MXGEMM_ERR_INVALID_ARG;
     int rc = grow(&h->partials, &h->partials_cap, static_cast<size_t>(pl.partial_bytes > 0 ? pl.partial_bytes : 16),
@@ -340,6 +341,14 @@ int mxgemm_set_schedule(mxgemm_handle h, int schedule, int splits, int workers)
     return MXGEMM_OK;
 }
 
+int mxgemm_set_kchunks(mxgemm_handle h, int kc)
+{
+    if (!h || kc < 0 || kc > 2)
+        return MXGEMM_ERR_INVALID_ARG;
+    h->kchunks = kc;
+    return MXGEMM_OK;
+}
+
 int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, char *buf, size_t cap)
 {
     if (!h || !buf || cap == 0)
@@ -347,11 +356,12 @@ int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t
     int rc = check_shape(fmt, M, N, K);
     if (rc != MXGEMM_OK)
         return rc;
-    const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers);
+    const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks);
     static const char *names[] = {"auto", "dp", "splitk", "streamk"};
     snprintf(buf, cap,
-             "fmt=%d swap=%d BN=%d stages=%d tiles=%lld kt=%lld workers=%lld grid=%d sched=%s partial_bytes=%lld",
-             pl.fmt, pl.swap, pl.bn, pl.stages, static_cast<long long>(pl.tiles), static_cast<long long>(pl.kt),
+             "fmt=%d swap=%d BN=%d kc=%d stages=%d tiles=%lld kt=%lld workers=%lld grid=%d sched=%s "
+             "partial_bytes=%lld",
+             pl.fmt, pl.swap, pl.bn, pl.kc, pl.stages, static_cast<long long>(pl.tiles), static_cast<long long>(pl.kt),
              static_cast<long long>(pl.workers), pl.grid, names[pl.sched & 3],
              static_cast<long long>(pl.partial_bytes));
     return MXGEMM_OK;

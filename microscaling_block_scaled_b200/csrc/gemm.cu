@@ -49,14 +49,16 @@ namespace mxg {
 
 // ------------------------------------------------------------ configuration
 
-template <int FMT, int BN>
+template <int FMT, int BN, int KC>
 struct Cfg {
     static constexpr int kBM = 128;
-    static constexpr int kStageKBytes = 128;                  // K bytes per stage per row
-    static constexpr int kAtoms = FMT == kFmtMXFP8 ? 1 : 2;   // 512B scale atoms per 128 rows
+    static constexpr int kAtomsPerChunk = FMT == kFmtMXFP8 ? 1 : 2;   // 512B scale atoms per 128-byte K chunk
+    static constexpr int kAtoms = kAtomsPerChunk * KC;        // scale atoms per 128 rows per stage
     static constexpr int kRBQ = (BN + 127) / 128;             // 128-row blocks of the column operand
-    static constexpr int kABytes = kBM * kStageKBytes;
-    static constexpr int kBBytes = BN * kStageKBytes;
+    static constexpr int kAChunk = kBM * 128;                 // one 128-byte K chunk of the row-operand tile
+    static constexpr int kBChunk = BN * 128;
+    static constexpr int kABytes = kAChunk * KC;
+    static constexpr int kBBytes = kBChunk * KC;
     static constexpr int kSFABytes = kAtoms * 512;
     static constexpr int kSFBBytes = kRBQ * kAtoms * 512;
     static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
@@ -71,7 +73,7 @@ struct Cfg {
     static constexpr int kNumAcc = (2 * BN + kSFCols <= 512) ? 2 : 1;
     static constexpr int kAccCols = kNumAcc * BN;
     static constexpr int kTmemCols = 512;
-    static constexpr int kMmaPerStage = 4;                    // 32 bytes of K per MMA
+    static constexpr int kMmaPerChunk = 4;                    // 32 bytes of K per MMA
     static constexpr uint32_t kTxBytes = kStageBytes;
     // shared memory layout (offsets from a 1024-aligned base)
     static constexpr int kOffA = 0;
@@ -85,9 +87,10 @@ struct Cfg {
     static constexpr int kSmemBytes = kOffMisc + 64 + 1024;   // + alignment slack
 
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be a multiple of 16 in [16, 256]");
+    static_assert(KC == 1 || KC == 2 || KC == 4, "1, 2 or 4 K chunks per stage");
     static_assert(kStages >= 2, "at least two pipeline stages");
     static_assert(kAccCols + kSFCols <= kTmemCols, "TMEM budget");
-    static_assert(kBBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
+    static_assert(kBChunk % 1024 == 0, "tiles must keep 1024-byte alignment");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -264,12 +267,12 @@ __device__ __forceinline__ void store_bf16(const OutView o, int64_t p, int64_t q
     }
 }
 
-template <int FMT, int BN>
+template <int FMT, int BN, int KC>
 __global__ void __launch_bounds__(192, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmC, const KParams kp_in)
 {
-    using C_ = Cfg<FMT, BN>;
+    using C_ = Cfg<FMT, BN, KC>;
     constexpr int S = C_::kStages;
     constexpr int CW = C_::kCW;
 
@@ -343,11 +346,19 @@ __global__ void __launch_bounds__(192, 1)
         auto load_operands = [&](int s, uint32_t tile, uint32_t k) {
             const uint32_t tq = tile / sc.tilesP, tp = tile - tq * sc.tilesP;
             const uint32_t fb = full_bar(s);
-            const int32_t x = static_cast<int32_t>(k * C_::kStageKBytes);
-            tma_load_2d(sbase + C_::kOffA + s * C_::kABytes, &tmP, x, static_cast<int32_t>(tp) * 128, fb,
-                        pol_stream);
-            tma_load_2d(sbase + C_::kOffB + s * C_::kBBytes, &tmQ, x, static_cast<int32_t>(tq) * BN, fb,
-                        pol_stream);
+            if constexpr (KC == 1) {       // 2-D maps: x = byte offset along K
+                const int32_t x = static_cast<int32_t>(k * 128);
+                tma_load_2d(sbase + C_::kOffA + s * C_::kABytes, &tmP, x, static_cast<int32_t>(tp) * 128, fb,
+                            pol_stream);
+                tma_load_2d(sbase + C_::kOffB + s * C_::kBBytes, &tmQ, x, static_cast<int32_t>(tq) * BN, fb,
+                            pol_stream);
+            } else {                       // 3-D maps: {byte in chunk, row, 128-byte K chunk}
+                const int32_t z = static_cast<int32_t>(k * KC);
+                tma_load_3d(sbase + C_::kOffA + s * C_::kABytes, &tmP, 0, static_cast<int32_t>(tp) * 128, z, fb,
+                            pol_stream);
+                tma_load_3d(sbase + C_::kOffB + s * C_::kBBytes, &tmQ, 0, static_cast<int32_t>(tq) * BN, z, fb,
+                            pol_stream);
+            }
         };
         auto load_scales = [&](int s, uint32_t tile, uint32_t k) {
             const uint32_t tq = tile / sc.tilesP, tp = tile - tq * sc.tilesP;
@@ -472,23 +483,28 @@ __global__ void __launch_bounds__(192, 1)
                             for (int a = 0; a < C_::kAtoms; ++a)
                                 tmem_cp_32x128b_x4(t_sfb + a * 4 * C_::kRBQ + 4 * rb,
                                                    sdesc_rows16(s_sfb + (rb * C_::kAtoms + a) * 512));
-                        const uint64_t adesc = sdesc_sw128_kmajor(sbase + C_::kOffA + s * C_::kABytes);
-                        const uint64_t bdesc = sdesc_sw128_kmajor(sbase + C_::kOffB + s * C_::kBBytes);
 #pragma unroll
-                        for (int j = 0; j < C_::kMmaPerStage; ++j) {
-                            // MXFP8: one scale block per MMA, id j of the atom's 4 bytes.
-                            // MXFP4: two scale blocks per MMA, atom j/2, byte pair 2*(j%2).
-                            const int atom = FMT == kFmtMXFP8 ? 0 : j / 2;
-                            const uint32_t sf_id = FMT == kFmtMXFP8 ? j : 2 * (j % 2);
-                            const uint32_t idesc = kIdesc | (sf_id << 4) | (sf_id << 29);
-                            const uint32_t acc_flag = (k > kb || j > 0) ? 1u : 0u;
-                            const uint64_t koff = static_cast<uint64_t>(j * 32) >> 4;
-                            if (FMT == kFmtMXFP8)
-                                mma_mxf8f6f4(t_acc, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
+                        for (int c = 0; c < KC; ++c) {
+                            const uint64_t adesc =
+                                sdesc_sw128_kmajor(sbase + C_::kOffA + s * C_::kABytes + c * C_::kAChunk);
+                            const uint64_t bdesc =
+                                sdesc_sw128_kmajor(sbase + C_::kOffB + s * C_::kBBytes + c * C_::kBChunk);
+#pragma unroll
+                            for (int j = 0; j < C_::kMmaPerChunk; ++j) {
+                                // MXFP8: one scale block per MMA, id j of the chunk's atom.
+                                // MXFP4: two scale blocks per MMA, atom 2c + j/2, byte pair 2*(j%2).
+                                const int atom = FMT == kFmtMXFP8 ? c : 2 * c + j / 2;
+                                const uint32_t sf_id = FMT == kFmtMXFP8 ? j : 2 * (j % 2);
+                                const uint32_t idesc = kIdesc | (sf_id << 4) | (sf_id << 29);
+                                const uint32_t acc_flag = (k > kb || c > 0 || j > 0) ? 1u : 0u;
+                                const uint64_t koff = static_cast<uint64_t>(j * 32) >> 4;
+                                if (FMT == kFmtMXFP8)
+                                    mma_mxf8f6f4(t_acc, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
+                                                 t_sfb + atom * 4 * C_::kRBQ, acc_flag);
+                                else
+                                    mma_mxf4(t_acc, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
                                              t_sfb + atom * 4 * C_::kRBQ, acc_flag);
-                            else
-                                mma_mxf4(t_acc, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
-                                         t_sfb + atom * 4 * C_::kRBQ, acc_flag);
+                            }
                         }
                         tc_commit(empty_bar(s));
                     }
@@ -728,11 +744,30 @@ bool make_operand_map(CUtensorMap *map, const void *base, int64_t rows, int64_t 
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, int BN>
+// 3-D uint8 map viewing [rows][row_bytes] as {128-byte piece, row, chunk}
+// (strides: row_bytes between rows, 128 bytes between chunks) with a box of
+// 128 bytes x box_rows x kc chunks, 128-byte swizzle, zero fill out of
+// bounds.  Needs row_bytes % 128 == 0.
+bool make_operand_map_3d(CUtensorMap *map, const void *base, int64_t rows, int64_t rbytes, int box_rows, int kc)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || rbytes % 128 != 0)
+        return false;
+    cuuint64_t dims[3] = {128u, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(rbytes / 128)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(rbytes), 128u};
+    cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(kc)};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int FMT, int BN, int KC>
 cudaError_t set_attrs()
 {
-    return cudaFuncSetAttribute(mx_gemm_kernel<FMT, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Cfg<FMT, BN>::kSmemBytes);
+    return cudaFuncSetAttribute(mx_gemm_kernel<FMT, BN, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Cfg<FMT, BN, KC>::kSmemBytes);
 }
 
 // 2-D BF16 map over C [M][N] with a box of box_x (inner, along N) x box_y
@@ -752,17 +787,23 @@ bool make_output_map(CUtensorMap *map, void *C, int64_t M, int64_t N, int box_x,
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, int BN>
+template <int FMT, int BN, int KC>
 cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
                      cudaStream_t st)
 {
-    using C_ = Cfg<FMT, BN>;
+    using C_ = Cfg<FMT, BN, KC>;
     const int64_t rbytes = row_bytes(FMT, pl.K);
     const void *Pptr = pl.swap ? b.B : b.A;
     const void *Qptr = pl.swap ? b.A : b.B;
     CUtensorMap tmP, tmQ, tmC;
-    if (!make_operand_map(&tmP, Pptr, pl.P, rbytes, 128) || !make_operand_map(&tmQ, Qptr, pl.Q, rbytes, BN))
-        return cudaErrorInvalidValue;
+    if (KC == 1) {
+        if (!make_operand_map(&tmP, Pptr, pl.P, rbytes, 128) || !make_operand_map(&tmQ, Qptr, pl.Q, rbytes, BN))
+            return cudaErrorInvalidValue;
+    } else {
+        if (!make_operand_map_3d(&tmP, Pptr, pl.P, rbytes, 128, KC) ||
+            !make_operand_map_3d(&tmQ, Qptr, pl.Q, rbytes, BN, KC))
+            return cudaErrorInvalidValue;
+    }
     // TMA stores need 16-byte row pitch; other widths take the predicated
     // store path (the map is then a never-used placeholder over C).
     const int tma_store = (pl.N % 8 == 0) ? 1 : 0;
@@ -802,34 +843,41 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, mx_gemm_kernel<FMT, BN>, tmP, tmQ, tmC, kp);
+    return cudaLaunchKernelEx(&cfg, mx_gemm_kernel<FMT, BN, KC>, tmP, tmQ, tmC, kp);
 }
 
-template <int FMT>
+template <int FMT, int KC>
 cudaError_t dispatch_bn(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
                         cudaStream_t st)
 {
     switch (pl.bn) {
-    case 16: return launch_t<FMT, 16>(pl, b, limit_ns, inject, pdl, st);
-    case 32: return launch_t<FMT, 32>(pl, b, limit_ns, inject, pdl, st);
-    case 64: return launch_t<FMT, 64>(pl, b, limit_ns, inject, pdl, st);
-    case 128: return launch_t<FMT, 128>(pl, b, limit_ns, inject, pdl, st);
-    case 256: return launch_t<FMT, 256>(pl, b, limit_ns, inject, pdl, st);
+    case 16: return launch_t<FMT, 16, KC>(pl, b, limit_ns, inject, pdl, st);
+    case 32: return launch_t<FMT, 32, KC>(pl, b, limit_ns, inject, pdl, st);
+    case 64: return launch_t<FMT, 64, KC>(pl, b, limit_ns, inject, pdl, st);
+    case 128: return launch_t<FMT, 128, KC>(pl, b, limit_ns, inject, pdl, st);
+    case 256: return launch_t<FMT, 256, KC>(pl, b, limit_ns, inject, pdl, st);
     default: return cudaErrorInvalidValue;
     }
 }
 
-template <int FMT>
-int stages_for(int bn)
+template <int FMT, int KC>
+int stages_kc(int bn)
 {
     switch (bn) {
-    case 16: return Cfg<FMT, 16>::kStages;
-    case 32: return Cfg<FMT, 32>::kStages;
-    case 64: return Cfg<FMT, 64>::kStages;
-    case 128: return Cfg<FMT, 128>::kStages;
-    case 256: return Cfg<FMT, 256>::kStages;
+    case 16: return Cfg<FMT, 16, KC>::kStages;
+    case 32: return Cfg<FMT, 32, KC>::kStages;
+    case 64: return Cfg<FMT, 64, KC>::kStages;
+    case 128: return Cfg<FMT, 128, KC>::kStages;
+    case 256: return Cfg<FMT, 256, KC>::kStages;
     default: return 0;
     }
+}
+
+int stages_for(int fmt, int bn, int kc)
+{
+    if (fmt == kFmtMXFP8)
+        return kc == 1 ? stages_kc<0, 1>(bn) : stages_kc<0, 2>(bn);
+    return kc == 1 ? stages_kc<1, 1>(bn) : stages_kc<1, 2>(bn);
 }
 
 }  // namespace
@@ -837,16 +885,19 @@ int stages_for(int bn)
 cudaError_t prepare_gemm_kernels()
 {
     cudaError_t e = cudaSuccess;
-#define MXG_ATTR(F, B)                 \
-    if (e == cudaSuccess)              \
-        e = set_attrs<F, B>();
+#define MXG_ATTR(F, B)                                                  \
+    if (e == cudaSuccess)                                               \
+        e = set_attrs<F, B, 1>();                                       \
+    if (e == cudaSuccess)                                               \
+        e = set_attrs<F, B, 2>();
     MXG_ATTR(0, 16) MXG_ATTR(0, 32) MXG_ATTR(0, 64) MXG_ATTR(0, 128) MXG_ATTR(0, 256)
     MXG_ATTR(1, 16) MXG_ATTR(1, 32) MXG_ATTR(1, 64) MXG_ATTR(1, 128) MXG_ATTR(1, 256)
 #undef MXG_ATTR
     return e;
 }
 
-GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sched, int splits, int workers)
+GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sched, int splits, int workers,
+                   int force_kc)
 {
     GemmPlan pl;
     pl.fmt = fmt;
@@ -863,10 +914,16 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
         pl.Q = N;
         pl.bn = 128;
     }
-    pl.stages = fmt == kFmtMXFP8 ? stages_for<0>(pl.bn) : stages_for<1>(pl.bn);
+    // Two 128-byte K chunks per stage halve the TMA operations per byte (each
+    // costs ~0.2 us of the SM's copy engine); rows must be whole chunks.
+    const int64_t chunks = (row_bytes(fmt, K) + 127) / 128;
+    pl.kc = (row_bytes(fmt, K) % 128 == 0 && chunks >= 2) ? 2 : 1;
+    if (force_kc == 1 || (force_kc == 2 && pl.kc == 2))
+        pl.kc = force_kc;
+    pl.stages = stages_for(fmt, pl.bn, pl.kc);
     pl.tilesP = (pl.P + 127) / 128;
     pl.tilesQ = (pl.Q + pl.bn - 1) / pl.bn;
-    pl.kt = (row_bytes(fmt, K) + 127) / 128;
+    pl.kt = (chunks + pl.kc - 1) / pl.kc;
     pl.tiles = pl.tilesP * pl.tilesQ;
     pl.iters = pl.tiles * pl.kt;
     const int64_t sms = num_sms > 0 ? num_sms : 1;
@@ -924,8 +981,10 @@ cudaError_t launch_gemm(const GemmPlan &plan, const GemmBuffers &buf, uint64_t w
                         cudaStream_t stream)
 {
     if (plan.fmt == kFmtMXFP8)
-        return dispatch_bn<0>(plan, buf, wait_limit_ns, inject, pdl, stream);
-    return dispatch_bn<1>(plan, buf, wait_limit_ns, inject, pdl, stream);
+        return plan.kc == 1 ? dispatch_bn<0, 1>(plan, buf, wait_limit_ns, inject, pdl, stream)
+                            : dispatch_bn<0, 2>(plan, buf, wait_limit_ns, inject, pdl, stream);
+    return plan.kc == 1 ? dispatch_bn<1, 1>(plan, buf, wait_limit_ns, inject, pdl, stream)
+                        : dispatch_bn<1, 2>(plan, buf, wait_limit_ns, inject, pdl, stream);
 }
 
 }  // namespace mxg

@@ -13,9 +13,9 @@ constexpr int kFmtMXFP4 = 1;
 // Bytes of one operand row of K elements.
 inline int64_t row_bytes(int fmt, int64_t K) { return fmt == kFmtMXFP8 ? K : K / 2; }
 
-// 512-byte scale atoms per 128-row block per pipeline stage (a stage spans
-// 128 bytes of K: 128 E4M3 elements = 4 scale blocks, or 256 E2M1 elements
-// = 8 scale blocks).
+// 512-byte scale atoms per 128-row block per 128-byte K chunk of the
+// operands (128 E4M3 elements = 4 scale blocks, or 256 E2M1 elements = 8
+// scale blocks); a pipeline stage holds 1, 2 or 4 chunks.
 inline int atoms_per_stage(int fmt) { return fmt == kFmtMXFP8 ? 1 : 2; }
 
 // Repacked scale layout of one operand with R rows: [ceil(R/256)*2][ka][512]
@@ -27,7 +27,7 @@ inline int atoms_per_stage(int fmt) { return fmt == kFmtMXFP8 ? 1 : 2; }
 // expects for block-scale factors.
 inline int64_t sf_atoms_per_rowblock(int fmt, int64_t K)
 {
-    const int64_t a = K / 128, s = atoms_per_stage(fmt);
+    const int64_t a = K / 128, s = 4 * atoms_per_stage(fmt);   // room for up to 4 chunks per stage
     return (a + s - 1) / s * s;
 }
 inline int64_t sf_repacked_bytes(int fmt, int64_t R, int64_t K)
@@ -48,6 +48,7 @@ struct GemmPlan {
     int fmt = 0;
     int swap = 0;          // 1: MMA rows come from B (C^T = B * A^T)
     int bn = 0;            // MMA N (columns of one output tile)
+    int kc = 1;            // 128-byte K chunks per pipeline stage
     int stages = 0;
     int64_t M = 0, N = 0, K = 0;
     int64_t P = 0, Q = 0;  // rows of the MMA's row operand / column operand
@@ -63,7 +64,7 @@ struct GemmPlan {
 
 // Build the plan for a shape.  sched/splits/workers as mxgemm_set_schedule.
 GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sched, int splits,
-                   int workers);
+                   int workers, int force_kc = 0);
 
 // Launch the GEMM kernel for `plan`.
 struct GemmBuffers {

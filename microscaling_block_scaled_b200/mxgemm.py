@@ -40,6 +40,7 @@ SIGNATURES = {
     "mxgemm_run_host": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "mxgemm_quantize": (ctypes.c_int, [ctypes.c_int, _i64, _i64, _vp, _vp, _vp, _vp]),
     "mxgemm_set_schedule": (ctypes.c_int, [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "mxgemm_set_kchunks": (ctypes.c_int, [_vp, ctypes.c_int]),
     "mxgemm_describe_plan": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, ctypes.c_char_p, ctypes.c_size_t]),
     "mxgemm_check_device_error": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_int)]),
     "mxgemm_set_wait_limit": (ctypes.c_int, [_vp, ctypes.c_uint64]),
@@ -137,6 +138,10 @@ def mxgemm_set_schedule(h, schedule, splits=1, workers=0) -> int:
     return load().mxgemm_set_schedule(h, schedule, splits, workers)
 
 
+def mxgemm_set_kchunks(h, kc) -> int:
+    return load().mxgemm_set_kchunks(h, kc)
+
+
 def mxgemm_describe_plan(h, fmt, M, N, K) -> str:
     buf = ctypes.create_string_buffer(256)
     _check("mxgemm_describe_plan", load().mxgemm_describe_plan(h, fmt, M, N, K, buf, 256))
@@ -190,6 +195,9 @@ class Handle:
 
     def set_schedule(self, schedule: int, splits: int = 1, workers: int = 0):
         _check("mxgemm_set_schedule", mxgemm_set_schedule(self.h, schedule, splits, workers))
+
+    def set_kchunks(self, kc: int):
+        _check("mxgemm_set_kchunks", mxgemm_set_kchunks(self.h, kc))
 
     def describe(self, fmt, M, N, K) -> str:
         return mxgemm_describe_plan(self.h, fmt, M, N, K)

@@ -95,6 +95,20 @@ def test_gemm_forced_schedules(fmt, sched, M, N, K):
     full_case(fmt, M, N, K, seed=9, schedule=sched)
 
 
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("kc", [1, 2])
+@pytest.mark.parametrize("M,N,K", [(32, 512, 1024), (200, 384, 640), (64, 256, 384), (130, 256, 896)])
+def test_gemm_k_chunks_per_stage(fmt, kc, M, N, K):
+    """One and two 128-byte K chunks per pipeline stage (2-D and 3-D TMA
+    boxes), including K whose last stage is partly past the end of a row."""
+    h = handle()
+    h.set_kchunks(kc)
+    try:
+        full_case(fmt, M, N, K, seed=kc * 100 + K)
+    finally:
+        h.set_kchunks(0)
+
+
 # ----------------------------------------------------------- edge cases
 
 def _codes_case(fmt, A, SA, B, SB, K):

@@ -135,8 +135,9 @@ MXGEMM_API int mxgemm_quantize(int fmt, int64_t R, int64_t K, const float *X,
 MXGEMM_API int mxgemm_set_schedule(mxgemm_handle h, int schedule, int splits, int workers);
 
 /* Force the number of 128-byte K chunks each pipeline stage of later GEMMs
- * on this handle loads: 1 or 2 (2 applies only when an operand row is a
- * whole number of 128-byte chunks), 0 = automatic (the default). */
+ * on this handle loads: 1, 2 or 4 (2 and 4 apply only when an operand row is
+ * a whole number of 128-byte chunks; 4 only to tiles of at most 64 columns),
+ * 0 = automatic (the default). */
 MXGEMM_API int mxgemm_set_kchunks(mxgemm_handle h, int kc);
 
 /* Describe the plan mxgemm_gemm would use for a shape: writes up to `cap`

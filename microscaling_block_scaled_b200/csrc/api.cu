@@ -343,7 +343,7 @@ int mxgemm_set_schedule(mxgemm_handle h, int schedule, int splits, int workers)
 
 int mxgemm_set_kchunks(mxgemm_handle h, int kc)
 {
-    if (!h || kc < 0 || kc > 2)
+    if (!h || kc < 0 || kc > 4 || kc == 3)
         return MXGEMM_ERR_INVALID_ARG;
     h->kchunks = kc;
     return MXGEMM_OK;

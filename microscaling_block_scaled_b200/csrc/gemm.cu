@@ -41,6 +41,7 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 
 #include "mx_internal.h"
 #include "sm100_ptx.cuh"
@@ -338,7 +339,11 @@ __global__ void __launch_bounds__(192, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
-        const uint64_t pol_stream = policy_evict_first();
+        // L2 policy per operand: in the swapped (decode) form the weights
+        // stream through once and the small activation is re-read by every
+        // tile; otherwise both operands are re-read across tiles.
+        const uint64_t polP = kp.swap ? policy_evict_first() : policy_evict_normal();
+        const uint64_t polQ = kp.swap ? policy_evict_last() : policy_evict_normal();
         uint32_t armed = 0;         // stages armed so far (round-robin over the ring)
         int skipped_stage = -1;
         bool inject = kp.inject == 1;
@@ -349,15 +354,15 @@ __global__ void __launch_bounds__(192, 1)
             if constexpr (KC == 1) {       // 2-D maps: x = byte offset along K
                 const int32_t x = static_cast<int32_t>(k * 128);
                 tma_load_2d(sbase + C_::kOffA + s * C_::kABytes, &tmP, x, static_cast<int32_t>(tp) * 128, fb,
-                            pol_stream);
+                            polP);
                 tma_load_2d(sbase + C_::kOffB + s * C_::kBBytes, &tmQ, x, static_cast<int32_t>(tq) * BN, fb,
-                            pol_stream);
+                            polQ);
             } else {                       // 3-D maps: {byte in chunk, row, 128-byte K chunk}
                 const int32_t z = static_cast<int32_t>(k * KC);
                 tma_load_3d(sbase + C_::kOffA + s * C_::kABytes, &tmP, 0, static_cast<int32_t>(tp) * 128, z, fb,
-                            pol_stream);
+                            polP);
                 tma_load_3d(sbase + C_::kOffB + s * C_::kBBytes, &tmQ, 0, static_cast<int32_t>(tq) * BN, z, fb,
-                            pol_stream);
+                            polQ);
             }
         };
         auto load_scales = [&](int s, uint32_t tile, uint32_t k) {
@@ -376,10 +381,11 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) {
             IterCursor cur(sc, blockIdx.x, gridDim.x);
             const uint32_t n_total = cur.total();
-            const uint32_t n_pre = n_total < static_cast<uint32_t>(S) ? n_total : static_cast<uint32_t>(S);
-            // Pass 1: operand tiles of the first ring's worth of stages (the
-            // ring is empty, no wait needed); they do not depend on the
-            // preceding kernel.
+            // Pass 1: the operand tiles of the first stage, which do not depend
+            // on the preceding kernel (the ring is empty, no wait needed).
+            // Only one stage: its scales queue behind whatever is issued here,
+            // and the first stage's latency is on the critical path.
+            const uint32_t n_pre = n_total < 1u ? n_total : 1u;
             for (uint32_t n = 0; n < n_pre; ++n, cur.advance()) {
                 const int s = static_cast<int>(n);
                 if (inject && n == 0) {
@@ -398,7 +404,7 @@ __global__ void __launch_bounds__(192, 1)
                     load_scales(static_cast<int>(n), cur2.tile, cur2.k);
             // Pass 3: the rest, one ring slot at a time.
             int s = static_cast<int>(n_pre % S);
-            uint32_t ph = n_pre == static_cast<uint32_t>(S) ? 1u : 0u;
+            uint32_t ph = 0u;
             for (uint32_t n = n_pre; n < n_total; ++n, cur.advance()) {
                 if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns)) {
                     record_error(kp.error, kErrProducerEmpty, s_abort);
@@ -860,6 +866,18 @@ cudaError_t dispatch_bn(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit
     }
 }
 
+template <int FMT>
+cudaError_t dispatch_bn4(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
+                         cudaStream_t st)
+{
+    switch (pl.bn) {
+    case 16: return launch_t<FMT, 16, 4>(pl, b, limit_ns, inject, pdl, st);
+    case 32: return launch_t<FMT, 32, 4>(pl, b, limit_ns, inject, pdl, st);
+    case 64: return launch_t<FMT, 64, 4>(pl, b, limit_ns, inject, pdl, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 template <int FMT, int KC>
 int stages_kc(int bn)
 {
@@ -873,8 +891,21 @@ int stages_kc(int bn)
     }
 }
 
+template <int FMT>
+int stages_kc4(int bn)
+{
+    switch (bn) {
+    case 16: return Cfg<FMT, 16, 4>::kStages;
+    case 32: return Cfg<FMT, 32, 4>::kStages;
+    case 64: return Cfg<FMT, 64, 4>::kStages;
+    default: return 0;
+    }
+}
+
 int stages_for(int fmt, int bn, int kc)
 {
+    if (kc == 4)
+        return fmt == kFmtMXFP8 ? stages_kc4<0>(bn) : stages_kc4<1>(bn);
     if (fmt == kFmtMXFP8)
         return kc == 1 ? stages_kc<0, 1>(bn) : stages_kc<0, 2>(bn);
     return kc == 1 ? stages_kc<1, 1>(bn) : stages_kc<1, 2>(bn);
@@ -893,6 +924,11 @@ cudaError_t prepare_gemm_kernels()
     MXG_ATTR(0, 16) MXG_ATTR(0, 32) MXG_ATTR(0, 64) MXG_ATTR(0, 128) MXG_ATTR(0, 256)
     MXG_ATTR(1, 16) MXG_ATTR(1, 32) MXG_ATTR(1, 64) MXG_ATTR(1, 128) MXG_ATTR(1, 256)
 #undef MXG_ATTR
+#define MXG_ATTR4(F, B)                                                 \
+    if (e == cudaSuccess)                                               \
+        e = set_attrs<F, B, 4>();
+    MXG_ATTR4(0, 16) MXG_ATTR4(0, 32) MXG_ATTR4(0, 64) MXG_ATTR4(1, 16) MXG_ATTR4(1, 32) MXG_ATTR4(1, 64)
+#undef MXG_ATTR4
     return e;
 }
 
@@ -913,13 +949,23 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
         pl.P = M;
         pl.Q = N;
         pl.bn = 128;
+        // measurement knob: MXGEMM_BN=256 selects 128x256 output tiles
+        if (const char *e = getenv("MXGEMM_BN"))
+            if (atoi(e) == 256 && N >= 256)
+                pl.bn = 256;
     }
     // Two 128-byte K chunks per stage halve the TMA operations per byte (each
     // costs ~0.2 us of the SM's copy engine); rows must be whole chunks.
     const int64_t chunks = (row_bytes(fmt, K) + 127) / 128;
-    pl.kc = (row_bytes(fmt, K) % 128 == 0 && chunks >= 2) ? 2 : 1;
-    if (force_kc == 1 || (force_kc == 2 && pl.kc == 2))
+    const bool whole = row_bytes(fmt, K) % 128 == 0;
+    pl.kc = (whole && chunks >= 2) ? 2 : 1;
+    // 64-column decode tiles: four chunks per stage measured faster
+    if (whole && pl.swap && pl.bn == 64 && chunks >= 4)
+        pl.kc = 4;
+    if (force_kc == 1 || (force_kc == 2 && whole))
         pl.kc = force_kc;
+    if (force_kc == 4 && whole && pl.bn <= 64)
+        pl.kc = 4;
     pl.stages = stages_for(fmt, pl.bn, pl.kc);
     pl.tilesP = (pl.P + 127) / 128;
     pl.tilesQ = (pl.Q + pl.bn - 1) / pl.bn;
@@ -980,6 +1026,9 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
 cudaError_t launch_gemm(const GemmPlan &plan, const GemmBuffers &buf, uint64_t wait_limit_ns, int inject, int pdl,
                         cudaStream_t stream)
 {
+    if (plan.kc == 4)
+        return plan.fmt == kFmtMXFP8 ? dispatch_bn4<0>(plan, buf, wait_limit_ns, inject, pdl, stream)
+                                     : dispatch_bn4<1>(plan, buf, wait_limit_ns, inject, pdl, stream);
     if (plan.fmt == kFmtMXFP8)
         return plan.kc == 1 ? dispatch_bn<0, 1>(plan, buf, wait_limit_ns, inject, pdl, stream)
                             : dispatch_bn<0, 2>(plan, buf, wait_limit_ns, inject, pdl, stream);

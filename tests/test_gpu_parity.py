@@ -96,11 +96,13 @@ def test_gemm_forced_schedules(fmt, sched, M, N, K):
 
 
 @pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
-@pytest.mark.parametrize("kc", [1, 2])
-@pytest.mark.parametrize("M,N,K", [(32, 512, 1024), (200, 384, 640), (64, 256, 384), (130, 256, 896)])
+@pytest.mark.parametrize("kc", [1, 2, 4])
+@pytest.mark.parametrize("M,N,K", [(32, 512, 1024), (200, 384, 640), (64, 256, 384), (130, 256, 896),
+                                   (16, 640, 2560)])
 def test_gemm_k_chunks_per_stage(fmt, kc, M, N, K):
-    """One and two 128-byte K chunks per pipeline stage (2-D and 3-D TMA
-    boxes), including K whose last stage is partly past the end of a row."""
+    """One, two and four 128-byte K chunks per pipeline stage (2-D and 3-D
+    TMA boxes), including K whose last stage is partly past the end of a
+    row; four chunks apply to tiles of at most 64 columns."""
     h = handle()
     h.set_kchunks(kc)
     try:

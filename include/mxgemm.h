@@ -67,7 +67,8 @@ enum {
     MXGEMM_ERR_UNSUPPORTED_DEVICE = 3, /* current device is not compute capability 10.0 */
     MXGEMM_ERR_OOM = 4,                /* workspace allocation failed */
     MXGEMM_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
-    MXGEMM_ERR_TIMEOUT = 6             /* a kernel gave up on a bounded wait */
+    MXGEMM_ERR_TIMEOUT = 6,            /* a kernel gave up on a bounded wait */
+    MXGEMM_ERR_TOO_LARGE = 7           /* exceeds mxgemm_run_noalloc's fixed scratch */
 };
 
 /* Schedules for the GEMM's persistent tile scheduler (mxgemm_set_schedule). */
@@ -161,6 +162,31 @@ MXGEMM_API int mxgemm_set_wait_limit(mxgemm_handle h, uint64_t ns);
  * out and the kernel reports MXGEMM_ERR_TIMEOUT through
  * mxgemm_check_device_error.  The hook disarms itself after one launch. */
 MXGEMM_API int mxgemm_debug_inject(mxgemm_handle h, int mode);
+
+/* mxgemm_run without a handle and without allocating device memory, for
+ * callers that cannot call cudaMalloc when they run the product: code inside
+ * an allocator or memory-pool hook that must not re-enter the allocator, or
+ * runtimes that make every allocation up front.  (The pages have no
+ * counterpart; this is a property of this library's interface.)
+ *
+ * Same operation, layouts and requirements as mxgemm_run, except:
+ *  - the repacked scales live in a fixed 8 MiB array inside the library
+ *    (held by every GPU that loads it until exit): (ceil(M/256) +
+ *    ceil(N/256)) * 2 * ka * 512 bytes must fit, where ka = K/128 rounded up
+ *    to a multiple of 4 (MXFP8) or 8 (MXFP4); larger problems return
+ *    MXGEMM_ERR_TOO_LARGE and launch nothing;
+ *  - the GEMM always computes whole output tiles (no split-K);
+ *  - the first call on a device sets that device up (checks it is sm_100,
+ *    looks up the array's device address); make that first call before any
+ *    stream capture;
+ *  - all calls share the array: calls whose work overlaps on the GPU race
+ *    and give wrong results, so order them on one stream;
+ *  - device timeouts of the bounded waits are not reported.
+ * Buffers are device memory; `stream` is a cudaStream_t. */
+MXGEMM_API int mxgemm_run_noalloc(int fmt, int64_t M, int64_t N, int64_t K,
+                       const void *A, const uint8_t *A_scales,
+                       const void *B, const uint8_t *B_scales,
+                       void *C, void *stream);
 
 /* Static description of a status code. */
 MXGEMM_API const char *mxgemm_status_string(int status);

@@ -20,7 +20,7 @@ ROOT = os.path.dirname(HERE)
 OUT = os.path.join(HERE, "libmxgemm.so")
 BUILD = os.path.join(ROOT, "_build")
 
-SOURCES = ["api.cu", "gemm.cu", "quant.cu", "repack.cu"]
+SOURCES = ["api.cu", "gemm.cu", "quant.cu", "repack.cu", "noalloc.cu"]
 HEADERS = ["mx_internal.h", "sm100_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

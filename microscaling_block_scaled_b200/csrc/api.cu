@@ -170,6 +170,7 @@ const char *mxgemm_status_string(int status)
     case MXGEMM_ERR_OOM: return "workspace allocation failed";
     case MXGEMM_ERR_CUDA: return "CUDA call failed";
     case MXGEMM_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case MXGEMM_ERR_TOO_LARGE: return "problem exceeds the fixed scratch of mxgemm_run_noalloc (8 MiB of scales)";
     default: return "unknown status";
     }
 }

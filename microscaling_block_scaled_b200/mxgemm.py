@@ -27,6 +27,7 @@ ERR_UNSUPPORTED_DEVICE = 3
 ERR_OOM = 4
 ERR_CUDA = 5
 ERR_TIMEOUT = 6
+ERR_TOO_LARGE = 7
 
 # Entry points and their C signatures (restype, argtypes).
 _i64 = ctypes.c_int64
@@ -45,6 +46,7 @@ SIGNATURES = {
     "mxgemm_check_device_error": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_int)]),
     "mxgemm_set_wait_limit": (ctypes.c_int, [_vp, ctypes.c_uint64]),
     "mxgemm_debug_inject": (ctypes.c_int, [_vp, ctypes.c_int]),
+    "mxgemm_run_noalloc": (ctypes.c_int, [ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "mxgemm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mxgemm_version": (ctypes.c_char_p, []),
 }
@@ -128,6 +130,24 @@ def mxgemm_gemm(h, fmt, M, N, K, A, B, C, stream) -> int:
 
 def mxgemm_run_host(h, fmt, M, N, K, A, SA, B, SB, C, stream) -> int:
     return load().mxgemm_run_host(h, fmt, M, N, K, A, SA, B, SB, C, stream)
+
+
+def mxgemm_run_noalloc(fmt, M, N, K, A, SA, B, SB, C, stream) -> int:
+    return load().mxgemm_run_noalloc(fmt, M, N, K, A, SA, B, SB, C, stream)
+
+
+def run_noalloc(fmt, A, SA, B, SB, C=None, K=None, stream=None):
+    """mxgemm_run_noalloc on torch CUDA tensors (no handle, no device
+    allocation inside the library); returns C (bfloat16 [M][N])."""
+    import torch
+    M, N = A.shape[0], B.shape[0]
+    if K is None:
+        K = SA.shape[1] * 32
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _check("mxgemm_run_noalloc", mxgemm_run_noalloc(fmt, M, N, K, _ptr(A), _ptr(SA), _ptr(B), _ptr(SB), _ptr(C),
+                                                    _stream_ptr(stream)))
+    return C
 
 
 def mxgemm_quantize(fmt, R, K, X, Q, S, stream) -> int:

@@ -360,9 +360,9 @@ int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t
     const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks);
     static const char *names[] = {"auto", "dp", "splitk", "streamk"};
     snprintf(buf, cap,
-             "fmt=%d swap=%d BN=%d kc=%d stages=%d tiles=%lld kt=%lld workers=%lld grid=%d sched=%s "
+             "fmt=%d swap=%d pair=%d BN=%d kc=%d stages=%d tiles=%lld kt=%lld workers=%lld grid=%d sched=%s "
              "partial_bytes=%lld",
-             pl.fmt, pl.swap, pl.bn, pl.kc, pl.stages, static_cast<long long>(pl.tiles), static_cast<long long>(pl.kt),
+             pl.fmt, pl.swap, pl.pair, pl.bn, pl.kc, pl.stages, static_cast<long long>(pl.tiles), static_cast<long long>(pl.kt),
              static_cast<long long>(pl.workers), pl.grid, names[pl.sched & 3],
              static_cast<long long>(pl.partial_bytes));
     return MXGEMM_OK;

@@ -125,6 +125,8 @@ struct KParams {
     int swap;
     int inject;
     int tma_store;         // 1: epilogue stores C through shared memory with TMA
+    const uint8_t *opP;    // the MMA row operand (for whole-tile L2 prefetch)
+    int64_t rbytes;        // bytes per operand row
 };
 
 // Error site codes written to the device error word.
@@ -269,8 +271,9 @@ __device__ __forceinline__ void store_bf16(const OutView o, int64_t p, int64_t q
 }
 
 template <int FMT, int BN, int KC>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(224, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
+                   const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
                    const __grid_constant__ CUtensorMap tmC, const KParams kp_in)
 {
     using C_ = Cfg<FMT, BN, KC>;
@@ -303,9 +306,11 @@ __global__ void __launch_bounds__(192, 1)
     if (threadIdx.x == 0) {
         tma_prefetch_desc(&tmP);
         tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmSP);
+        tma_prefetch_desc(&tmSQ);
         tma_prefetch_desc(&tmC);
         for (int s = 0; s < S; ++s) {
-            mbar_init(full_bar(s), 1);
+            mbar_init(full_bar(s), 2);          // one arming per producer warp
             mbar_init(empty_bar(s), 1);
         }
         for (int a = 0; a < C_::kNumAcc; ++a) {
@@ -330,96 +335,78 @@ __global__ void __launch_bounds__(192, 1)
     const Sched sc{kp.iters, kp.workers, kp.kt, kp.tilesP, kp.dp != 0};
     const uint32_t W = sc.W;
 
-    // Everything except the producer's first operand loads may depend on the
+    // Everything except the producers' first operand loads may depend on the
     // preceding kernel in the stream (the scale repack, or the previous GEMM
     // that used the same workspace): wait for it here.  Without a
     // programmatic launch this returns at once.
-    if (warp != 0)
+    if (warp != 0 && warp != 6)
         grid_dependency_wait();
 
-    if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
-        // L2 policy per operand: in the swapped (decode) form the weights
-        // stream through once and the small activation is re-read by every
-        // tile; otherwise both operands are re-read across tiles.
-        const uint64_t polP = kp.swap ? policy_evict_first() : policy_evict_normal();
-        const uint64_t polQ = kp.swap ? policy_evict_last() : policy_evict_normal();
-        uint32_t armed = 0;         // stages armed so far (round-robin over the ring)
-        int skipped_stage = -1;
-        bool inject = kp.inject == 1;
-        bool ok = true;
-        auto load_operands = [&](int s, uint32_t tile, uint32_t k) {
-            const uint32_t tq = tile / sc.tilesP, tp = tile - tq * sc.tilesP;
-            const uint32_t fb = full_bar(s);
-            if constexpr (KC == 1) {       // 2-D maps: x = byte offset along K
-                const int32_t x = static_cast<int32_t>(k * 128);
-                tma_load_2d(sbase + C_::kOffA + s * C_::kABytes, &tmP, x, static_cast<int32_t>(tp) * 128, fb,
-                            polP);
-                tma_load_2d(sbase + C_::kOffB + s * C_::kBBytes, &tmQ, x, static_cast<int32_t>(tq) * BN, fb,
-                            polQ);
-            } else {                       // 3-D maps: {byte in chunk, row, 128-byte K chunk}
-                const int32_t z = static_cast<int32_t>(k * KC);
-                tma_load_3d(sbase + C_::kOffA + s * C_::kABytes, &tmP, 0, static_cast<int32_t>(tp) * 128, z, fb,
-                            polP);
-                tma_load_3d(sbase + C_::kOffB + s * C_::kBBytes, &tmQ, 0, static_cast<int32_t>(tq) * BN, z, fb,
-                            polQ);
-            }
-        };
-        auto load_scales = [&](int s, uint32_t tile, uint32_t k) {
-            const uint32_t tq = tile / sc.tilesP, tp = tile - tq * sc.tilesP;
-            const uint32_t fb = full_bar(s);
-            const uint8_t *sfa = kp.sfP + (static_cast<int64_t>(tp) * kp.kaP + k * C_::kAtoms) * 512;
-            bulk_load(sbase + C_::kOffSFA + s * C_::kSFABytes, sfa, C_::kSFABytes, fb);
-            const int64_t rb0 = (static_cast<int64_t>(tq) * BN) / 128;
-#pragma unroll
-            for (int rb = 0; rb < C_::kRBQ; ++rb) {
-                const uint8_t *sfb = kp.sfQ + ((rb0 + rb) * kp.kaQ + k * C_::kAtoms) * 512;
-                bulk_load(sbase + C_::kOffSFB + s * C_::kSFBBytes + rb * C_::kAtoms * 512, sfb, C_::kAtoms * 512,
-                          fb);
-            }
-        };
+    if (warp == 0 || warp == 6) {
+        // ----------------------------------------------------- TMA producers
+        // Warp 0 loads the MMA row operand and its scale atoms, warp 6 the
+        // column operand and its scale atoms; each arms the stage's full
+        // barrier for its own bytes.  Every TMA operation costs the issuing
+        // thread and the SM's copy engine a fixed ~0.1-0.2 us, so two issuing
+        // threads and one box per operand (scales included) per stage.
+        // L2 policy: in the swapped (decode) form the weights stream through
+        // once and the small activation is re-read by every tile; otherwise
+        // both operands are re-read across tiles.
+        const bool sideP = warp == 0;
         if (lane == 0) {
-            IterCursor cur(sc, blockIdx.x, gridDim.x);
-            const uint32_t n_total = cur.total();
-            // Pass 1: the operand tiles of the first stage, which do not depend
-            // on the preceding kernel (the ring is empty, no wait needed).
-            // Only one stage: its scales queue behind whatever is issued here,
-            // and the first stage's latency is on the critical path.
-            const uint32_t n_pre = n_total < 1u ? n_total : 1u;
-            for (uint32_t n = 0; n < n_pre; ++n, cur.advance()) {
-                const int s = static_cast<int>(n);
-                if (inject && n == 0) {
-                    skipped_stage = s;          // test hook: leave this stage unarmed
-                } else {
-                    mbar_arrive_expect_tx(full_bar(s), C_::kTxBytes);
-                    load_operands(s, cur.tile, cur.k);
-                }
-                ++armed;
-            }
-            grid_dependency_wait();
-            // Pass 2: the scales of those stages.
-            IterCursor cur2(sc, blockIdx.x, gridDim.x);
-            for (uint32_t n = 0; n < n_pre; ++n, cur2.advance())
-                if (static_cast<int>(n) != skipped_stage)
-                    load_scales(static_cast<int>(n), cur2.tile, cur2.k);
-            // Pass 3: the rest, one ring slot at a time.
-            int s = static_cast<int>(n_pre % S);
-            uint32_t ph = 0u;
-            for (uint32_t n = n_pre; n < n_total; ++n, cur.advance()) {
+            const uint64_t pol = sideP ? (kp.swap ? policy_evict_first() : policy_evict_normal())
+                                       : (kp.swap ? policy_evict_last() : policy_evict_normal());
+            const CUtensorMap *tmOp = sideP ? &tmP : &tmQ;
+            const CUtensorMap *tmSf = sideP ? &tmSP : &tmSQ;
+            const uint32_t opBytes = sideP ? C_::kABytes : C_::kBBytes;
+            const uint32_t sfBytes = sideP ? C_::kSFABytes : C_::kSFBBytes;
+            const uint32_t offOp = sideP ? C_::kOffA : C_::kOffB;
+            const uint32_t offSf = sideP ? C_::kOffSFA : C_::kOffSFB;
+            uint32_t armed = 0;         // stages armed so far (round-robin over the ring)
+            int skipped_stage = -1;
+            bool inject = sideP && kp.inject == 1;
+            bool first = true;
+            int s = 0;
+            uint32_t ph = 0;
+            for (IterCursor cur(sc, blockIdx.x, gridDim.x); cur.valid(); cur.advance()) {
                 if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns)) {
                     record_error(kp.error, kErrProducerEmpty, s_abort);
-                    ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(full_bar(s), C_::kTxBytes);
-                load_operands(s, cur.tile, cur.k);
-                load_scales(s, cur.tile, cur.k);
+                const uint32_t tq = cur.tile / sc.tilesP, tp = cur.tile - tq * sc.tilesP;
+                const int32_t row = sideP ? static_cast<int32_t>(tp) * 128 : static_cast<int32_t>(tq) * BN;
+                const int32_t sf_rb = sideP ? static_cast<int32_t>(tp) : static_cast<int32_t>((tq * BN) / 128);
+                const uint32_t fb = full_bar(s);
+                if (inject) {
+                    inject = false;             // test hook: leave this stage unarmed
+                    skipped_stage = s;
+                    if (first) {
+                        grid_dependency_wait();
+                        first = false;
+                    }
+                } else {
+                    mbar_arrive_expect_tx(fb, opBytes + sfBytes);
+                    if constexpr (KC == 1)      // 2-D maps: x = byte offset along K
+                        tma_load_2d(sbase + offOp + s * opBytes, tmOp, static_cast<int32_t>(cur.k * 128), row, fb,
+                                    pol);
+                    else                        // 3-D maps: {byte in chunk, row, 128-byte K chunk}
+                        tma_load_3d(sbase + offOp + s * opBytes, tmOp, 0, row, static_cast<int32_t>(cur.k * KC),
+                                    fb, pol);
+                    if (first) {                // the first operand tile may overlap the preceding kernel
+                        grid_dependency_wait();
+                        first = false;
+                    }
+                    tma_load_3d(sbase + offSf + s * sfBytes, tmSf, 0, static_cast<int32_t>(cur.k * C_::kAtoms),
+                                sf_rb, fb, pol);
+                }
                 ++armed;
                 if (++s == S) {
                     s = 0;
                     ph ^= 1u;
                 }
             }
+            if (first)
+                grid_dependency_wait();
             // Let every armed copy land before the CTA can exit: wait for the
             // latest armed phase of each stage (already complete on the normal
             // path, where the MMA warp consumed every stage).
@@ -432,7 +419,6 @@ __global__ void __launch_bounds__(192, 1)
                 if (!mbar_wait_bounded(full_bar(st), parity, &dummy_abort, kp.limit_ns))
                     atomicCAS(kp.error, 0, kErrDrain);
             }
-            (void)ok;
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -540,7 +526,7 @@ __global__ void __launch_bounds__(192, 1)
                 atomicCAS(kp.error, 0, kErrDrain);
         }
         __syncwarp();
-    } else {
+    } else if (warp >= 2 && warp <= 5) {
         // ---------------------------------------------------------- epilogue
         const int quad = warp & 3;             // TMEM lanes 32*quad .. +31
         const int row = quad * 32 + lane;      // accumulator row = MMA row in tile
@@ -549,6 +535,7 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t acc_ph = 0;
         uint32_t out_chunks = 0;               // BF16 chunks staged so far (buffer = parity)
         bool stop = false;
+
 
         // Convert one CW-column chunk of the tile (this thread's row) to BF16
         // and write it to C: through shared memory and a TMA store when the
@@ -603,7 +590,7 @@ __global__ void __launch_bounds__(192, 1)
                 const int64_t tp = sg.tp, tq = sg.tq;
                 int good = 1;
                 if (lane == 0)
-                    good = mbar_wait_bounded(accf_bar(acc), acc_ph, s_abort, kp.limit_ns);
+                    good = mbar_wait_sleepy(accf_bar(acc), acc_ph, s_abort, kp.limit_ns, 200);
                 good = __shfl_sync(0xffffffffu, good, 0);
                 if (!good && lane == 0)
                     record_error(kp.error, kErrEpiAccFull, s_abort);
@@ -616,16 +603,35 @@ __global__ void __launch_bounds__(192, 1)
                 const uint32_t t_acc = tmem + acc * BN + (static_cast<uint32_t>(quad * 32) << 16);
                 const uint32_t g_first = sc.dp ? tile : sc.owner(tile * sc.KT);
                 const uint32_t g_last = sc.dp ? tile : sc.owner(tile * sc.KT + sc.KT - 1);
+                bool released = false;
                 if (g_first == g_last) {
-#pragma unroll 1
+                    // Drain the accumulator row into registers as BF16 pairs and
+                    // hand the accumulator back before any store, so the next
+                    // tile's MMAs overlap this tile's output traffic.
+                    uint32_t packed[BN / 2];
+#pragma unroll
                     for (int c = 0; c < BN; c += CW) {
                         uint32_t r[CW];
                         tmem_ld_cols<CW>(t_acc + c, r);
                         tmem_ld_wait();
-                        float v[CW];
 #pragma unroll
-                        for (int j = 0; j < CW; ++j)
-                            v[j] = __uint_as_float(r[j]);
+                        for (int j = 0; j < CW / 2; ++j)
+                            packed[c / 2 + j] =
+                                pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(acce_bar(acc));
+                    released = true;
+#pragma unroll
+                    for (int c = 0; c < BN; c += CW) {
+                        float v[CW];     // BF16 values widened back exactly
+#pragma unroll
+                        for (int j = 0; j < CW / 2; ++j) {
+                            v[2 * j] = __uint_as_float(packed[c / 2 + j] << 16);
+                            v[2 * j + 1] = __uint_as_float(packed[c / 2 + j] & 0xFFFF0000u);
+                        }
                         emit(v, tp, tq * BN + c);
                     }
                 } else {
@@ -687,10 +693,12 @@ __global__ void __launch_bounds__(192, 1)
                         }
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(acce_bar(acc));
+                if (!released) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(acce_bar(acc));
+                }
                 if (++acc == C_::kNumAcc) {
                     acc = 0;
                     acc_ph ^= 1u;
@@ -709,6 +717,380 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     if (warp == 1)
         tmem_dealloc(tmem, C_::kTmemCols);
+}
+
+// ------------------------------------------------------ CTA-pair kernel
+//
+// Large-M form: a cluster of two CTAs computes a 256x256 output tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256).  Each CTA loads its own 128
+// rows of A and its own 128 rows of B (no multicast), the scale atoms of its
+// A rows and of all 256 B rows; the even CTA (the leader) issues the scale
+// copies and MMAs for both and its commits arrive in both CTAs.  Per CTA this
+// halves the operand bytes per MMA against a 128x256 tile on one SM.
+//
+// Hand-offs across the pair: the odd CTA's MMA warp is idle, so it relays
+// "my stage has landed" to the leader (wait on its own full barrier, then a
+// cluster-scope remote arrive); both CTAs' epilogues tell the leader when the
+// accumulator may be reused with remote arrives as well.
+
+template <int FMT, int KC>
+struct PairCfg {
+    static constexpr int kAtomsPerChunk = FMT == kFmtMXFP8 ? 1 : 2;
+    static constexpr int kAtoms = kAtomsPerChunk * KC;
+    static constexpr int kChunk = 128 * 128;                  // 128 rows x 128 bytes of K
+    static constexpr int kABytes = kChunk * KC;               // this CTA's 128 rows of A
+    static constexpr int kBBytes = kChunk * KC;               // this CTA's 128 rows of B
+    static constexpr int kSFABytes = kAtoms * 512;            // scales of this CTA's A rows
+    static constexpr int kSFBBytes = 2 * kAtoms * 512;        // scales of all 256 B rows
+    static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
+    static constexpr int kCW = 32;
+    static constexpr int kOutBytes = 128 * kCW * 2;
+    static constexpr int kSmemBudget = 227 * 1024 - 2048 - 2 * kOutBytes;
+    static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
+    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
+    static constexpr int kSFACols = kAtoms * 4;
+    static constexpr int kSFBCols = 2 * kAtoms * 4;
+    static constexpr int kAccCols = 256;
+    static constexpr int kTmemCols = 512;
+    static constexpr uint32_t kTxBytes = kStageBytes;
+    static constexpr int kOffA = 0;
+    static constexpr int kOffB = kOffA + kStages * kABytes;
+    static constexpr int kOffSFA = kOffB + kStages * kBBytes;
+    static constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
+    static constexpr int kOffOut = (kOffSFB + kStages * kSFBBytes + 1023) / 1024 * 1024;
+    static constexpr int kOffBar = kOffOut + 2 * kOutBytes;
+    static constexpr int kNumBars = 3 * kStages + 3;         // full, empty, pair_full; accf, acce, drain
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+
+    static_assert(kStages >= 2, "at least two pipeline stages");
+    static_assert(kAccCols + kStages * (kSFACols + kSFBCols) <= kTmemCols, "TMEM budget");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+template <int FMT>
+__host__ __device__ constexpr uint32_t idesc_pair()
+{
+    constexpr uint32_t t = FMT == kFmtMXFP8 ? 0u : 1u;
+    return (t << 7) | (t << 10) | (static_cast<uint32_t>(256 >> 3) << 17) | (1u << 23) |
+           (static_cast<uint32_t>(256 >> 4) << 24);
+}
+
+template <int FMT, int KC>
+__global__ void __launch_bounds__(224, 1)
+    mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
+                        const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
+                        const __grid_constant__ CUtensorMap tmC, const KParams kp_in)
+{
+    using C_ = PairCfg<FMT, KC>;
+    constexpr int S = C_::kStages;
+    constexpr int CW = C_::kCW;
+    const KParams kp = kp_in;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + C_::kOffBar;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+    auto pfull_bar = [&](int s) { return bar0 + 8u * (2 * S + s); };
+    const uint32_t accf_bar = bar0 + 8u * (3 * S);
+    const uint32_t acce_bar = bar0 + 8u * (3 * S + 1);
+    const uint32_t drain_bar = bar0 + 8u * (3 * S + 2);
+    volatile uint32_t *s_tmem = reinterpret_cast<volatile uint32_t *>(smem + C_::kOffMisc);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C_::kOffMisc + 4);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const uint32_t pair = blockIdx.x / 2, npairs = gridDim.x / 2;
+    const uint32_t tiles = kp.workers, tilesP = kp.tilesP, KT = kp.kt;
+
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&tmP);
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmSP);
+        tma_prefetch_desc(&tmSQ);
+        tma_prefetch_desc(&tmC);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full_bar(s), 2);          // one arming per producer warp
+            mbar_init(empty_bar(s), 1);
+            mbar_init(pfull_bar(s), 1);
+        }
+        mbar_init(accf_bar, 1);
+        mbar_init(acce_bar, 8);
+        mbar_init(drain_bar, 1);
+        *s_abort = 0;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(sbase + C_::kOffMisc, C_::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp != 0 && warp != 6)
+        grid_dependency_wait();
+
+    if (warp == 0 || warp == 6) {
+        // ----------------------------------------------------- TMA producers
+        // Warp 0: this CTA's 128 rows of A and their scale atoms; warp 6: its
+        // 128 rows of B and the scale atoms of all 256 B rows of the tile.
+        const bool sideA = warp == 0;
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_normal();
+            const CUtensorMap *tmOp = sideA ? &tmP : &tmQ;
+            const CUtensorMap *tmSf = sideA ? &tmSP : &tmSQ;
+            const uint32_t opBytes = sideA ? C_::kABytes : C_::kBBytes;
+            const uint32_t sfBytes = sideA ? C_::kSFABytes : C_::kSFBBytes;
+            const uint32_t offOp = sideA ? C_::kOffA : C_::kOffB;
+            const uint32_t offSf = sideA ? C_::kOffSFA : C_::kOffSFB;
+            uint32_t armed = 0;
+            int skipped_stage = -1;
+            bool inject = sideA && kp.inject == 1;
+            int s = 0;
+            uint32_t ph = 0;
+            bool first = true;
+            for (uint32_t tile = pair; tile < tiles; tile += npairs) {
+                const uint32_t tq = tile / tilesP, tp = tile - tq * tilesP;
+                const int32_t row = static_cast<int32_t>((sideA ? tp : tq) * 256 + rank * 128);
+                const int32_t sf_rb = sideA ? static_cast<int32_t>(tp * 2 + rank) : static_cast<int32_t>(tq * 2);
+                bool ok = true;
+                for (uint32_t k = 0; k < KT; ++k) {
+                    if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns)) {
+                        record_error(kp.error, kErrProducerEmpty, s_abort);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = full_bar(s);
+                    if (inject) {
+                        inject = false;
+                        skipped_stage = s;
+                    } else {
+                        mbar_arrive_expect_tx(fb, opBytes + sfBytes);
+                        if constexpr (KC == 1)
+                            tma_load_2d(sbase + offOp + s * opBytes, tmOp, static_cast<int32_t>(k * 128), row, fb, pol);
+                        else
+                            tma_load_3d(sbase + offOp + s * opBytes, tmOp, 0, row, static_cast<int32_t>(k * KC), fb,
+                                        pol);
+                        if (first) {            // operands of stage 0 may overlap the preceding kernel
+                            grid_dependency_wait();
+                            first = false;
+                        }
+                        tma_load_3d(sbase + offSf + s * sfBytes, tmSf, 0, static_cast<int32_t>(k * C_::kAtoms),
+                                    sf_rb, fb, pol);
+                    }
+                    ++armed;
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+            }
+            if (first)
+                grid_dependency_wait();
+            for (int st = 0; st < S; ++st) {
+                const uint32_t n = armed / S + (static_cast<uint32_t>(st) < armed % S ? 1u : 0u);
+                if (n == 0 || (st == skipped_stage && n == 1))
+                    continue;
+                int dummy_abort = 0;
+                if (!mbar_wait_bounded(full_bar(st), (n - 1) & 1u, &dummy_abort, kp.limit_ns))
+                    atomicCAS(kp.error, 0, kErrDrain);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1 && !leader) {
+        // ------------------------------------- relay: this CTA's stages landed
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (uint32_t tile = pair; tile < tiles && ok; tile += npairs) {
+                for (uint32_t k = 0; k < KT; ++k) {
+                    if (!mbar_wait_bounded(full_bar(s), ph, s_abort, kp.limit_ns)) {
+                        record_error(kp.error, kErrMmaFull, s_abort);
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_remote(pfull_bar(s), 0);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------- MMA issuer (leader CTA)
+        constexpr uint32_t kIdesc = idesc_pair<FMT>();
+        const uint32_t t_sfa0 = tmem + C_::kAccCols;
+        const uint32_t t_sfb0 = t_sfa0 + S * C_::kSFACols;
+        int s = 0;
+        uint32_t ph = 0;
+        uint32_t acc_ph = 0;
+        bool ok = true;
+        for (uint32_t tile = pair; tile < tiles && ok; tile += npairs) {
+            int good = 1;
+            if (lane == 0)
+                good = mbar_wait_cluster_bounded(acce_bar, acc_ph ^ 1u, s_abort, kp.limit_ns);
+            good = __shfl_sync(0xffffffffu, good, 0);
+            if (!good) {
+                if (lane == 0)
+                    record_error(kp.error, kErrMmaAccEmpty, s_abort);
+                break;
+            }
+            tc_fence_after();
+            for (uint32_t k = 0; k < KT; ++k) {
+                good = 1;
+                if (lane == 0) {
+                    good = mbar_wait_bounded(full_bar(s), ph, s_abort, kp.limit_ns);
+                    if (good)
+                        good = mbar_wait_cluster_bounded(pfull_bar(s), ph, s_abort, kp.limit_ns);
+                }
+                good = __shfl_sync(0xffffffffu, good, 0);
+                if (!good) {
+                    if (lane == 0)
+                        record_error(kp.error, kErrMmaFull, s_abort);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t t_sfa = t_sfa0 + s * C_::kSFACols;
+                    const uint32_t t_sfb = t_sfb0 + s * C_::kSFBCols;
+                    const uint32_t s_sfa = sbase + C_::kOffSFA + s * C_::kSFABytes;
+                    const uint32_t s_sfb = sbase + C_::kOffSFB + s * C_::kSFBBytes;
+#pragma unroll
+                    for (int a = 0; a < C_::kAtoms; ++a)
+                        tmem_cp_32x128b_x4_pair(t_sfa + 4 * a, sdesc_rows16(s_sfa + 512 * a));
+#pragma unroll
+                    for (int rb = 0; rb < 2; ++rb)
+#pragma unroll
+                        for (int a = 0; a < C_::kAtoms; ++a)
+                            tmem_cp_32x128b_x4_pair(t_sfb + a * 8 + 4 * rb,
+                                                    sdesc_rows16(s_sfb + (rb * C_::kAtoms + a) * 512));
+#pragma unroll
+                    for (int c = 0; c < KC; ++c) {
+                        const uint64_t adesc = sdesc_sw128_kmajor(sbase + C_::kOffA + s * C_::kABytes + c * C_::kChunk);
+                        const uint64_t bdesc = sdesc_sw128_kmajor(sbase + C_::kOffB + s * C_::kBBytes + c * C_::kChunk);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int atom = FMT == kFmtMXFP8 ? c : 2 * c + j / 2;
+                            const uint32_t sf_id = FMT == kFmtMXFP8 ? j : 2 * (j % 2);
+                            const uint32_t idesc = kIdesc | (sf_id << 4) | (sf_id << 29);
+                            const uint32_t acc_flag = (k > 0 || c > 0 || j > 0) ? 1u : 0u;
+                            const uint64_t koff = static_cast<uint64_t>(j * 32) >> 4;
+                            if (FMT == kFmtMXFP8)
+                                mma_mxf8f6f4_pair(tmem, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
+                                                  t_sfb + atom * 8, acc_flag);
+                            else
+                                mma_mxf4_pair(tmem, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
+                                              t_sfb + atom * 8, acc_flag);
+                        }
+                    }
+                    tc_commit_pair(empty_bar(s), 0x3);
+                }
+                __syncwarp();
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (!ok)
+                break;
+            if (lane == 0)
+                tc_commit_pair(accf_bar, 0x3);
+            __syncwarp();
+            acc_ph ^= 1u;
+        }
+        if (lane == 0) {
+            tc_commit_pair(drain_bar, 0x1);
+            int dummy_abort = 0;
+            if (!mbar_wait_bounded(drain_bar, 0, &dummy_abort, kp.limit_ns))
+                atomicCAS(kp.error, 0, kErrDrain);
+        }
+        __syncwarp();
+    } else if (warp >= 2 && warp <= 5) {
+        // ---------------------------------------------------------- epilogue
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const int etid = threadIdx.x - 64;
+        uint32_t acc_ph = 0;
+        uint32_t out_chunks = 0;
+        for (uint32_t tile = pair; tile < tiles; tile += npairs) {
+            const uint32_t tq = tile / tilesP, tp = tile - tq * tilesP;
+            int good = 1;
+            if (lane == 0)
+                good = mbar_wait_sleepy(accf_bar, acc_ph, s_abort, kp.limit_ns, 200);
+            good = __shfl_sync(0xffffffffu, good, 0);
+            if (!good && lane == 0)
+                record_error(kp.error, kErrEpiAccFull, s_abort);
+            if (named_bar_or(1, 128, (!good || *s_abort) ? 1 : 0))
+                break;
+            tc_fence_after();
+            const uint32_t t_acc = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+            // Drain the whole accumulator row into registers (BF16 pairs) and
+            // hand the accumulator back to the MMA warp before any store, so
+            // the next tile's MMAs overlap this tile's output traffic.
+            uint32_t packed[128];
+#pragma unroll
+            for (int c = 0; c < 256; c += CW) {
+                uint32_t r[CW];
+                tmem_ld_cols<CW>(t_acc + c, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < CW / 2; ++j)
+                    packed[c / 2 + j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader)
+                    mbar_arrive(acce_bar);
+                else
+                    mbar_arrive_remote(acce_bar, 0);
+            }
+#pragma unroll
+            for (int c = 0; c < 256; c += CW) {
+                const int b = static_cast<int>(out_chunks & 1u);
+                uint8_t *buf = smem + C_::kOffOut + b * C_::kOutBytes;
+                if (etid == 0)
+                    bulk_wait_group_read<1>();
+                named_bar_sync(1, 128);
+                uint4 *dst = reinterpret_cast<uint4 *>(buf + row * CW * 2);
+#pragma unroll
+                for (int j = 0; j < CW / 8; ++j)
+                    dst[j] = make_uint4(packed[c / 2 + 4 * j], packed[c / 2 + 4 * j + 1], packed[c / 2 + 4 * j + 2],
+                                        packed[c / 2 + 4 * j + 3]);
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (etid == 0) {
+                    tma_store_2d(&tmC, smem_u32(buf), static_cast<int32_t>(tq * 256 + c),
+                                 static_cast<int32_t>(tp * 256 + rank * 128));
+                    bulk_commit_group();
+                }
+                ++out_chunks;
+            }
+            acc_ph ^= 1u;
+        }
+        if (etid == 0)
+            bulk_wait_group<0>();
+    }
+
+    tc_fence_before();
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == 1)
+        tmem_dealloc_pair(tmem, C_::kTmemCols);
 }
 
 // ------------------------------------------------------------------- host
@@ -769,6 +1151,25 @@ bool make_operand_map_3d(CUtensorMap *map, const void *base, int64_t rows, int64
     return r == CUDA_SUCCESS;
 }
 
+// 3-D uint32 map over a repacked scale buffer [row blocks][ka][512 bytes]:
+// {128 words of an atom, atom, 128-row block}, box {128, atoms, row blocks}.
+bool make_sf_map(CUtensorMap *map, const uint8_t *base, int64_t ka, int64_t row_blocks, int atoms, int rbs)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[3] = {128u, static_cast<cuuint64_t>(ka), static_cast<cuuint64_t>(row_blocks)};
+    cuuint64_t strides[2] = {512u, static_cast<cuuint64_t>(ka) * 512u};
+    cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(atoms), static_cast<cuuint32_t>(rbs)};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+inline int64_t sf_row_blocks(int64_t rows) { return (rows + 255) / 256 * 2; }
+
 template <int FMT, int BN, int KC>
 cudaError_t set_attrs()
 {
@@ -818,6 +1219,12 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
                                : make_output_map(&tmC, b.C, 1, 8, 8, 1);
     if (!okC)
         return cudaErrorInvalidValue;
+    CUtensorMap tmSP, tmSQ;
+    const uint8_t *sfP = pl.swap ? b.sfB : b.sfA;
+    const uint8_t *sfQ = pl.swap ? b.sfA : b.sfB;
+    if (!make_sf_map(&tmSP, sfP, pl.kaP, sf_row_blocks(pl.P), C_::kAtoms, 1) ||
+        !make_sf_map(&tmSQ, sfQ, pl.kaQ, sf_row_blocks(pl.Q), C_::kAtoms, C_::kRBQ))
+        return cudaErrorInvalidValue;
     KParams kp;
     kp.sfP = pl.swap ? b.sfB : b.sfA;
     kp.sfQ = pl.swap ? b.sfA : b.sfB;
@@ -839,9 +1246,11 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     kp.swap = pl.swap;
     kp.inject = inject;
     kp.tma_store = tma_store;
+    kp.opP = static_cast<const uint8_t *>(Pptr);
+    kp.rbytes = rbytes;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(224);
     cfg.dynamicSmemBytes = C_::kSmemBytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -849,7 +1258,7 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, mx_gemm_kernel<FMT, BN, KC>, tmP, tmQ, tmC, kp);
+    return cudaLaunchKernelEx(&cfg, mx_gemm_kernel<FMT, BN, KC>, tmP, tmQ, tmSP, tmSQ, tmC, kp);
 }
 
 template <int FMT, int KC>
@@ -864,6 +1273,67 @@ cudaError_t dispatch_bn(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit
     case 256: return launch_t<FMT, 256, KC>(pl, b, limit_ns, inject, pdl, st);
     default: return cudaErrorInvalidValue;
     }
+}
+
+template <int FMT, int KC>
+cudaError_t launch_pair_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
+                          cudaStream_t st)
+{
+    using C_ = PairCfg<FMT, KC>;
+    const int64_t rbytes = row_bytes(FMT, pl.K);
+    CUtensorMap tmP, tmQ, tmC;
+    if (KC == 1) {
+        if (!make_operand_map(&tmP, b.A, pl.M, rbytes, 128) || !make_operand_map(&tmQ, b.B, pl.N, rbytes, 128))
+            return cudaErrorInvalidValue;
+    } else {
+        if (!make_operand_map_3d(&tmP, b.A, pl.M, rbytes, 128, KC) ||
+            !make_operand_map_3d(&tmQ, b.B, pl.N, rbytes, 128, KC))
+            return cudaErrorInvalidValue;
+    }
+    if (!make_output_map(&tmC, b.C, pl.M, pl.N, C_::kCW, 128))
+        return cudaErrorInvalidValue;
+    CUtensorMap tmSP, tmSQ;
+    if (!make_sf_map(&tmSP, b.sfA, pl.kaP, sf_row_blocks(pl.M), C_::kAtoms, 1) ||
+        !make_sf_map(&tmSQ, b.sfB, pl.kaQ, sf_row_blocks(pl.N), C_::kAtoms, 2))
+        return cudaErrorInvalidValue;
+    KParams kp;
+    kp.sfP = b.sfA;
+    kp.sfQ = b.sfB;
+    kp.C = reinterpret_cast<__nv_bfloat16 *>(b.C);
+    kp.partials = nullptr;
+    kp.counters = nullptr;
+    kp.error = b.error;
+    kp.P = pl.M;
+    kp.Q = pl.N;
+    kp.ldc = pl.N;
+    kp.tilesP = static_cast<uint32_t>(pl.tilesP);
+    kp.kt = static_cast<uint32_t>(pl.kt);
+    kp.iters = static_cast<uint32_t>(pl.iters);
+    kp.workers = static_cast<uint32_t>(pl.tiles);
+    kp.dp = 1;
+    kp.kaP = pl.kaP;
+    kp.kaQ = pl.kaQ;
+    kp.limit_ns = limit_ns;
+    kp.swap = 0;
+    kp.inject = inject;
+    kp.tma_store = 1;
+    kp.opP = static_cast<const uint8_t *>(b.A);
+    kp.rbytes = rbytes;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+    cfg.blockDim = dim3(224);
+    cfg.dynamicSmemBytes = C_::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, mx_gemm_pair_kernel<FMT, KC>, tmP, tmQ, tmSP, tmSQ, tmC, kp);
 }
 
 template <int FMT>
@@ -924,6 +1394,12 @@ cudaError_t prepare_gemm_kernels()
     MXG_ATTR(0, 16) MXG_ATTR(0, 32) MXG_ATTR(0, 64) MXG_ATTR(0, 128) MXG_ATTR(0, 256)
     MXG_ATTR(1, 16) MXG_ATTR(1, 32) MXG_ATTR(1, 64) MXG_ATTR(1, 128) MXG_ATTR(1, 256)
 #undef MXG_ATTR
+#define MXG_ATTRP(F, KCV)                                               \
+    if (e == cudaSuccess)                                               \
+        e = cudaFuncSetAttribute(mx_gemm_pair_kernel<F, KCV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                 PairCfg<F, KCV>::kSmemBytes);
+    MXG_ATTRP(0, 1) MXG_ATTRP(0, 2) MXG_ATTRP(1, 1) MXG_ATTRP(1, 2)
+#undef MXG_ATTRP
 #define MXG_ATTR4(F, B)                                                 \
     if (e == cudaSuccess)                                               \
         e = set_attrs<F, B, 4>();
@@ -966,6 +1442,38 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
         pl.kc = force_kc;
     if (force_kc == 4 && whole && pl.bn <= 64)
         pl.kc = 4;
+    // Large M: 256x256 tiles on CTA pairs (cta_group::2) when they fill the GPU.
+    {
+        const int64_t ptiles = ((M + 255) / 256) * ((N + 255) / 256);
+        const char *e = getenv("MXGEMM_PAIR");
+        const bool allow = !(e && atoi(e) == 0);
+        if (allow && !pl.swap && M >= 512 && N >= 256 && N % 8 == 0 && ptiles >= 64)
+            pl.pair = 1;
+    }
+    if (pl.pair) {
+        pl.bn = 256;
+        if (force_kc == 0)
+            pl.kc = (whole && chunks >= 2) ? 2 : 1;
+        else
+            pl.kc = (force_kc == 2 && whole) ? 2 : 1;
+        pl.stages = fmt == kFmtMXFP8 ? (pl.kc == 1 ? PairCfg<0, 1>::kStages : PairCfg<0, 2>::kStages)
+                                     : (pl.kc == 1 ? PairCfg<1, 1>::kStages : PairCfg<1, 2>::kStages);
+        pl.tilesP = (M + 255) / 256;
+        pl.tilesQ = (N + 255) / 256;
+        pl.kt = (chunks + pl.kc - 1) / pl.kc;
+        pl.tiles = pl.tilesP * pl.tilesQ;
+        pl.iters = pl.tiles * pl.kt;
+        const int64_t pairs = (num_sms > 0 ? num_sms : 2) / 2;
+        pl.workers = pl.tiles;
+        pl.grid = static_cast<int>(2 * (pl.tiles < pairs ? pl.tiles : pairs));
+        pl.sched = 1;
+        pl.kaP = sf_atoms_per_rowblock(fmt, K);
+        pl.kaQ = pl.kaP;
+        pl.partial_bytes = 0;
+        pl.counter_bytes = 4;
+        pl.valid = pl.iters < (int64_t(1) << 31);
+        return pl;
+    }
     pl.stages = stages_for(fmt, pl.bn, pl.kc);
     pl.tilesP = (pl.P + 127) / 128;
     pl.tilesQ = (pl.Q + pl.bn - 1) / pl.bn;
@@ -1026,6 +1534,13 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
 cudaError_t launch_gemm(const GemmPlan &plan, const GemmBuffers &buf, uint64_t wait_limit_ns, int inject, int pdl,
                         cudaStream_t stream)
 {
+    if (plan.pair) {
+        if (plan.fmt == kFmtMXFP8)
+            return plan.kc == 1 ? launch_pair_t<0, 1>(plan, buf, wait_limit_ns, inject, pdl, stream)
+                                : launch_pair_t<0, 2>(plan, buf, wait_limit_ns, inject, pdl, stream);
+        return plan.kc == 1 ? launch_pair_t<1, 1>(plan, buf, wait_limit_ns, inject, pdl, stream)
+                            : launch_pair_t<1, 2>(plan, buf, wait_limit_ns, inject, pdl, stream);
+    }
     if (plan.kc == 4)
         return plan.fmt == kFmtMXFP8 ? dispatch_bn4<0>(plan, buf, wait_limit_ns, inject, pdl, stream)
                                      : dispatch_bn4<1>(plan, buf, wait_limit_ns, inject, pdl, stream);

@@ -49,6 +49,7 @@ struct GemmPlan {
     int swap = 0;          // 1: MMA rows come from B (C^T = B * A^T)
     int bn = 0;            // MMA N (columns of one output tile)
     int kc = 1;            // 128-byte K chunks per pipeline stage
+    int pair = 0;          // 1: 256x256 tiles on CTA pairs (tcgen05 cta_group::2)
     int stages = 0;
     int64_t M = 0, N = 0, K = 0;
     int64_t P = 0, Q = 0;  // rows of the MMA's row operand / column operand

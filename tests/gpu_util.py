@@ -90,3 +90,24 @@ def sampled_case(fmt: int, M: int, N: int, K: int, seed: int, kind: str = "norma
     # properties that hold at any size: finite inputs give a finite output
     assert bool(torch.isfinite(C.float()).all())
     return rep
+
+
+def rows_case(fmt: int, M: int, N: int, K: int, seed: int, n_rows: int = 48, rng_seed: int = 7):
+    """CPU-drawn inputs, GPU GEMM through mxgemm_run, oracle on a sample of
+    whole output rows (every column of those rows)."""
+    A32, B32 = synth.operands(M, N, K, seed=seed, kind="normal", device="cpu")
+    qa, sa = gpu_quantize(fmt, A32)
+    qb, sb = gpu_quantize(fmt, B32)
+    h = handle()
+    C = h.run(fmt, qa, sa, qb, sb, K=K)
+    torch.cuda.synchronize()
+    st, code = h.check_device_error()
+    assert st == mxgemm.OK and code == 0, ("device error word", code)
+    rng = np.random.default_rng(rng_seed)
+    rm = np.unique(np.concatenate([[0, M - 1], rng.integers(0, M, n_rows)]))
+    oa, osa = oracle.quantize(fmt, A32.numpy()[rm])
+    ob, osb = oracle.quantize(fmt, B32.numpy())
+    assert np.array_equal(qb.cpu().numpy(), ob) and np.array_equal(sb.cpu().numpy(), osb), "B quantiser mismatch"
+    ref, _, mag = oracle.gemm(fmt, K, oa, osa, ob, osb)
+    got = bits(C)[rm]
+    return assert_parity(got, ref, mag, "rows fmt=%d %dx%dx%d" % (fmt, M, N, K)), h.describe(fmt, M, N, K)

@@ -11,7 +11,7 @@ import torch
 import oracle
 from microscaling_block_scaled_b200 import mxgemm, synth
 
-from gpu_util import assert_parity, bits, full_case, handle, sampled_case
+from gpu_util import assert_parity, bits, full_case, handle, rows_case, sampled_case
 
 pytestmark = pytest.mark.gpu
 
@@ -109,6 +109,21 @@ def test_gemm_k_chunks_per_stage(fmt, kc, M, N, K):
         full_case(fmt, M, N, K, seed=kc * 100 + K)
     finally:
         h.set_kchunks(0)
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("kc", [0, 1, 2])
+@pytest.mark.parametrize("M,N,K", [(512, 8192, 256), (640, 8448, 384), (1000, 4104, 512)])
+def test_gemm_cta_pair_tiles(fmt, kc, M, N, K):
+    """Large-M shapes take 256x256 tiles on CTA pairs (cta_group::2); ragged
+    M and N, K tails, and one or two K chunks per stage."""
+    h = handle()
+    h.set_kchunks(kc)
+    try:
+        _, plan = rows_case(fmt, M, N, K, seed=M + kc)
+    finally:
+        h.set_kchunks(0)
+    assert "pair=1" in plan, plan
 
 
 # ----------------------------------------------------------- edge cases

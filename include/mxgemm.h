@@ -149,8 +149,11 @@ MXGEMM_API int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t
 
 /* Read and clear the device error word that kernels set when a bounded wait
  * runs out.  Synchronises the device.  *code receives 0 if no kernel gave
- * up, else a nonzero site code; the return value is MXGEMM_ERR_TIMEOUT in
- * that case, else MXGEMM_OK. */
+ * up, else a nonzero site code (1 producer waiting for a free stage, 2 MMA
+ * waiting for a loaded stage, 3 MMA waiting for a free accumulator,
+ * 4 epilogue waiting for a finished accumulator, 5 end-of-kernel drain,
+ * 6 kernel launched with a block size it was not built for); the return
+ * value is MXGEMM_ERR_TIMEOUT in that case, else MXGEMM_OK. */
 MXGEMM_API int mxgemm_check_device_error(mxgemm_handle h, int *code);
 
 /* Set the per-wait time limit of the kernels' bounded waits in nanoseconds

@@ -71,9 +71,21 @@ struct Cfg {
     static constexpr int kSFACols = kAtoms * 4;
     static constexpr int kSFBCols = kRBQ * kAtoms * 4;
     static constexpr int kSFCols = kStages * (kSFACols + kSFBCols);
-    static constexpr int kNumAcc = (2 * BN + kSFCols <= 512) ? 2 : 1;
-    static constexpr int kAccCols = kNumAcc * BN;
+    // MMA issue costs the issuing thread ~25-50 ns per tcgen05 instruction,
+    // so the K chunks of a stage are split over several MMA warps, each with
+    // its own accumulator (summed by the epilogue), when TMEM holds two
+    // accumulator sets of them.
+    static constexpr int kNMma = (KC >= 4 && 2 * 4 * BN + kSFCols <= 512)   ? 4
+                                 : (KC >= 2 && 2 * 2 * BN + kSFCols <= 512) ? 2
+                                                                            : 1;
+    static constexpr int kChunksPerMma = KC / kNMma;
+    static constexpr int kNumAcc = (2 * kNMma * BN + kSFCols <= 512) ? 2 : 1;
+    static constexpr int kAccCols = kNumAcc * kNMma * BN;
     static constexpr int kTmemCols = 512;
+    // warps: 0 row-operand TMA, 1 MMA, 2..5 epilogue, 6 column-operand TMA,
+    // 7 row-scale TMA, 8 column-scale TMA, 9.. further MMA warps
+    static constexpr int kWarps = 9 + kNMma - 1;
+    static constexpr int kThreads = 32 * kWarps;
     static constexpr int kMmaPerChunk = 4;                    // 32 bytes of K per MMA
     static constexpr uint32_t kTxBytes = kStageBytes;
     // shared memory layout (offsets from a 1024-aligned base)
@@ -136,6 +148,7 @@ enum : int {
     kErrMmaAccEmpty = 3,
     kErrEpiAccFull = 4,
     kErrDrain = 5,
+    kErrLaunch = 6,        // launched with a block size the kernel was not built for
 };
 
 __device__ __forceinline__ void record_error(int *err, int code, volatile int *abort_flag)
@@ -271,7 +284,7 @@ __device__ __forceinline__ void store_bf16(const OutView o, int64_t p, int64_t q
 }
 
 template <int FMT, int BN, int KC>
-__global__ void __launch_bounds__(224, 1)
+__global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
                    const __grid_constant__ CUtensorMap tmC, const KParams kp_in)
@@ -279,6 +292,7 @@ __global__ void __launch_bounds__(224, 1)
     using C_ = Cfg<FMT, BN, KC>;
     constexpr int S = C_::kStages;
     constexpr int CW = C_::kCW;
+    constexpr int NM = C_::kNMma;
 
     // Work on a register copy of the parameters: the inline-asm memory
     // clobbers of the pipeline would otherwise force reloads from parameter
@@ -300,24 +314,39 @@ __global__ void __launch_bounds__(224, 1)
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C_::kOffMisc + 4);
     volatile int *s_last = reinterpret_cast<volatile int *>(smem + C_::kOffMisc + 8);
 
+    if (blockDim.x != C_::kThreads) {
+        if (threadIdx.x == 0)
+            atomicCAS(kp.error, 0, kErrLaunch);
+        return;
+    }
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
+    const bool producer = warp == 0 || (warp >= 6 && warp <= 8);
+    const int mma_idx = warp == 1 ? 0 : (warp >= 9 ? warp - 8 : -1);
 
+    // Each producer fetches its own tensor map while the CTA sets up.
+    if (lane == 0) {
+        if (warp == 0)
+            tma_prefetch_desc(&tmP);
+        else if (warp == 6)
+            tma_prefetch_desc(&tmQ);
+        else if (warp == 7)
+            tma_prefetch_desc(&tmSP);
+        else if (warp == 8)
+            tma_prefetch_desc(&tmSQ);
+        else if (warp == 2)
+            tma_prefetch_desc(&tmC);
+    }
     if (threadIdx.x == 0) {
-        tma_prefetch_desc(&tmP);
-        tma_prefetch_desc(&tmQ);
-        tma_prefetch_desc(&tmSP);
-        tma_prefetch_desc(&tmSQ);
-        tma_prefetch_desc(&tmC);
         for (int s = 0; s < S; ++s) {
-            mbar_init(full_bar(s), 2);          // one arming per producer warp
-            mbar_init(empty_bar(s), 1);
+            mbar_init(full_bar(s), 4);          // one arming per producer warp
+            mbar_init(empty_bar(s), NM);        // one commit per MMA warp
         }
         for (int a = 0; a < C_::kNumAcc; ++a) {
-            mbar_init(accf_bar(a), 1);
+            mbar_init(accf_bar(a), NM);
             mbar_init(acce_bar(a), 4);
         }
-        mbar_init(drain_bar, 1);
+        mbar_init(drain_bar, NM);
         *s_abort = 0;
         *s_last = 0;
         fence_mbar_init();
@@ -335,37 +364,31 @@ __global__ void __launch_bounds__(224, 1)
     const Sched sc{kp.iters, kp.workers, kp.kt, kp.tilesP, kp.dp != 0};
     const uint32_t W = sc.W;
 
-    // Everything except the producers' first operand loads may depend on the
-    // preceding kernel in the stream (the scale repack, or the previous GEMM
-    // that used the same workspace): wait for it here.  Without a
-    // programmatic launch this returns at once.
-    if (warp != 0 && warp != 6)
-        grid_dependency_wait();
-
-    if (warp == 0 || warp == 6) {
+    if (producer) {
         // ----------------------------------------------------- TMA producers
-        // Warp 0 loads the MMA row operand and its scale atoms, warp 6 the
-        // column operand and its scale atoms; each arms the stage's full
-        // barrier for its own bytes.  Every TMA operation costs the issuing
-        // thread and the SM's copy engine a fixed ~0.1-0.2 us, so two issuing
-        // threads and one box per operand (scales included) per stage.
+        // Four producer warps, one TMA operation each per stage: warp 0 the
+        // MMA row-operand tile, warp 6 the column-operand tile, warps 7 and 8
+        // their scale atoms.  Issuing a TMA operation occupies the issuing
+        // thread for ~0.1-0.15 us, so one thread per operation keeps the
+        // ring's refill off the critical path.  Operand tiles are never
+        // written by the kernel this one may overlap (the scale repack), so
+        // only the scale producers wait for it.
         // L2 policy: in the swapped (decode) form the weights stream through
         // once and the small activation is re-read by every tile; otherwise
         // both operands are re-read across tiles.
-        const bool sideP = warp == 0;
         if (lane == 0) {
+            const bool sideP = warp == 0 || warp == 7;
+            const bool scales = warp >= 7;
             const uint64_t pol = sideP ? (kp.swap ? policy_evict_first() : policy_evict_normal())
                                        : (kp.swap ? policy_evict_last() : policy_evict_normal());
-            const CUtensorMap *tmOp = sideP ? &tmP : &tmQ;
-            const CUtensorMap *tmSf = sideP ? &tmSP : &tmSQ;
-            const uint32_t opBytes = sideP ? C_::kABytes : C_::kBBytes;
-            const uint32_t sfBytes = sideP ? C_::kSFABytes : C_::kSFBBytes;
-            const uint32_t offOp = sideP ? C_::kOffA : C_::kOffB;
-            const uint32_t offSf = sideP ? C_::kOffSFA : C_::kOffSFB;
+            const uint32_t bytes = scales ? (sideP ? C_::kSFABytes : C_::kSFBBytes)
+                                          : (sideP ? C_::kABytes : C_::kBBytes);
+            const uint32_t off = scales ? (sideP ? C_::kOffSFA : C_::kOffSFB) : (sideP ? C_::kOffA : C_::kOffB);
+            if (scales)
+                grid_dependency_wait();
             uint32_t armed = 0;         // stages armed so far (round-robin over the ring)
             int skipped_stage = -1;
-            bool inject = sideP && kp.inject == 1;
-            bool first = true;
+            bool inject = warp == 0 && kp.inject == 1;
             int s = 0;
             uint32_t ph = 0;
             for (IterCursor cur(sc, blockIdx.x, gridDim.x); cur.valid(); cur.advance()) {
@@ -374,30 +397,32 @@ __global__ void __launch_bounds__(224, 1)
                     break;
                 }
                 const uint32_t tq = cur.tile / sc.tilesP, tp = cur.tile - tq * sc.tilesP;
-                const int32_t row = sideP ? static_cast<int32_t>(tp) * 128 : static_cast<int32_t>(tq) * BN;
-                const int32_t sf_rb = sideP ? static_cast<int32_t>(tp) : static_cast<int32_t>((tq * BN) / 128);
                 const uint32_t fb = full_bar(s);
+                const uint32_t dst = sbase + off + s * bytes;
                 if (inject) {
                     inject = false;             // test hook: leave this stage unarmed
                     skipped_stage = s;
-                    if (first) {
-                        grid_dependency_wait();
-                        first = false;
-                    }
                 } else {
-                    mbar_arrive_expect_tx(fb, opBytes + sfBytes);
-                    if constexpr (KC == 1)      // 2-D maps: x = byte offset along K
-                        tma_load_2d(sbase + offOp + s * opBytes, tmOp, static_cast<int32_t>(cur.k * 128), row, fb,
-                                    pol);
-                    else                        // 3-D maps: {byte in chunk, row, 128-byte K chunk}
-                        tma_load_3d(sbase + offOp + s * opBytes, tmOp, 0, row, static_cast<int32_t>(cur.k * KC),
-                                    fb, pol);
-                    if (first) {                // the first operand tile may overlap the preceding kernel
-                        grid_dependency_wait();
-                        first = false;
+                    mbar_arrive_expect_tx(fb, bytes);
+                    if (warp == 0) {
+                        const int32_t row = static_cast<int32_t>(tp) * 128;
+                        if constexpr (KC == 1)      // 2-D maps: x = byte offset along K
+                            tma_load_2d(dst, &tmP, static_cast<int32_t>(cur.k * 128), row, fb, pol);
+                        else                        // 3-D maps: {byte in chunk, row, 128-byte K chunk}
+                            tma_load_3d(dst, &tmP, 0, row, static_cast<int32_t>(cur.k * KC), fb, pol);
+                    } else if (warp == 6) {
+                        const int32_t row = static_cast<int32_t>(tq) * BN;
+                        if constexpr (KC == 1)
+                            tma_load_2d(dst, &tmQ, static_cast<int32_t>(cur.k * 128), row, fb, pol);
+                        else
+                            tma_load_3d(dst, &tmQ, 0, row, static_cast<int32_t>(cur.k * KC), fb, pol);
+                    } else if (warp == 7) {
+                        tma_load_3d(dst, &tmSP, 0, static_cast<int32_t>(cur.k * C_::kAtoms),
+                                    static_cast<int32_t>(tp), fb, pol);
+                    } else {
+                        tma_load_3d(dst, &tmSQ, 0, static_cast<int32_t>(cur.k * C_::kAtoms),
+                                    static_cast<int32_t>((tq * BN) / 128), fb, pol);
                     }
-                    tma_load_3d(sbase + offSf + s * sfBytes, tmSf, 0, static_cast<int32_t>(cur.k * C_::kAtoms),
-                                sf_rb, fb, pol);
                 }
                 ++armed;
                 if (++s == S) {
@@ -405,11 +430,9 @@ __global__ void __launch_bounds__(224, 1)
                     ph ^= 1u;
                 }
             }
-            if (first)
-                grid_dependency_wait();
             // Let every armed copy land before the CTA can exit: wait for the
             // latest armed phase of each stage (already complete on the normal
-            // path, where the MMA warp consumed every stage).
+            // path, where the MMA warps consumed every stage).
             for (int st = 0; st < S; ++st) {
                 const uint32_t n = armed / S + (static_cast<uint32_t>(st) < armed % S ? 1u : 0u);
                 if (n == 0 || (st == skipped_stage && n == 1))
@@ -421,11 +444,16 @@ __global__ void __launch_bounds__(224, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------- MMA issuer
+    } else if (mma_idx >= 0) {
+        // ------------------------------------------------------ MMA issuers
+        // MMA warp m takes K chunks [m * kChunksPerMma, (m + 1) * kChunksPerMma)
+        // of every stage: their scale copies into TMEM and their block-scaled
+        // MMAs, into its own accumulator.  Each commit releases the stage once
+        // that warp's MMAs have read it; the stage is free after all NM commits.
         constexpr uint32_t kIdesc = idesc_base<FMT, BN>();
         const uint32_t t_sfa0 = tmem + C_::kAccCols;
         const uint32_t t_sfb0 = t_sfa0 + S * C_::kSFACols;
+        const int c_begin = mma_idx * C_::kChunksPerMma;
         int s = 0;
         uint32_t ph = 0;
         int acc = 0;
@@ -448,7 +476,7 @@ __global__ void __launch_bounds__(224, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t t_acc = tmem + acc * BN;
+                const uint32_t t_acc = tmem + (acc * NM + mma_idx) * BN;
                 for (uint32_t k = kb; k < ke; ++k) {
                     good = 1;
                     if (lane == 0)
@@ -466,17 +494,18 @@ __global__ void __launch_bounds__(224, 1)
                         const uint32_t t_sfb = t_sfb0 + s * C_::kSFBCols;
                         const uint32_t s_sfa = sbase + C_::kOffSFA + s * C_::kSFABytes;
                         const uint32_t s_sfb = sbase + C_::kOffSFB + s * C_::kSFBBytes;
+                        constexpr int kApc = C_::kAtomsPerChunk;
 #pragma unroll
-                        for (int a = 0; a < C_::kAtoms; ++a)
+                        for (int a = c_begin * kApc; a < (c_begin + C_::kChunksPerMma) * kApc; ++a)
                             tmem_cp_32x128b_x4(t_sfa + 4 * a, sdesc_rows16(s_sfa + 512 * a));
 #pragma unroll
                         for (int rb = 0; rb < C_::kRBQ; ++rb)
 #pragma unroll
-                            for (int a = 0; a < C_::kAtoms; ++a)
+                            for (int a = c_begin * kApc; a < (c_begin + C_::kChunksPerMma) * kApc; ++a)
                                 tmem_cp_32x128b_x4(t_sfb + a * 4 * C_::kRBQ + 4 * rb,
                                                    sdesc_rows16(s_sfb + (rb * C_::kAtoms + a) * 512));
 #pragma unroll
-                        for (int c = 0; c < KC; ++c) {
+                        for (int c = c_begin; c < c_begin + C_::kChunksPerMma; ++c) {
                             const uint64_t adesc =
                                 sdesc_sw128_kmajor(sbase + C_::kOffA + s * C_::kABytes + c * C_::kAChunk);
                             const uint64_t bdesc =
@@ -488,7 +517,7 @@ __global__ void __launch_bounds__(224, 1)
                                 const int atom = FMT == kFmtMXFP8 ? c : 2 * c + j / 2;
                                 const uint32_t sf_id = FMT == kFmtMXFP8 ? j : 2 * (j % 2);
                                 const uint32_t idesc = kIdesc | (sf_id << 4) | (sf_id << 29);
-                                const uint32_t acc_flag = (k > kb || c > 0 || j > 0) ? 1u : 0u;
+                                const uint32_t acc_flag = (k > kb || c > c_begin || j > 0) ? 1u : 0u;
                                 const uint64_t koff = static_cast<uint64_t>(j * 32) >> 4;
                                 if (FMT == kFmtMXFP8)
                                     mma_mxf8f6f4(t_acc, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
@@ -518,7 +547,7 @@ __global__ void __launch_bounds__(224, 1)
                 it += ke - kb;
             }
         }
-        // Drain: every tcgen05 operation this thread issued has completed.
+        // Drain: every tcgen05 operation of every MMA warp has completed.
         if (lane == 0) {
             tc_commit(drain_bar);
             int dummy_abort = 0;
@@ -528,6 +557,7 @@ __global__ void __launch_bounds__(224, 1)
         __syncwarp();
     } else if (warp >= 2 && warp <= 5) {
         // ---------------------------------------------------------- epilogue
+        grid_dependency_wait();
         const int quad = warp & 3;             // TMEM lanes 32*quad .. +31
         const int row = quad * 32 + lane;      // accumulator row = MMA row in tile
         const int etid = threadIdx.x - 64;     // 0..127
@@ -536,6 +566,23 @@ __global__ void __launch_bounds__(224, 1)
         uint32_t out_chunks = 0;               // BF16 chunks staged so far (buffer = parity)
         bool stop = false;
 
+        // The tile's accumulator is the sum of the NM MMA warps' accumulators.
+        auto load_acc = [&](uint32_t t_acc, int c, float (&v)[CW]) {
+            uint32_t r[CW];
+            tmem_ld_cols<CW>(t_acc + c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < CW; ++j)
+                v[j] = __uint_as_float(r[j]);
+#pragma unroll
+            for (int m = 1; m < NM; ++m) {
+                tmem_ld_cols<CW>(t_acc + m * BN + c, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < CW; ++j)
+                    v[j] += __uint_as_float(r[j]);
+            }
+        };
 
         // Convert one CW-column chunk of the tile (this thread's row) to BF16
         // and write it to C: through shared memory and a TMA store when the
@@ -590,7 +637,7 @@ __global__ void __launch_bounds__(224, 1)
                 const int64_t tp = sg.tp, tq = sg.tq;
                 int good = 1;
                 if (lane == 0)
-                    good = mbar_wait_sleepy(accf_bar(acc), acc_ph, s_abort, kp.limit_ns, 200);
+                    good = mbar_wait_parked(accf_bar(acc), acc_ph, s_abort, kp.limit_ns);
                 good = __shfl_sync(0xffffffffu, good, 0);
                 if (!good && lane == 0)
                     record_error(kp.error, kErrEpiAccFull, s_abort);
@@ -600,7 +647,7 @@ __global__ void __launch_bounds__(224, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t t_acc = tmem + acc * BN + (static_cast<uint32_t>(quad * 32) << 16);
+                const uint32_t t_acc = tmem + acc * NM * BN + (static_cast<uint32_t>(quad * 32) << 16);
                 const uint32_t g_first = sc.dp ? tile : sc.owner(tile * sc.KT);
                 const uint32_t g_last = sc.dp ? tile : sc.owner(tile * sc.KT + sc.KT - 1);
                 bool released = false;
@@ -611,13 +658,11 @@ __global__ void __launch_bounds__(224, 1)
                     uint32_t packed[BN / 2];
 #pragma unroll
                     for (int c = 0; c < BN; c += CW) {
-                        uint32_t r[CW];
-                        tmem_ld_cols<CW>(t_acc + c, r);
-                        tmem_ld_wait();
+                        float v[CW];
+                        load_acc(t_acc, c, v);
 #pragma unroll
                         for (int j = 0; j < CW / 2; ++j)
-                            packed[c / 2 + j] =
-                                pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                            packed[c / 2 + j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -639,13 +684,12 @@ __global__ void __launch_bounds__(224, 1)
                     float *mine = kp.partials + (slot * 128 + row) * BN;
 #pragma unroll 1
                     for (int c = 0; c < BN; c += CW) {
-                        uint32_t r[CW];
-                        tmem_ld_cols<CW>(t_acc + c, r);
-                        tmem_ld_wait();
+                        float v[CW];
+                        load_acc(t_acc, c, v);
 #pragma unroll
                         for (int j = 0; j < CW / 4; ++j)
-                            reinterpret_cast<uint4 *>(mine + c)[j] =
-                                make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+                            reinterpret_cast<float4 *>(mine + c)[j] =
+                                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
                     }
                     __threadfence();
                     named_bar_sync(1, 128);
@@ -662,9 +706,8 @@ __global__ void __launch_bounds__(224, 1)
                         __threadfence();
 #pragma unroll 1
                         for (int c = 0; c < BN; c += CW) {
-                            uint32_t r[CW];
-                            tmem_ld_cols<CW>(t_acc + c, r);
-                            tmem_ld_wait();
+                            float own[CW];
+                            load_acc(t_acc, c, own);
                             float v[CW];
 #pragma unroll
                             for (int j = 0; j < CW; ++j)
@@ -673,7 +716,7 @@ __global__ void __launch_bounds__(224, 1)
                                 if (g == w) {
 #pragma unroll
                                     for (int j = 0; j < CW; ++j)
-                                        v[j] += __uint_as_float(r[j]);
+                                        v[j] += own[j];
                                 } else {
                                     const int64_t gslot =
                                         2 * static_cast<int64_t>(g) + ((sc.begin(g) / sc.KT == tile) ? 0 : 1);
@@ -1250,7 +1293,7 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     kp.rbytes = rbytes;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
-    cfg.blockDim = dim3(224);
+    cfg.blockDim = dim3(C_::kThreads);
     cfg.dynamicSmemBytes = C_::kSmemBytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];

@@ -128,6 +128,28 @@ __device__ __forceinline__ bool mbar_wait_sleepy(uint32_t bar, uint32_t parity, 
     }
 }
 
+// Wait for a phase that may take a while without spending issue slots: the
+// suspending try_wait parks the thread in hardware until the phase completes
+// (or a hardware time slice passes), so a completed phase is seen at once.
+// Bounded like mbar_wait_bounded.
+__device__ __forceinline__ bool mbar_wait_parked(uint32_t bar, uint32_t parity, const volatile int *abort,
+                                                 uint64_t limit_ns)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((i & 7u) == 0u) {
+            if (*abort)
+                return false;
+            if (globaltimer_ns() - t0 > limit_ns)
+                return false;
+        }
+    }
+}
+
 // ----------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap)

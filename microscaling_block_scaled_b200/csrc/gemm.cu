@@ -786,7 +786,13 @@ struct PairCfg {
     static constexpr int kSFABytes = kAtoms * 512;            // scales of this CTA's A rows
     static constexpr int kSFBBytes = 2 * kAtoms * 512;        // scales of all 256 B rows
     static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
-    static constexpr int kCW = 32;
+    // output staging: two BF16 chunks of 128 rows x kCW columns; 16-column
+    // chunks when the smaller staging buys the ring another stage
+    static constexpr int stages_with(int cw)
+    {
+        return (227 * 1024 - 2048 - 2 * 128 * cw * 2) / kStageBytes;
+    }
+    static constexpr int kCW = stages_with(16) > stages_with(32) ? 16 : 32;
     static constexpr int kOutBytes = 128 * kCW * 2;
     static constexpr int kSmemBudget = 227 * 1024 - 2048 - 2 * kOutBytes;
     static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
@@ -802,7 +808,8 @@ struct PairCfg {
     static constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
     static constexpr int kOffOut = (kOffSFB + kStages * kSFBBytes + 1023) / 1024 * 1024;
     static constexpr int kOffBar = kOffOut + 2 * kOutBytes;
-    static constexpr int kNumBars = 3 * kStages + 3;         // full, empty, pair_full; accf, acce, drain
+    static constexpr int kNumBars = 4 * kStages + 3;   // full, empty, pair_full, scales-ready; accf, acce, drain
+    static constexpr int kThreads = 256;                 // warps 0..6 as the 1-CTA kernel, 7 scale copies
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 
@@ -820,7 +827,7 @@ __host__ __device__ constexpr uint32_t idesc_pair()
 }
 
 template <int FMT, int KC>
-__global__ void __launch_bounds__(224, 1)
+__global__ void __launch_bounds__(256, 1)
     mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
                         const __grid_constant__ CUtensorMap tmC, const KParams kp_in)
@@ -838,12 +845,18 @@ __global__ void __launch_bounds__(224, 1)
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
     auto pfull_bar = [&](int s) { return bar0 + 8u * (2 * S + s); };
-    const uint32_t accf_bar = bar0 + 8u * (3 * S);
-    const uint32_t acce_bar = bar0 + 8u * (3 * S + 1);
-    const uint32_t drain_bar = bar0 + 8u * (3 * S + 2);
+    auto sfr_bar = [&](int s) { return bar0 + 8u * (3 * S + s); };     // leader: stage's scales in TMEM
+    const uint32_t accf_bar = bar0 + 8u * (4 * S);
+    const uint32_t acce_bar = bar0 + 8u * (4 * S + 1);
+    const uint32_t drain_bar = bar0 + 8u * (4 * S + 2);
     volatile uint32_t *s_tmem = reinterpret_cast<volatile uint32_t *>(smem + C_::kOffMisc);
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C_::kOffMisc + 4);
 
+    if (blockDim.x != C_::kThreads) {     // uniform over the cluster: both CTAs return
+        if (threadIdx.x == 0)
+            atomicCAS(kp.error, 0, kErrLaunch);
+        return;
+    }
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const uint32_t rank = cluster_ctarank();
@@ -861,10 +874,11 @@ __global__ void __launch_bounds__(224, 1)
             mbar_init(full_bar(s), 2);          // one arming per producer warp
             mbar_init(empty_bar(s), 1);
             mbar_init(pfull_bar(s), 1);
+            mbar_init(sfr_bar(s), 1);
         }
         mbar_init(accf_bar, 1);
         mbar_init(acce_bar, 8);
-        mbar_init(drain_bar, 1);
+        mbar_init(drain_bar, 2);            // MMA warp and scale-copy warp of the leader
         *s_abort = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -994,11 +1008,8 @@ __global__ void __launch_bounds__(224, 1)
             tc_fence_after();
             for (uint32_t k = 0; k < KT; ++k) {
                 good = 1;
-                if (lane == 0) {
-                    good = mbar_wait_bounded(full_bar(s), ph, s_abort, kp.limit_ns);
-                    if (good)
-                        good = mbar_wait_cluster_bounded(pfull_bar(s), ph, s_abort, kp.limit_ns);
-                }
+                if (lane == 0)
+                    good = mbar_wait_bounded(sfr_bar(s), ph, s_abort, kp.limit_ns);
                 good = __shfl_sync(0xffffffffu, good, 0);
                 if (!good) {
                     if (lane == 0)
@@ -1010,17 +1021,6 @@ __global__ void __launch_bounds__(224, 1)
                 if (lane == 0) {
                     const uint32_t t_sfa = t_sfa0 + s * C_::kSFACols;
                     const uint32_t t_sfb = t_sfb0 + s * C_::kSFBCols;
-                    const uint32_t s_sfa = sbase + C_::kOffSFA + s * C_::kSFABytes;
-                    const uint32_t s_sfb = sbase + C_::kOffSFB + s * C_::kSFBBytes;
-#pragma unroll
-                    for (int a = 0; a < C_::kAtoms; ++a)
-                        tmem_cp_32x128b_x4_pair(t_sfa + 4 * a, sdesc_rows16(s_sfa + 512 * a));
-#pragma unroll
-                    for (int rb = 0; rb < 2; ++rb)
-#pragma unroll
-                        for (int a = 0; a < C_::kAtoms; ++a)
-                            tmem_cp_32x128b_x4_pair(t_sfb + a * 8 + 4 * rb,
-                                                    sdesc_rows16(s_sfb + (rb * C_::kAtoms + a) * 512));
 #pragma unroll
                     for (int c = 0; c < KC; ++c) {
                         const uint64_t adesc = sdesc_sw128_kmajor(sbase + C_::kOffA + s * C_::kABytes + c * C_::kChunk);
@@ -1062,6 +1062,64 @@ __global__ void __launch_bounds__(224, 1)
                 atomicCAS(kp.error, 0, kErrDrain);
         }
         __syncwarp();
+    } else if (warp == 7 && leader) {
+        // ------------------------------ scale copies into TMEM (leader CTA)
+        // Once both CTAs' stage has landed, copy the scale atoms of both
+        // CTAs' A rows and of the tile's B rows into the stage's TMEM slots
+        // (cta_group::2 copies write both CTAs' TMEM), then signal the MMA
+        // warp.  Issuing the copies beside the MMAs keeps them off the MMA
+        // warp's issue stream, where they would add to every stage.
+        const uint32_t t_sfa0 = tmem + C_::kAccCols;
+        const uint32_t t_sfb0 = t_sfa0 + S * C_::kSFACols;
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (uint32_t tile = pair; tile < tiles && ok; tile += npairs) {
+            for (uint32_t k = 0; k < KT; ++k) {
+                int good = 1;
+                if (lane == 0) {
+                    good = mbar_wait_bounded(full_bar(s), ph, s_abort, kp.limit_ns);
+                    if (good)
+                        good = mbar_wait_cluster_bounded(pfull_bar(s), ph, s_abort, kp.limit_ns);
+                }
+                good = __shfl_sync(0xffffffffu, good, 0);
+                if (!good) {
+                    if (lane == 0)
+                        record_error(kp.error, kErrMmaFull, s_abort);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t t_sfa = t_sfa0 + s * C_::kSFACols;
+                    const uint32_t t_sfb = t_sfb0 + s * C_::kSFBCols;
+                    const uint32_t s_sfa = sbase + C_::kOffSFA + s * C_::kSFABytes;
+                    const uint32_t s_sfb = sbase + C_::kOffSFB + s * C_::kSFBBytes;
+#pragma unroll
+                    for (int a = 0; a < C_::kAtoms; ++a)
+                        tmem_cp_32x128b_x4_pair(t_sfa + 4 * a, sdesc_rows16(s_sfa + 512 * a));
+#pragma unroll
+                    for (int rb = 0; rb < 2; ++rb)
+#pragma unroll
+                        for (int a = 0; a < C_::kAtoms; ++a)
+                            tmem_cp_32x128b_x4_pair(t_sfb + a * 8 + 4 * rb,
+                                                    sdesc_rows16(s_sfb + (rb * C_::kAtoms + a) * 512));
+                    tc_commit_pair(sfr_bar(s), 0x1);
+                }
+                __syncwarp();
+                if (++s == S) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+        if (lane == 0) {
+            tc_commit_pair(drain_bar, 0x1);
+            int dummy_abort = 0;
+            if (!mbar_wait_bounded(drain_bar, 0, &dummy_abort, kp.limit_ns))
+                atomicCAS(kp.error, 0, kErrDrain);
+        }
+        __syncwarp();
     } else if (warp >= 2 && warp <= 5) {
         // ---------------------------------------------------------- epilogue
         const int quad = warp & 3;
@@ -1073,7 +1131,7 @@ __global__ void __launch_bounds__(224, 1)
             const uint32_t tq = tile / tilesP, tp = tile - tq * tilesP;
             int good = 1;
             if (lane == 0)
-                good = mbar_wait_sleepy(accf_bar, acc_ph, s_abort, kp.limit_ns, 200);
+                good = mbar_wait_parked(accf_bar, acc_ph, s_abort, kp.limit_ns);
             good = __shfl_sync(0xffffffffu, good, 0);
             if (!good && lane == 0)
                 record_error(kp.error, kErrEpiAccFull, s_abort);
@@ -1364,7 +1422,7 @@ cudaError_t launch_pair_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t lim
     kp.rbytes = rbytes;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
-    cfg.blockDim = dim3(224);
+    cfg.blockDim = dim3(C_::kThreads);
     cfg.dynamicSmemBytes = C_::kSmemBytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];

@@ -120,6 +120,20 @@ MXGEMM_API int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, i
                     const void *B_host, const uint8_t *B_scales_host,
                     void *C_host, void *stream);
 
+/* Profiling switch (an addition; the pages have no counterpart): with `on`
+ * = 1, mxgemm_run and mxgemm_run_host record CUDA events on their stream
+ * before the scale repack, between repack and GEMM, and after the GEMM.  The
+ * middle event keeps the GEMM from overlapping the repack, so profiled runs
+ * are slightly slower than unprofiled ones.  `on` = 0 turns it off.  Returns
+ * MXGEMM_ERR_INVALID_ARG for a NULL handle or another value of `on`. */
+MXGEMM_API int mxgemm_set_profiling(mxgemm_handle h, int on);
+
+/* Device times of the last profiled mxgemm_run / mxgemm_run_host on this
+ * handle: *repack_ms for the scale repack, *gemm_ms for the GEMM.  Waits for
+ * that run to finish.  MXGEMM_ERR_INVALID_ARG when profiling was off for the
+ * last run, or for NULL arguments. */
+MXGEMM_API int mxgemm_last_timing(mxgemm_handle h, float *repack_ms, float *gemm_ms);
+
 /* OCP MX quantisation (the input generator; not part of the timed path).
  * X: FP32 [R][K] device.  Q: codes [R][row_bytes(K)] device.  scales: E8M0
  * [R][K/32] device.  Per 32-element block: amax = max|x|, scale exponent

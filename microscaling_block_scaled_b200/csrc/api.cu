@@ -42,6 +42,10 @@ struct mxgemm_ctx {
     // shape of the last repack
     int last_fmt = -1;
     int64_t last_M = 0, last_N = 0, last_K = 0;
+    // profiling: events around the repack and the GEMM of the last run
+    int profiling = 0;
+    cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
+    int ev_valid = 0;
 };
 
 namespace {
@@ -154,6 +158,32 @@ int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const voi
     return MXGEMM_OK;
 }
 
+// The hot path: scale repack, then the GEMM as a programmatic dependent of
+// it.  With profiling on, events bracket both launches (the middle event
+// keeps the GEMM from starting before the repack ends).
+int repack_and_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const uint8_t *SA,
+                    const void *B, const uint8_t *SB, void *C, cudaStream_t st)
+{
+    const bool prof = h->profiling != 0;
+    h->ev_valid = 0;
+    if (prof && cudaEventRecord(h->ev[0], st) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    int rc = do_repack(h, fmt, M, N, K, SA, SB, st);
+    if (rc != MXGEMM_OK)
+        return rc;
+    if (prof && cudaEventRecord(h->ev[1], st) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    rc = do_gemm(h, fmt, M, N, K, A, B, C, st, prof ? 0 : 1);
+    if (rc != MXGEMM_OK)
+        return rc;
+    if (prof) {
+        if (cudaEventRecord(h->ev[2], st) != cudaSuccess)
+            return MXGEMM_ERR_CUDA;
+        h->ev_valid = 1;
+    }
+    return MXGEMM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -220,6 +250,9 @@ int mxgemm_destroy(mxgemm_handle h)
     cudaFree(h->counters);
     cudaFree(h->err);
     cudaFree(h->stage);
+    for (cudaEvent_t &e : h->ev)
+        if (e)
+            cudaEventDestroy(e);
     delete h;
     return rc;
 }
@@ -267,10 +300,7 @@ int mxgemm_run(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const 
     if (rc != MXGEMM_OK)
         return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    rc = do_repack(h, fmt, M, N, K, A_scales, B_scales, st);
-    if (rc != MXGEMM_OK)
-        return rc;
-    return do_gemm(h, fmt, M, N, K, A, B, C, st, 1);
+    return repack_and_gemm(h, fmt, M, N, K, A, A_scales, B, B_scales, C, st);
 }
 
 int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A_host,
@@ -303,15 +333,42 @@ int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
         cudaMemcpyAsync(d + oB, B_host, nB, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(d + oSB, B_scales_host, nSB, cudaMemcpyHostToDevice, st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
-    rc = do_repack(h, fmt, M, N, K, d + oSA, d + oSB, st);
-    if (rc != MXGEMM_OK)
-        return rc;
-    rc = do_gemm(h, fmt, M, N, K, d + oA, d + oB, d + oC, st, 1);
+    rc = repack_and_gemm(h, fmt, M, N, K, d + oA, d + oSA, d + oB, d + oSB, d + oC, st);
     if (rc != MXGEMM_OK)
         return rc;
     if (cudaMemcpyAsync(C_host, d + oC, nC, cudaMemcpyDeviceToHost, st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    return MXGEMM_OK;
+}
+
+int mxgemm_set_profiling(mxgemm_handle h, int on)
+{
+    if (!h || (on != 0 && on != 1))
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = enter_device(h);
+    if (rc != MXGEMM_OK)
+        return rc;
+    if (on)
+        for (cudaEvent_t &e : h->ev)
+            if (!e && cudaEventCreate(&e) != cudaSuccess)
+                return MXGEMM_ERR_CUDA;
+    h->profiling = on;
+    h->ev_valid = 0;
+    return MXGEMM_OK;
+}
+
+int mxgemm_last_timing(mxgemm_handle h, float *repack_ms, float *gemm_ms)
+{
+    if (!h || !repack_ms || !gemm_ms || !h->ev_valid)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = enter_device(h);
+    if (rc != MXGEMM_OK)
+        return rc;
+    if (cudaEventSynchronize(h->ev[2]) != cudaSuccess ||
+        cudaEventElapsedTime(repack_ms, h->ev[0], h->ev[1]) != cudaSuccess ||
+        cudaEventElapsedTime(gemm_ms, h->ev[1], h->ev[2]) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
     return MXGEMM_OK;
 }

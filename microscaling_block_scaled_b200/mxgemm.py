@@ -47,6 +47,8 @@ SIGNATURES = {
     "mxgemm_set_wait_limit": (ctypes.c_int, [_vp, ctypes.c_uint64]),
     "mxgemm_debug_inject": (ctypes.c_int, [_vp, ctypes.c_int]),
     "mxgemm_run_noalloc": (ctypes.c_int, [ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "mxgemm_set_profiling": (ctypes.c_int, [_vp, ctypes.c_int]),
+    "mxgemm_last_timing": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
     "mxgemm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mxgemm_version": (ctypes.c_char_p, []),
 }
@@ -182,6 +184,16 @@ def mxgemm_debug_inject(h, mode: int) -> int:
     return load().mxgemm_debug_inject(h, mode)
 
 
+def mxgemm_set_profiling(h, on: int) -> int:
+    return load().mxgemm_set_profiling(h, on)
+
+
+def mxgemm_last_timing(h) -> tuple[int, float, float]:
+    rep, gem = ctypes.c_float(0.0), ctypes.c_float(0.0)
+    st = load().mxgemm_last_timing(h, ctypes.byref(rep), ctypes.byref(gem))
+    return st, rep.value, gem.value
+
+
 # ------------------------------------------------------- torch helpers
 
 def quantize(fmt: int, X, stream=None):
@@ -253,3 +265,12 @@ class Handle:
 
     def debug_inject(self, mode: int):
         _check("mxgemm_debug_inject", mxgemm_debug_inject(self.h, mode))
+
+    def set_profiling(self, on: bool):
+        _check("mxgemm_set_profiling", mxgemm_set_profiling(self.h, 1 if on else 0))
+
+    def last_timing(self) -> tuple[float, float]:
+        """(repack_ms, gemm_ms) of the last profiled run on this handle."""
+        st, rep, gem = mxgemm_last_timing(self.h)
+        _check("mxgemm_last_timing", st)
+        return rep, gem

@@ -249,6 +249,26 @@ def run_reference(args):
 
 # ---------------------------------------------------------------- GPU arm
 
+def max_over_ranks(values, device=None):
+    """Elementwise maximum of `values` over the ranks of the default process
+    group (the values themselves without one): the job's time is its slowest
+    rank's.  NCCL reduces device tensors, gloo host tensors."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    dev = device if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_tflops(fmt_flops, world, steps, ms):
+    """Whole-job throughput: every rank runs `steps` replicas of the GEMM in
+    the slowest rank's `ms` milliseconds."""
+    return fmt_flops * world * steps / (ms * 1e-3) / 1e12
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -341,13 +361,10 @@ def run_ours(args):
     del g_step, g_gemm, g_rep
     torch.cuda.synchronize()
 
-    if world > 1:
-        t = torch.tensor([ms, ms_gemm, ms_rep], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, ms_gemm, ms_rep = (float(x) for x in t.tolist())
+    ms, ms_gemm, ms_rep = max_over_ranks([ms, ms_gemm, ms_rep], dev)
 
     ms_per_step = ms / args.steps
-    value = flops(M, N, K) * world * args.steps / (ms * 1e-3) / 1e12
+    value = job_tflops(flops(M, N, K), world, args.steps, ms)
     gemm_us = ms_gemm / args.steps * 1e3
     rep_us = ms_rep / args.steps * 1e3
 
@@ -392,11 +409,8 @@ def run_ours(args):
     e1.record(st)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = flops(M, N, K) * world * args.e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks([e2e_ms], dev)[0]
+    e2e_value = job_tflops(flops(M, N, K), world, args.e2e_steps, e2e_ms)
     h2d = pa.numel() + psa.numel() + pb.numel() + psb.numel()
     d2h = pc.numel() * 2
 

@@ -71,14 +71,23 @@ struct Cfg {
     static constexpr int kSFACols = kAtoms * 4;
     static constexpr int kSFBCols = kRBQ * kAtoms * 4;
     static constexpr int kSFCols = kStages * (kSFACols + kSFBCols);
-    // MMA issue costs the issuing thread ~25-50 ns per tcgen05 instruction,
-    // so the K chunks of a stage are split over several MMA warps, each with
-    // its own accumulator (summed by the epilogue), when TMEM holds two
-    // accumulator sets of them.
-    static constexpr int kNMma = (KC >= 4 && 2 * 4 * BN + kSFCols <= 512)   ? 4
-                                 : (KC >= 2 && 2 * 2 * BN + kSFCols <= 512) ? 2
-                                                                            : 1;
-    static constexpr int kChunksPerMma = KC / kNMma;
+    // A tcgen05 instruction holds its issuing thread ~40 ns, so a stage's
+    // scale copies and MMAs are split over kNMma MMA warps, each with its own
+    // accumulator (summed by the epilogue).  Warp m owns a contiguous run of
+    // the stage's scale atoms: it copies them and issues exactly the MMAs
+    // that read them, so no warp's MMA depends on another warp's copy.
+    // Narrow (decode) tiles take up to four warps where TMEM holds one
+    // accumulator set; wider ones keep two accumulator sets.
+    static constexpr int kMmaPerAtom = FMT == kFmtMXFP8 ? 4 : 2;   // MMAs reading one 512B atom
+    static constexpr int pick_nmma()
+    {
+        for (int nm = 4; nm > 1; nm /= 2)
+            if (kAtoms % nm == 0 && (BN <= 64 ? nm * BN : 2 * nm * BN) + kSFCols <= 512)
+                return nm;
+        return 1;
+    }
+    static constexpr int kNMma = pick_nmma();
+    static constexpr int kAtomsPerMma = kAtoms / kNMma;
     static constexpr int kNumAcc = (2 * kNMma * BN + kSFCols <= 512) ? 2 : 1;
     static constexpr int kAccCols = kNumAcc * kNMma * BN;
     static constexpr int kTmemCols = 512;
@@ -446,14 +455,14 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         __syncwarp();
     } else if (mma_idx >= 0) {
         // ------------------------------------------------------ MMA issuers
-        // MMA warp m takes K chunks [m * kChunksPerMma, (m + 1) * kChunksPerMma)
+        // MMA warp m takes scale atoms [m * kAtomsPerMma, (m + 1) * kAtomsPerMma)
         // of every stage: their scale copies into TMEM and their block-scaled
         // MMAs, into its own accumulator.  Each commit releases the stage once
         // that warp's MMAs have read it; the stage is free after all NM commits.
         constexpr uint32_t kIdesc = idesc_base<FMT, BN>();
         const uint32_t t_sfa0 = tmem + C_::kAccCols;
         const uint32_t t_sfb0 = t_sfa0 + S * C_::kSFACols;
-        const int c_begin = mma_idx * C_::kChunksPerMma;
+        const int a_begin = mma_idx * C_::kAtomsPerMma;
         int s = 0;
         uint32_t ph = 0;
         int acc = 0;
@@ -494,38 +503,37 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                         const uint32_t t_sfb = t_sfb0 + s * C_::kSFBCols;
                         const uint32_t s_sfa = sbase + C_::kOffSFA + s * C_::kSFABytes;
                         const uint32_t s_sfb = sbase + C_::kOffSFB + s * C_::kSFBBytes;
-                        constexpr int kApc = C_::kAtomsPerChunk;
 #pragma unroll
-                        for (int a = c_begin * kApc; a < (c_begin + C_::kChunksPerMma) * kApc; ++a)
+                        for (int a = a_begin; a < a_begin + C_::kAtomsPerMma; ++a)
                             tmem_cp_32x128b_x4(t_sfa + 4 * a, sdesc_rows16(s_sfa + 512 * a));
 #pragma unroll
                         for (int rb = 0; rb < C_::kRBQ; ++rb)
 #pragma unroll
-                            for (int a = c_begin * kApc; a < (c_begin + C_::kChunksPerMma) * kApc; ++a)
+                            for (int a = a_begin; a < a_begin + C_::kAtomsPerMma; ++a)
                                 tmem_cp_32x128b_x4(t_sfb + a * 4 * C_::kRBQ + 4 * rb,
                                                    sdesc_rows16(s_sfb + (rb * C_::kAtoms + a) * 512));
+                        // MMA q of the stage (chunk q / 4, 32-byte step q % 4) reads atom
+                        // q / kMmaPerAtom: MXFP8 one scale block per MMA (byte q % 4 of
+                        // the chunk's atom), MXFP4 two (byte pair 2 * (q % 2)).
 #pragma unroll
-                        for (int c = c_begin; c < c_begin + C_::kChunksPerMma; ++c) {
+                        for (int q = a_begin * C_::kMmaPerAtom; q < (a_begin + C_::kAtomsPerMma) * C_::kMmaPerAtom;
+                             ++q) {
+                            const int c = q / C_::kMmaPerChunk, j = q % C_::kMmaPerChunk;
+                            const int atom = q / C_::kMmaPerAtom;
                             const uint64_t adesc =
                                 sdesc_sw128_kmajor(sbase + C_::kOffA + s * C_::kABytes + c * C_::kAChunk);
                             const uint64_t bdesc =
                                 sdesc_sw128_kmajor(sbase + C_::kOffB + s * C_::kBBytes + c * C_::kBChunk);
-#pragma unroll
-                            for (int j = 0; j < C_::kMmaPerChunk; ++j) {
-                                // MXFP8: one scale block per MMA, id j of the chunk's atom.
-                                // MXFP4: two scale blocks per MMA, atom 2c + j/2, byte pair 2*(j%2).
-                                const int atom = FMT == kFmtMXFP8 ? c : 2 * c + j / 2;
-                                const uint32_t sf_id = FMT == kFmtMXFP8 ? j : 2 * (j % 2);
-                                const uint32_t idesc = kIdesc | (sf_id << 4) | (sf_id << 29);
-                                const uint32_t acc_flag = (k > kb || c > c_begin || j > 0) ? 1u : 0u;
-                                const uint64_t koff = static_cast<uint64_t>(j * 32) >> 4;
-                                if (FMT == kFmtMXFP8)
-                                    mma_mxf8f6f4(t_acc, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
-                                                 t_sfb + atom * 4 * C_::kRBQ, acc_flag);
-                                else
-                                    mma_mxf4(t_acc, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
+                            const uint32_t sf_id = FMT == kFmtMXFP8 ? j : 2 * (j % 2);
+                            const uint32_t idesc = kIdesc | (sf_id << 4) | (sf_id << 29);
+                            const uint32_t acc_flag = (k > kb || q > a_begin * C_::kMmaPerAtom) ? 1u : 0u;
+                            const uint64_t koff = static_cast<uint64_t>(j * 32) >> 4;
+                            if (FMT == kFmtMXFP8)
+                                mma_mxf8f6f4(t_acc, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
                                              t_sfb + atom * 4 * C_::kRBQ, acc_flag);
-                            }
+                            else
+                                mma_mxf4(t_acc, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
+                                         t_sfb + atom * 4 * C_::kRBQ, acc_flag);
                         }
                         tc_commit(empty_bar(s));
                     }

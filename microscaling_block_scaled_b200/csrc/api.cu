@@ -127,10 +127,13 @@ int do_repack(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const u
     return MXGEMM_OK;
 }
 
+// GEMM launch.  With raw scales (SA, SB non-NULL) the kernel converts the
+// row-major scales itself; otherwise it reads the last repack's workspace,
+// which must be for this shape.
 int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const void *B, void *C,
-            cudaStream_t st, int pdl)
+            cudaStream_t st, int pdl, const uint8_t *SA = nullptr, const uint8_t *SB = nullptr)
 {
-    if (h->last_fmt != fmt || h->last_M != M || h->last_N != N || h->last_K != K)
+    if (!SA && (h->last_fmt != fmt || h->last_M != M || h->last_N != N || h->last_K != K))
         return MXGEMM_ERR_INVALID_ARG;
     const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks);
     if (!pl.valid)
@@ -151,6 +154,8 @@ int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const voi
     b.partials = h->partials;
     b.counters = h->counters;
     b.error = h->err;
+    b.rawA = SA;
+    b.rawB = SB;
     const int inject = h->inject;
     h->inject = 0;
     if (mxg::launch_gemm(pl, b, h->limit_ns, inject, pdl, st) != cudaSuccess)
@@ -158,22 +163,31 @@ int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const voi
     return MXGEMM_OK;
 }
 
-// The hot path: scale repack, then the GEMM as a programmatic dependent of
-// it.  With profiling on, events bracket both launches (the middle event
-// keeps the GEMM from starting before the repack ends).
+// The hot path.  Plans on one CTA per tile convert the row-major scales
+// inside the GEMM (one launch); CTA-pair plans run the scale repack, then
+// the GEMM as a programmatic dependent of it.  With profiling on, events
+// bracket the launches (the middle event keeps the GEMM from starting
+// before the repack ends; with the conversion fused it records no repack
+// time).
 int repack_and_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const uint8_t *SA,
                     const void *B, const uint8_t *SB, void *C, cudaStream_t st)
 {
     const bool prof = h->profiling != 0;
     h->ev_valid = 0;
+    const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks);
+    const bool fused = pl.valid && !pl.pair;
     if (prof && cudaEventRecord(h->ev[0], st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
-    int rc = do_repack(h, fmt, M, N, K, SA, SB, st);
-    if (rc != MXGEMM_OK)
-        return rc;
+    int rc = MXGEMM_OK;
+    if (!fused) {
+        rc = do_repack(h, fmt, M, N, K, SA, SB, st);
+        if (rc != MXGEMM_OK)
+            return rc;
+    }
     if (prof && cudaEventRecord(h->ev[1], st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
-    rc = do_gemm(h, fmt, M, N, K, A, B, C, st, prof ? 0 : 1);
+    rc = fused ? do_gemm(h, fmt, M, N, K, A, B, C, st, 0, SA, SB)
+               : do_gemm(h, fmt, M, N, K, A, B, C, st, prof ? 0 : 1);
     if (rc != MXGEMM_OK)
         return rc;
     if (prof) {

@@ -148,6 +148,12 @@ struct KParams {
     int tma_store;         // 1: epilogue stores C through shared memory with TMA
     const uint8_t *opP;    // the MMA row operand (for whole-tile L2 prefetch)
     int64_t rbytes;        // bytes per operand row
+    // Fused scale conversion (1-CTA kernel): the scale producers gather each
+    // stage's atoms from the row-major scales [rows][K/32] themselves instead
+    // of loading the repacked layout.
+    int fused_sf;
+    const uint8_t *rawP, *rawQ;   // row-major scales of the row / column operand
+    int64_t ldS;                  // K / 32: scale bytes per row
 };
 
 // Error site codes written to the device error word.
@@ -348,7 +354,9 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(full_bar(s), 4);          // one arming per producer warp
+            // one arming per producer warp; with fused scales, one async
+            // arrival per lane of the two scale warps
+            mbar_init(full_bar(s), kp.fused_sf ? 2 + 64 : 4);
             mbar_init(empty_bar(s), NM);        // one commit per MMA warp
         }
         for (int a = 0; a < C_::kNumAcc; ++a) {
@@ -373,7 +381,61 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
     const Sched sc{kp.iters, kp.workers, kp.kt, kp.tilesP, kp.dp != 0};
     const uint32_t W = sc.W;
 
-    if (producer) {
+    if (producer && kp.fused_sf && warp >= 7) {
+        // ------------------------------------- scale atoms gathered directly
+        // Warp 7 (row operand) and warp 8 (column operand) build each stage's
+        // scale atoms in shared memory from the row-major scales: atom a of a
+        // 128-row block holds, for row r and K block 4a + j, the byte at
+        // (r % 32) * 16 + (r / 32) * 4 + j.  Lane l moves rows l, l+32, l+64,
+        // l+96 with 4-byte cp.async copies (rows past the operand and K
+        // blocks past K are zero-filled) and arrives on the stage's full
+        // barrier once its copies have landed.
+        const bool sideP = warp == 7;
+        const uint8_t *raw = sideP ? kp.rawP : kp.rawQ;
+        const int64_t nrows = sideP ? kp.P : kp.Q;
+        const uint32_t bytes = sideP ? C_::kSFABytes : C_::kSFBBytes;
+        const uint32_t off = sideP ? C_::kOffSFA : C_::kOffSFB;
+        const int nrb = sideP ? 1 : C_::kRBQ;
+        const int64_t kblocks = kp.ldS;
+        int s = 0;
+        uint32_t ph = 0;
+        for (IterCursor cur(sc, blockIdx.x, gridDim.x); cur.valid(); cur.advance()) {
+            int good = 1;
+            if (lane == 0)
+                good = mbar_wait_bounded(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns);
+            good = __shfl_sync(0xffffffffu, good, 0);
+            if (!good) {
+                if (lane == 0)
+                    record_error(kp.error, kErrProducerEmpty, s_abort);
+                break;
+            }
+            const uint32_t tq = cur.tile / sc.tilesP, tp = cur.tile - tq * sc.tilesP;
+            const int64_t rb0 = sideP ? static_cast<int64_t>(tp) : static_cast<int64_t>((tq * BN) / 128);
+            const int64_t kb0 = static_cast<int64_t>(cur.k) * C_::kAtoms * 4;
+            const uint32_t dst0 = sbase + off + s * bytes + lane * 16;
+            for (int rb = 0; rb < nrb; ++rb) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int64_t row = (rb0 + rb) * 128 + i * 32 + lane;
+                    const bool rv = row < nrows;
+#pragma unroll
+                    for (int a = 0; a < C_::kAtoms; ++a) {
+                        const int64_t kb = kb0 + 4 * a;
+                        const bool v = rv && kb < kblocks;
+                        cp_async_4(dst0 + (rb * C_::kAtoms + a) * 512 + i * 4, v ? raw + row * kblocks + kb : raw,
+                                   v ? 4u : 0u);
+                    }
+                }
+            }
+            cp_async_arrive_noinc(full_bar(s));
+            if (++s == S) {
+                s = 0;
+                ph ^= 1u;
+            }
+        }
+        cp_async_wait_all();
+        __syncwarp();
+    } else if (producer) {
         // ----------------------------------------------------- TMA producers
         // Four producer warps, one TMA operation each per stage: warp 0 the
         // MMA row-operand tile, warp 6 the column-operand tile, warps 7 and 8
@@ -499,6 +561,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                     }
                     tc_fence_after();
                     if (lane == 0) {
+                        if (kp.fused_sf)            // scale atoms written by cp.async (generic proxy)
+                            fence_proxy_async_smem();
                         const uint32_t t_sfa = t_sfa0 + s * C_::kSFACols;
                         const uint32_t t_sfb = t_sfb0 + s * C_::kSFBCols;
                         const uint32_t s_sfa = sbase + C_::kOffSFA + s * C_::kSFABytes;
@@ -1329,8 +1393,13 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     if (!okC)
         return cudaErrorInvalidValue;
     CUtensorMap tmSP, tmSQ;
-    const uint8_t *sfP = pl.swap ? b.sfB : b.sfA;
-    const uint8_t *sfQ = pl.swap ? b.sfA : b.sfB;
+    const bool fused = b.rawA != nullptr;
+    const uint8_t *rawP = pl.swap ? b.rawB : b.rawA;
+    const uint8_t *rawQ = pl.swap ? b.rawA : b.rawB;
+    // with fused scales the repacked maps are never read: encode them over
+    // the row-major scales so they are valid
+    const uint8_t *sfP = fused ? rawP : (pl.swap ? b.sfB : b.sfA);
+    const uint8_t *sfQ = fused ? rawQ : (pl.swap ? b.sfA : b.sfB);
     if (!make_sf_map(&tmSP, sfP, pl.kaP, sf_row_blocks(pl.P), C_::kAtoms, 1) ||
         !make_sf_map(&tmSQ, sfQ, pl.kaQ, sf_row_blocks(pl.Q), C_::kAtoms, C_::kRBQ))
         return cudaErrorInvalidValue;
@@ -1357,6 +1426,10 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     kp.tma_store = tma_store;
     kp.opP = static_cast<const uint8_t *>(Pptr);
     kp.rbytes = rbytes;
+    kp.fused_sf = fused ? 1 : 0;
+    kp.rawP = rawP;
+    kp.rawQ = rawQ;
+    kp.ldS = pl.K / 32;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
     cfg.blockDim = dim3(C_::kThreads);
@@ -1428,6 +1501,10 @@ cudaError_t launch_pair_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t lim
     kp.tma_store = 1;
     kp.opP = static_cast<const uint8_t *>(b.A);
     kp.rbytes = rbytes;
+    kp.fused_sf = 0;
+    kp.rawP = nullptr;
+    kp.rawQ = nullptr;
+    kp.ldS = pl.K / 32;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
     cfg.blockDim = dim3(C_::kThreads);

@@ -71,6 +71,9 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
 struct GemmBuffers {
     const void *A, *B;
     const uint8_t *sfA, *sfB;   // repacked scales of A and of B
+    // row-major scales of A and B: when set (1-CTA plans only), the GEMM
+    // converts them itself and sfA / sfB are not read
+    const uint8_t *rawA = nullptr, *rawB = nullptr;
     void *C;
     float *partials;
     uint32_t *counters;

@@ -373,7 +373,7 @@ def run_ours(args):
     # mxgemm_run on a one-CTA plan is one kernel (scale conversion fused into
     # the GEMM's scale producers): the step's kernel time is the step time.
     # CTA-pair plans run the repack and then the GEMM: their kernel is the GEMM.
-    fused = "pair=1" not in plan
+    fused = "scales=fused" in plan
     kernel_us = ms / args.steps * 1e3 if fused else gemm_us
     rep_us = ms_rep / args.steps * 1e3
 
@@ -394,7 +394,8 @@ def run_ours(args):
     roof["traffic"] = tr
     roof["peak_source"] = "%s (%s)" % (peak_src, "hbm_gbs" if roof["bound"] == "hbm" else
                                        "bf16_tflops x %d (nominal MX/bf16 ratio)" % (2 if fmt == 0 else 4))
-    roof["kernel"] = "mx_gemm_kernel (scale conversion fused)" if fused else "mx_gemm_pair_kernel"
+    roof["kernel"] = ("mx_gemm_kernel (scale conversion fused)" if fused else
+                      "mx_gemm_pair_kernel" if "pair=1" in plan else "mx_gemm_kernel")
     roof["algorithmic_bytes"] = algorithmic_bytes(fmt, M, N, K)
     roof["flops"] = flops(M, N, K)
 
@@ -445,7 +446,7 @@ def run_ours(args):
                        "timing": "CUDA graph of K steps, CUDA events on the launch stream",
                        "plan": plan, "kernel_us": kernel_us, "gemm_us": gemm_us, "repack_us": rep_us,
                        "step_kernels": "mx_gemm_kernel with fused scale conversion" if fused
-                       else "mx_repack_kernel + mx_gemm_pair_kernel",
+                       else "mx_repack_kernel + " + roof["kernel"],
                        "gemm_tflops": flops(M, N, K) / (gemm_us * 1e-6) / 1e12},
             "clocks": clocks,
             "roofline": roof,

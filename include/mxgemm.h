@@ -89,11 +89,13 @@ MXGEMM_API int mxgemm_create(mxgemm_handle *out);
  * NULL is accepted and ignored. */
 MXGEMM_API int mxgemm_destroy(mxgemm_handle h);
 
-/* Full hot path on `stream`: repack A_scales and B_scales from the canonical
- * row-major layout into the tensor-core scale layout (in the handle's
- * workspace), then run the block-scaled GEMM writing C.  Two kernel launches,
- * no host synchronisation.  All buffers are device memory.  `stream` is a
- * cudaStream_t (NULL = legacy default stream). */
+/* Full hot path on `stream`: convert A_scales and B_scales from the
+ * canonical row-major layout into the tensor-core scale layout and run the
+ * block-scaled GEMM writing C.  Where the plan allows (see
+ * mxgemm_describe_plan, "scales=fused") the GEMM gathers the scales itself:
+ * one kernel launch.  Otherwise the scales are repacked into the handle's
+ * workspace first: two launches.  No host synchronisation.  All buffers are
+ * device memory.  `stream` is a cudaStream_t (NULL = legacy default stream). */
 MXGEMM_API int mxgemm_run(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
                const void *A, const uint8_t *A_scales,
                const void *B, const uint8_t *B_scales,
@@ -157,7 +159,11 @@ MXGEMM_API int mxgemm_set_kchunks(mxgemm_handle h, int kc);
 
 /* Describe the plan mxgemm_gemm would use for a shape: writes up to `cap`
  * bytes of a NUL-terminated text such as
- * "fmt=1 swap=1 BN=32 kc=2 stages=4 tiles=112 kt=8 workers=112 grid=112 sched=dp partial_bytes=0". */
+ * "fmt=1 swap=1 pair=0 BN=32 kc=2 stages=4 tiles=112 kt=8 workers=112
+ * grid=112 sched=dp partial_bytes=0 scales=fused".  The last field says how
+ * mxgemm_run treats the scales for this shape: "fused" (the GEMM converts
+ * the row-major scales itself, one launch) or "repack" (scale repack, then
+ * the GEMM). */
 MXGEMM_API int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
                          char *buf, size_t cap);
 

@@ -127,6 +127,11 @@ int do_repack(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const u
     return MXGEMM_OK;
 }
 
+// mxgemm_run converts the row-major scales inside the GEMM for one-CTA
+// plans whose ring is at least four stages deep (the gather's latency hides
+// behind the ring); otherwise it runs the separate repack first.
+bool fuse_scales(const mxg::GemmPlan &pl) { return pl.valid && !pl.pair && pl.stages >= 4; }
+
 // GEMM launch.  With raw scales (SA, SB non-NULL) the kernel converts the
 // row-major scales itself; otherwise it reads the last repack's workspace,
 // which must be for this shape.
@@ -175,7 +180,7 @@ int repack_and_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
     const bool prof = h->profiling != 0;
     h->ev_valid = 0;
     const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks);
-    const bool fused = pl.valid && !pl.pair;
+    const bool fused = fuse_scales(pl);
     if (prof && cudaEventRecord(h->ev[0], st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
     int rc = MXGEMM_OK;
@@ -432,10 +437,10 @@ int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t
     static const char *names[] = {"auto", "dp", "splitk", "streamk"};
     snprintf(buf, cap,
              "fmt=%d swap=%d pair=%d BN=%d kc=%d stages=%d tiles=%lld kt=%lld workers=%lld grid=%d sched=%s "
-             "partial_bytes=%lld",
+             "partial_bytes=%lld scales=%s",
              pl.fmt, pl.swap, pl.pair, pl.bn, pl.kc, pl.stages, static_cast<long long>(pl.tiles), static_cast<long long>(pl.kt),
              static_cast<long long>(pl.workers), pl.grid, names[pl.sched & 3],
-             static_cast<long long>(pl.partial_bytes));
+             static_cast<long long>(pl.partial_bytes), fuse_scales(pl) ? "fused" : "repack");
     return MXGEMM_OK;
 }
 

@@ -232,8 +232,12 @@ def test_gemm_integer_exact(fmt):
 
 # -------------------------------------------------------- entry points
 
-def test_repack_then_gemm_equals_run_and_host_path():
-    fmt, M, N, K = F4, 48, 512, 1024
+@pytest.mark.parametrize("fmt,M,N,K", [(F4, 48, 512, 1024), (F4, 32, 512, 1024), (F8, 16, 384, 512)],
+                         ids=["repack-plan", "fused-plan", "fused-plan-mxfp8"])
+def test_repack_then_gemm_equals_run_and_host_path(fmt, M, N, K):
+    """mxgemm_run (one launch with the scale conversion fused into the GEMM,
+    or repack + GEMM, per the plan), mxgemm_repack + mxgemm_gemm and the
+    host-buffer path give bit-identical C."""
     A32, B32 = synth.operands(M, N, K, seed=31)
     qa, sa = mxgemm.quantize(fmt, A32.cuda())
     qb, sb = mxgemm.quantize(fmt, B32.cuda())
@@ -248,6 +252,24 @@ def test_repack_then_gemm_equals_run_and_host_path():
     torch.cuda.synchronize()
     assert torch.equal(C1.view(torch.int16), C2.view(torch.int16))
     assert torch.equal(C1.view(torch.int16).cpu(), C3.view(torch.int16))
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("sched", [
+    (mxgemm.SCHED_SPLITK, 3, 0), (mxgemm.SCHED_STREAMK, 1, 0), (mxgemm.SCHED_STREAMK, 1, 37),
+])
+def test_fused_scales_with_split_schedules(fmt, sched):
+    """The GEMM's own scale conversion under split-K and stream-K, where a
+    CTA's work spans several tiles and K ranges."""
+    M, N, K = 32, 1536, 2048
+    h = handle()
+    h.set_schedule(*sched)
+    try:
+        plan = h.describe(fmt, M, N, K)
+    finally:
+        h.set_schedule(mxgemm.SCHED_AUTO)
+    assert "scales=fused" in plan, plan
+    full_case(fmt, M, N, K, seed=77, schedule=sched)
 
 
 def test_gemm_rejects_shape_not_repacked():

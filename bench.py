@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--reps", type=int, default=20, help="extra replays of the step graph for the spread")
     ap.add_argument("--e2e-steps", type=int, default=20)
     return ap.parse_args()
 
@@ -351,6 +352,8 @@ def run_ours(args):
         ms = timed(g_step, s_step)
         clk.active = False
     clocks = clk.summary()
+    # spread: the same graph replayed again (not part of `value`)
+    reps = [timed(g_step, s_step) / args.steps * 1e3 for _ in range(args.reps)]
     # the GEMM-only graph reads the repacked-scale workspace (mxgemm_run on a
     # one-CTA plan converts the scales inside the GEMM and leaves none)
     h.repack(fmt, M, N, K, sets[0][1], sets[0][3])
@@ -394,6 +397,10 @@ def run_ours(args):
     roof["traffic"] = tr
     roof["peak_source"] = "%s (%s)" % (peak_src, "hbm_gbs" if roof["bound"] == "hbm" else
                                        "bf16_tflops x %d (nominal MX/bf16 ratio)" % (2 if fmt == 0 else 4))
+    if algorithmic_bytes(fmt, M, N, K) < (1 << 20):
+        roof["note"] = ("latency-bound: %d bytes per launch take ~%.0f ns at HBM speed, far below a launch; "
+                        "the fraction is not meaningful, the us are" % (algorithmic_bytes(fmt, M, N, K),
+                                                                        algorithmic_bytes(fmt, M, N, K) / hbm))
     roof["kernel"] = ("mx_gemm_kernel (scale conversion fused)" if fused else
                       "mx_gemm_pair_kernel" if "pair=1" in plan else "mx_gemm_kernel")
     roof["algorithmic_bytes"] = algorithmic_bytes(fmt, M, N, K)
@@ -445,6 +452,8 @@ def run_ours(args):
                            nsets, set_bytes / 1e6, nsets * set_bytes / 1e6, l2 / 1e6),
                        "timing": "CUDA graph of K steps, CUDA events on the launch stream",
                        "plan": plan, "kernel_us": kernel_us, "gemm_us": gemm_us, "repack_us": rep_us,
+                       "step_us_spread": {"n": len(reps), "median": statistics.median(reps) if reps else None,
+                                          "min": min(reps) if reps else None, "max": max(reps) if reps else None},
                        "step_kernels": "mx_gemm_kernel with fused scale conversion" if fused
                        else "mx_repack_kernel + " + roof["kernel"],
                        "gemm_tflops": flops(M, N, K) / (gemm_us * 1e-6) / 1e12},

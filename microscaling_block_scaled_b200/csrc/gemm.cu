@@ -9,16 +9,25 @@
 // carries an operand tile pair together with the scale tiles of exactly
 // those K elements, released by one mbarrier.
 //
-// Structure of one persistent CTA (192 threads, one per SM):
-//   warp 0      TMA producer: per stage, the 128x128-byte row-operand tile,
-//               the BNx128-byte column-operand tile (both 128B-swizzled) and
-//               the matching repacked scale atoms (plain bulk copies).
-//   warp 1      MMA issuer and TMEM owner: tcgen05.cp of the stage's scales
-//               into TMEM, then four tcgen05.mma block_scale instructions
-//               (kind::mxf8f6f4 K=32 / kind::mxf4 K=64) into an FP32 TMEM
-//               accumulator; tcgen05.commit releases the stage.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator, BF16 (RNE) stores;
-//               for split tiles an FP32 partial plus a last-arriver fixup.
+// Two kernels.  mx_gemm_kernel: one persistent CTA per SM, 128-row tiles.
+//   warps 0, 6  TMA producers of the row / column operand tile of each stage
+//               (128B-swizzled, KC 128-byte K chunks per 3-D box);
+//   warps 7, 8  their scale atoms: a TMA box of the repacked layout, or, with
+//               the scale conversion fused (mxgemm_run), 4-byte cp.async
+//               gathers from the row-major scales;
+//   warps 1, 9.. MMA warps, up to four: each owns a run of the stage's scale
+//               atoms, copies them into TMEM (tcgen05.cp) and issues the
+//               block-scaled MMAs (kind::mxf8f6f4 K=32 / kind::mxf4 K=64) that
+//               read them into its own FP32 accumulator; its tcgen05.commit
+//               counts toward releasing the stage;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulators, summed in FP32,
+//               BF16 (RNE) through shared memory and TMA stores; for split
+//               tiles an FP32 partial plus a last-arriver fixup.
+// mx_gemm_pair_kernel: a cluster of two CTAs per 256x256 tile
+// (tcgen05.mma.cta_group::2); the leader's warp 7 copies both CTAs' scale
+// atoms, its warp 1 issues the MMAs, the peer's warp 1 relays its landed
+// stages.  Every instruction-issuing role has its own warp because a TMA or
+// tcgen05 instruction holds the issuing thread for tens to hundreds of ns.
 //
 // Work decomposition (stream-K family): the I = tiles * kt K-iterations of
 // all output tiles, tile-major, are cut into W contiguous ranges, one per
@@ -131,8 +140,6 @@ __host__ __device__ constexpr uint32_t idesc_base()
 }
 
 struct KParams {
-    const uint8_t *sfP;   // repacked scales of the MMA row operand
-    const uint8_t *sfQ;   // repacked scales of the MMA column operand
     __nv_bfloat16 *C;
     float *partials;
     uint32_t *counters;
@@ -141,13 +148,10 @@ struct KParams {
     int64_t ldc;           // = N
     uint32_t tilesP, kt, iters, workers;   // host guarantees iters * workers < 2^32
     int dp;                // workers == tiles: worker w is exactly tile w
-    int64_t kaP, kaQ;      // scale atoms per 128-row block
     uint64_t limit_ns;
     int swap;
     int inject;
     int tma_store;         // 1: epilogue stores C through shared memory with TMA
-    const uint8_t *opP;    // the MMA row operand (for whole-tile L2 prefetch)
-    int64_t rbytes;        // bytes per operand row
     // Fused scale conversion (1-CTA kernel): the scale producers gather each
     // stage's atoms from the row-major scales [rows][K/32] themselves instead
     // of loading the repacked layout.
@@ -1404,8 +1408,6 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
         !make_sf_map(&tmSQ, sfQ, pl.kaQ, sf_row_blocks(pl.Q), C_::kAtoms, C_::kRBQ))
         return cudaErrorInvalidValue;
     KParams kp;
-    kp.sfP = pl.swap ? b.sfB : b.sfA;
-    kp.sfQ = pl.swap ? b.sfA : b.sfB;
     kp.C = reinterpret_cast<__nv_bfloat16 *>(b.C);
     kp.partials = b.partials;
     kp.counters = b.counters;
@@ -1418,14 +1420,10 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     kp.iters = static_cast<uint32_t>(pl.iters);
     kp.workers = static_cast<uint32_t>(pl.workers);
     kp.dp = pl.workers == pl.tiles ? 1 : 0;
-    kp.kaP = pl.kaP;
-    kp.kaQ = pl.kaQ;
     kp.limit_ns = limit_ns;
     kp.swap = pl.swap;
     kp.inject = inject;
     kp.tma_store = tma_store;
-    kp.opP = static_cast<const uint8_t *>(Pptr);
-    kp.rbytes = rbytes;
     kp.fused_sf = fused ? 1 : 0;
     kp.rawP = rawP;
     kp.rawQ = rawQ;
@@ -1479,8 +1477,6 @@ cudaError_t launch_pair_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t lim
         !make_sf_map(&tmSQ, b.sfB, pl.kaQ, sf_row_blocks(pl.N), C_::kAtoms, 2))
         return cudaErrorInvalidValue;
     KParams kp;
-    kp.sfP = b.sfA;
-    kp.sfQ = b.sfB;
     kp.C = reinterpret_cast<__nv_bfloat16 *>(b.C);
     kp.partials = nullptr;
     kp.counters = nullptr;
@@ -1493,14 +1489,10 @@ cudaError_t launch_pair_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t lim
     kp.iters = static_cast<uint32_t>(pl.iters);
     kp.workers = static_cast<uint32_t>(pl.tiles);
     kp.dp = 1;
-    kp.kaP = pl.kaP;
-    kp.kaQ = pl.kaQ;
     kp.limit_ns = limit_ns;
     kp.swap = 0;
     kp.inject = inject;
     kp.tma_store = 1;
-    kp.opP = static_cast<const uint8_t *>(b.A);
-    kp.rbytes = rbytes;
     kp.fused_sf = 0;
     kp.rawP = nullptr;
     kp.rawQ = nullptr;

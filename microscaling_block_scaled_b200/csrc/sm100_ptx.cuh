@@ -105,29 +105,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
-// Wait for a long-pending phase (an epilogue waiting for a tile's whole
-// K loop): poll with __nanosleep backoff so the waiting warp gives its issue
-// slots to the producer and MMA warps that share its scheduler.  Bounded like
-// mbar_wait_bounded; a completed phase is seen within ~sleep_ns.
-__device__ __forceinline__ bool mbar_wait_sleepy(uint32_t bar, uint32_t parity, const volatile int *abort,
-                                                 uint64_t limit_ns, uint32_t sleep_ns)
-{
-    if (mbar_test_wait(bar, parity))
-        return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
-        __nanosleep(sleep_ns);
-        if (mbar_test_wait(bar, parity))
-            return true;
-        if ((i & 15u) == 0u) {
-            if (*abort)
-                return false;
-            if (globaltimer_ns() - t0 > limit_ns)
-                return false;
-        }
-    }
-}
-
 // Wait for a phase that may take a while without spending issue slots: the
 // suspending try_wait parks the thread in hardware until the phase completes
 // (or a hardware time slice passes), so a completed phase is seen at once.
@@ -178,22 +155,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int3
         " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(cache_hint)
         : "memory");
-}
-
-// Plain (untiled) bulk copy global -> shared; size and both addresses are
-// multiples of 16 bytes.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-        : "memory");
-}
-
-// Bring the 128-byte line holding `p` into L2 (no register result).
-__device__ __forceinline__ void prefetch_l2(const void *p)
-{
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)) : "memory");
 }
 
 // 4-byte asynchronous copy global -> shared (the non-bulk cp.async path):

@@ -196,14 +196,18 @@ def mxgemm_last_timing(h) -> tuple[int, float, float]:
 
 # ------------------------------------------------------- torch helpers
 
-def quantize(fmt: int, X, stream=None):
+def quantize(fmt: int, X, stream=None, out=None):
     """OCP MX quantisation of an FP32 CUDA tensor [R][K] on the device.
-    Returns (codes uint8 [R][row_bytes], scales uint8 [R][K/32])."""
+    Returns (codes uint8 [R][row_bytes], scales uint8 [R][K/32]), written into
+    `out` = (codes, scales) when given."""
     import torch
     assert X.is_cuda and X.dtype == torch.float32 and X.is_contiguous()
     R, K = X.shape
-    Q = torch.empty((R, row_bytes(fmt, K)), dtype=torch.uint8, device=X.device)
-    S = torch.empty((R, K // 32), dtype=torch.uint8, device=X.device)
+    if out is None:
+        Q = torch.empty((R, row_bytes(fmt, K)), dtype=torch.uint8, device=X.device)
+        S = torch.empty((R, K // 32), dtype=torch.uint8, device=X.device)
+    else:
+        Q, S = out
     _check("mxgemm_quantize", mxgemm_quantize(fmt, R, K, _ptr(X), _ptr(Q), _ptr(S), _stream_ptr(stream)))
     return Q, S
 

@@ -338,6 +338,9 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
             atomicCAS(kp.error, 0, kErrLaunch);
         return;
     }
+    // Every wait in this kernel parks the thread in the suspending try_wait
+    // at once: the producer and MMA warps share SM sub-partitions, and a
+    // warp spinning on test_wait would take issue slots from an MMA warp.
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const bool producer = warp == 0 || (warp >= 6 && warp <= 8);
@@ -406,7 +409,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         for (IterCursor cur(sc, blockIdx.x, gridDim.x); cur.valid(); cur.advance()) {
             int good = 1;
             if (lane == 0)
-                good = mbar_wait_bounded(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns);
+                good = mbar_wait_parked(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns);
             good = __shfl_sync(0xffffffffu, good, 0);
             if (!good) {
                 if (lane == 0)
@@ -467,7 +470,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
             int s = 0;
             uint32_t ph = 0;
             for (IterCursor cur(sc, blockIdx.x, gridDim.x); cur.valid(); cur.advance()) {
-                if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns)) {
+                if (!mbar_wait_parked(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns)) {
                     record_error(kp.error, kErrProducerEmpty, s_abort);
                     break;
                 }
@@ -514,7 +517,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                     continue;
                 const uint32_t parity = static_cast<uint32_t>((n - 1) & 1);
                 int dummy_abort = 0;
-                if (!mbar_wait_bounded(full_bar(st), parity, &dummy_abort, kp.limit_ns))
+                if (!mbar_wait_parked(full_bar(st), parity, &dummy_abort, kp.limit_ns))
                     atomicCAS(kp.error, 0, kErrDrain);
             }
         }
@@ -542,7 +545,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                 const uint32_t kb = sg.kb, ke = sg.ke;
                 int good = 1;
                 if (lane == 0)
-                    good = mbar_wait_bounded(acce_bar(acc), acc_ph ^ 1u, s_abort, kp.limit_ns);
+                    good = mbar_wait_parked(acce_bar(acc), acc_ph ^ 1u, s_abort, kp.limit_ns);
                 good = __shfl_sync(0xffffffffu, good, 0);
                 if (!good) {
                     if (lane == 0)
@@ -555,7 +558,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                 for (uint32_t k = kb; k < ke; ++k) {
                     good = 1;
                     if (lane == 0)
-                        good = mbar_wait_bounded(full_bar(s), ph, s_abort, kp.limit_ns);
+                        good = mbar_wait_parked(full_bar(s), ph, s_abort, kp.limit_ns);
                     good = __shfl_sync(0xffffffffu, good, 0);
                     if (!good) {
                         if (lane == 0)
@@ -627,7 +630,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         if (lane == 0) {
             tc_commit(drain_bar);
             int dummy_abort = 0;
-            if (!mbar_wait_bounded(drain_bar, 0, &dummy_abort, kp.limit_ns))
+            if (!mbar_wait_parked(drain_bar, 0, &dummy_abort, kp.limit_ns))
                 atomicCAS(kp.error, 0, kErrDrain);
         }
         __syncwarp();
@@ -996,7 +999,7 @@ __global__ void __launch_bounds__(256, 1)
                 const int32_t sf_rb = sideA ? static_cast<int32_t>(tp * 2 + rank) : static_cast<int32_t>(tq * 2);
                 bool ok = true;
                 for (uint32_t k = 0; k < KT; ++k) {
-                    if (!mbar_wait_bounded(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns)) {
+                    if (!mbar_wait_parked(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns)) {
                         record_error(kp.error, kErrProducerEmpty, s_abort);
                         ok = false;
                         break;
@@ -1035,7 +1038,7 @@ __global__ void __launch_bounds__(256, 1)
                 if (n == 0 || (st == skipped_stage && n == 1))
                     continue;
                 int dummy_abort = 0;
-                if (!mbar_wait_bounded(full_bar(st), (n - 1) & 1u, &dummy_abort, kp.limit_ns))
+                if (!mbar_wait_parked(full_bar(st), (n - 1) & 1u, &dummy_abort, kp.limit_ns))
                     atomicCAS(kp.error, 0, kErrDrain);
             }
         }
@@ -1048,7 +1051,7 @@ __global__ void __launch_bounds__(256, 1)
             bool ok = true;
             for (uint32_t tile = pair; tile < tiles && ok; tile += npairs) {
                 for (uint32_t k = 0; k < KT; ++k) {
-                    if (!mbar_wait_bounded(full_bar(s), ph, s_abort, kp.limit_ns)) {
+                    if (!mbar_wait_parked(full_bar(s), ph, s_abort, kp.limit_ns)) {
                         record_error(kp.error, kErrMmaFull, s_abort);
                         ok = false;
                         break;
@@ -1085,6 +1088,7 @@ __global__ void __launch_bounds__(256, 1)
             for (uint32_t k = 0; k < KT; ++k) {
                 good = 1;
                 if (lane == 0)
+                    // the MMA warp alone spins: it feeds the tensor pipe
                     good = mbar_wait_bounded(sfr_bar(s), ph, s_abort, kp.limit_ns);
                 good = __shfl_sync(0xffffffffu, good, 0);
                 if (!good) {
@@ -1134,7 +1138,7 @@ __global__ void __launch_bounds__(256, 1)
         if (lane == 0) {
             tc_commit_pair(drain_bar, 0x1);
             int dummy_abort = 0;
-            if (!mbar_wait_bounded(drain_bar, 0, &dummy_abort, kp.limit_ns))
+            if (!mbar_wait_parked(drain_bar, 0, &dummy_abort, kp.limit_ns))
                 atomicCAS(kp.error, 0, kErrDrain);
         }
         __syncwarp();
@@ -1154,7 +1158,7 @@ __global__ void __launch_bounds__(256, 1)
             for (uint32_t k = 0; k < KT; ++k) {
                 int good = 1;
                 if (lane == 0) {
-                    good = mbar_wait_bounded(full_bar(s), ph, s_abort, kp.limit_ns);
+                    good = mbar_wait_parked(full_bar(s), ph, s_abort, kp.limit_ns);
                     if (good)
                         good = mbar_wait_cluster_bounded(pfull_bar(s), ph, s_abort, kp.limit_ns);
                 }
@@ -1192,7 +1196,7 @@ __global__ void __launch_bounds__(256, 1)
         if (lane == 0) {
             tc_commit_pair(drain_bar, 0x1);
             int dummy_abort = 0;
-            if (!mbar_wait_bounded(drain_bar, 0, &dummy_abort, kp.limit_ns))
+            if (!mbar_wait_parked(drain_bar, 0, &dummy_abort, kp.limit_ns))
                 atomicCAS(kp.error, 0, kErrDrain);
         }
         __syncwarp();

@@ -449,3 +449,23 @@ def test_tolerance_ulp_rule():
     assert u[3] == 2.0 ** 0 and u[4] == 2.0 ** 0   # +-128
     assert np.isinf(u[5])
     assert u[6] == 2.0 ** -8          # just below 1.0
+
+
+def test_compare_accepts_and_rejects_by_the_rule():
+    """The parity comparison itself: within 1 ulp + 2^-18 * sum|ab| passes,
+    2 ulp with no magnitude term fails, and the NaN / +Inf / -Inf positions
+    must match exactly (an Inf of the wrong sign, or a NaN for a finite
+    value, fails)."""
+    one, one_up, one_up2 = 0x3F80, 0x3F81, 0x3F82       # 1, 1 + 2^-7, 1 + 2^-6
+    pinf, ninf, qnan = 0x7F80, 0xFF80, 0x7FC0
+    z = np.zeros(1)
+    ok, _ = oracle.compare(np.array([one_up], np.uint16), np.array([one], np.uint16), z)
+    assert ok                                            # exactly 1 ulp
+    ok, rep = oracle.compare(np.array([one_up2], np.uint16), np.array([one], np.uint16), z)
+    assert not ok and rep["n_bad"] == 1                  # 2 ulp
+    ok, _ = oracle.compare(np.array([one_up2], np.uint16), np.array([one], np.uint16), np.array([2.0 ** 11]))
+    assert ok                                            # 2^-18 * 2^11 = 2^-7 of extra slack
+    for got, ref, want in [(qnan, qnan, True), (pinf, pinf, True), (ninf, ninf, True),
+                           (pinf, ninf, False), (qnan, one, False), (one, qnan, False), (pinf, one, False)]:
+        ok, rep = oracle.compare(np.array([got], np.uint16), np.array([ref], np.uint16), z)
+        assert ok == want, (hex(got), hex(ref), rep)

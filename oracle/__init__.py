@@ -203,7 +203,8 @@ def compare(got_bits: np.ndarray, ref_bits: np.ndarray, abssum: np.ndarray):
         np.array_equal(inf_g & (got < 0), inf_r & (ref < 0)))
     fin = ~(nan_r | inf_r) & ~(nan_g | inf_g)
     tol = tolerance(ref_bits, abssum)
-    err = np.abs(got - ref)
+    with np.errstate(invalid="ignore"):      # inf - inf where both are infinite: not compared
+        err = np.abs(got - ref)
     bad = fin & ~(err <= tol)
     rep = {
         "n": int(got.size),

@@ -73,7 +73,14 @@ struct Cfg {
     static constexpr int kSFBBytes = kRBQ * kAtoms * 512;
     static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
     static constexpr int kCW = BN < 32 ? BN : 32;             // accumulator columns per epilogue chunk
-    static constexpr int kOutBytes = 128 * kCW * 2;           // one BF16 output chunk
+    // Output staging for TMA stores: two BF16 chunks of the 128-row tile.
+    // Tiles of at most 32 columns (decode, M <= 32) have none of their own
+    // and give the space to a fifth ring stage: a CTA's final tile stages its
+    // output in the then idle first ring stage, an earlier one stores from
+    // registers.
+    static constexpr bool kStaged = BN > 32;
+    static constexpr int kChunkOutBytes = 128 * kCW * 2;      // one BF16 output chunk
+    static constexpr int kOutBytes = kStaged ? kChunkOutBytes : 0;
     static constexpr int kSmemBudget = 227 * 1024 - 2048 - 2 * kOutBytes;
     static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
@@ -122,6 +129,7 @@ struct Cfg {
     static_assert(kStages >= 2, "at least two pipeline stages");
     static_assert(kAccCols + kSFCols <= kTmemCols, "TMEM budget");
     static_assert(kBChunk % 1024 == 0, "tiles must keep 1024-byte alignment");
+    static_assert(kStaged || 2 * kChunkOutBytes <= kABytes, "ring stage 0 holds two output chunks");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -644,6 +652,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         uint32_t acc_ph = 0;
         uint32_t out_chunks = 0;               // BF16 chunks staged so far (buffer = parity)
         bool stop = false;
+        bool ring_out = false;                 // this segment may stage its output in ring stage 0
 
         // The tile's accumulator is the sum of the NM MMA warps' accumulators.
         auto load_acc = [&](uint32_t t_acc, int c, float (&v)[CW]) {
@@ -668,12 +677,13 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         // output layout allows, else with predicated global stores.
         auto emit = [&](const float (&v)[CW], int64_t tp, int64_t qcol) {
             const int64_t p = tp * 128 + row;
-            if (!kp.tma_store) {
+            if (!kp.tma_store || !(C_::kStaged || ring_out)) {
                 store_bf16<CW>(out, p, qcol, v);
                 return;
             }
             const int b = static_cast<int>(out_chunks & 1u);
-            uint8_t *buf = smem + C_::kOffOut + b * C_::kOutBytes;
+            uint8_t *buf = C_::kStaged ? smem + C_::kOffOut + b * C_::kOutBytes
+                                       : smem + C_::kOffA + b * C_::kChunkOutBytes;
             if (etid == 0)
                 bulk_wait_group_read<1>();      // the store that last read this buffer is done
             named_bar_sync(1, 128);
@@ -714,6 +724,9 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                 const Segment sg = segment_at(sc, it, end);
                 const uint32_t tile = sg.tile, kb = sg.kb, ke = sg.ke;
                 const int64_t tp = sg.tp, tq = sg.tq;
+                // the CTA's final segment: once its accumulator is complete every
+                // stage has been consumed and no further loads are coming
+                ring_out = (w + gridDim.x >= W) && (it + (ke - kb) >= end);
                 int good = 1;
                 if (lane == 0)
                     good = mbar_wait_parked(accf_bar(acc), acc_ph, s_abort, kp.limit_ns);

@@ -139,16 +139,25 @@ class ClockSampler:
             self.max_mhz = None
         self.t = threading.Thread(target=self._loop, daemon=True)
 
+    def sample_now(self):
+        """One sample from the calling thread (the bench takes one while the
+        timed graph is executing, after its end event has been queued)."""
+        if not self.ok:
+            return
+        try:
+            mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+            rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            self.samples.append((mhz, rs))
+        except Exception:
+            pass
+
     def _loop(self):
+        # the first sample waits one period, so the thread does not compete
+        # with the launch of the timed region for the interpreter
         while not self._stop:
-            if self.active and self.ok:
-                try:
-                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
-                    rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                    self.samples.append((mhz, rs))
-                except Exception:
-                    pass
             time.sleep(self.period)
+            if self.active and not self._stop:
+                self.sample_now()
 
     def __enter__(self):
         self.t.start()
@@ -159,14 +168,8 @@ class ClockSampler:
         self.t.join(timeout=1)
 
     def summary(self):
-        if not self.samples:
-            if self.ok:   # region too short for the thread: one sample right now
-                try:
-                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
-                    rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                    self.samples.append((mhz, rs))
-                except Exception:
-                    pass
+        if not self.samples:     # no sample was taken in the region: one now
+            self.sample_now()
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
         reasons = set()
@@ -309,6 +312,9 @@ def run_ours(args):
     sets = [(qa.clone(), sa.clone(), qb.clone(), sb.clone(), torch.empty((M, N), dtype=torch.bfloat16, device=dev))
             for _ in range(nsets)]
     h = mxgemm.Handle()
+    # B (the weights) is never written by the step before: consecutive steps
+    # may overlap B's stream with the previous GEMM's tail
+    h.set_prefetch_b(True)
     plan = h.describe(fmt, M, N, K)
 
     def step(i, stream=None):
@@ -340,7 +346,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         return g, s
 
-    def timed(g, s):
+    def timed(g, s, probe=None):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
@@ -350,17 +356,19 @@ def run_ours(args):
         e0.record(launch)
         g.replay()
         e1.record(launch)
+        if probe is not None:                     # the GPU is still running the graph
+            probe()
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         return e0.elapsed_time(e1)
 
     g_step, s_step = capture(step, args.steps)
-    g_step.replay()                      # untimed replay (graph upload)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(local) as clk:     # NVML set up before the GPU's last untimed work
+        g_step.replay()                  # untimed replay (graph upload)
+        torch.cuda.synchronize()
         clk.active = True
-        ms = timed(g_step, s_step)
+        ms = timed(g_step, s_step, probe=clk.sample_now)
         clk.active = False
     clocks = clk.summary()
     # spread: the same graph replayed again (not part of `value`)
@@ -475,6 +483,8 @@ def run_ours(args):
                        "l2": "inputs rotate over %d copies (%.1f MB each, %.0f MB > 2x L2 %.0f MB)" % (
                            nsets, set_bytes / 1e6, nsets * set_bytes / 1e6, l2 / 1e6),
                        "timing": "CUDA graph of K steps, CUDA events on the launch stream",
+                       "chaining": "each step's GEMM is a programmatic dependent of the previous one; "
+                                   "B is promised constant (mxgemm_set_prefetch_b), A and C wait for it",
                        "plan": plan, "kernel_us": kernel_us, "gemm_us": gemm_us, "repack_us": rep_us,
                        "quantize_A": {"us": quant_us, "bytes": quant_bytes,
                                       "GB/s": quant_bytes / (quant_us * 1e-6) / 1e9,

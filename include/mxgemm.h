@@ -95,7 +95,11 @@ MXGEMM_API int mxgemm_destroy(mxgemm_handle h);
  * mxgemm_describe_plan, "scales=fused") the GEMM gathers the scales itself:
  * one kernel launch.  Otherwise the scales are repacked into the handle's
  * workspace first: two launches.  No host synchronisation.  All buffers are
- * device memory.  `stream` is a cudaStream_t (NULL = legacy default stream). */
+ * device memory.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ * The GEMM launches as a programmatic dependent of the work before it on
+ * `stream`: when that is a GEMM of this library, the new GEMM's CTAs set up
+ * while it finishes, and read or write no buffer before it has completed
+ * (except B under mxgemm_set_prefetch_b). */
 MXGEMM_API int mxgemm_run(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
                const void *A, const uint8_t *A_scales,
                const void *B, const uint8_t *B_scales,
@@ -135,6 +139,17 @@ MXGEMM_API int mxgemm_set_profiling(mxgemm_handle h, int on);
  * that run to finish.  MXGEMM_ERR_INVALID_ARG when profiling was off for the
  * last run, or for NULL arguments. */
 MXGEMM_API int mxgemm_last_timing(mxgemm_handle h, float *repack_ms, float *gemm_ms);
+
+/* Prefetch-B promise (an addition; the pages have no counterpart): with
+ * `on` = 1 the caller promises that B and B_scales of every later
+ * mxgemm_run on this handle are not written by the work queued before that
+ * call on its stream, as for the constant weights of a decode layer.  A
+ * one-launch mxgemm_run may then stream B into its pipeline while a
+ * preceding GEMM of this library still runs; A, A_scales and C still wait
+ * for it.  Results are unchanged; breaking the promise gives undefined
+ * results.  `on` = 0 (the default) withdraws it.  Returns
+ * MXGEMM_ERR_INVALID_ARG for a NULL handle or another value of `on`. */
+MXGEMM_API int mxgemm_set_prefetch_b(mxgemm_handle h, int on);
 
 /* OCP MX quantisation (the input generator; not part of the timed path).
  * X: FP32 [R][K] device.  Q: codes [R][row_bytes(K)] device.  scales: E8M0

@@ -46,6 +46,9 @@ struct mxgemm_ctx {
     int profiling = 0;
     cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
     int ev_valid = 0;
+    // caller's promise: B and its scales are not written by the work that
+    // precedes mxgemm_run on its stream (constant weights)
+    int prefetch_b = 0;
 };
 
 namespace {
@@ -134,9 +137,10 @@ bool fuse_scales(const mxg::GemmPlan &pl) { return pl.valid && !pl.pair && pl.st
 
 // GEMM launch.  With raw scales (SA, SB non-NULL) the kernel converts the
 // row-major scales itself; otherwise it reads the last repack's workspace,
-// which must be for this shape.
+// which must be for this shape.  pdl and early as mxg::launch_gemm and
+// GemmBuffers::early.
 int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const void *B, void *C,
-            cudaStream_t st, int pdl, const uint8_t *SA = nullptr, const uint8_t *SB = nullptr)
+            cudaStream_t st, int pdl, int early, const uint8_t *SA = nullptr, const uint8_t *SB = nullptr)
 {
     if (!SA && (h->last_fmt != fmt || h->last_M != M || h->last_N != N || h->last_K != K))
         return MXGEMM_ERR_INVALID_ARG;
@@ -161,6 +165,7 @@ int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const voi
     b.error = h->err;
     b.rawA = SA;
     b.rawB = SB;
+    b.early = early;
     const int inject = h->inject;
     h->inject = 0;
     if (mxg::launch_gemm(pl, b, h->limit_ns, inject, pdl, st) != cudaSuccess)
@@ -170,10 +175,13 @@ int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const voi
 
 // The hot path.  Plans on one CTA per tile convert the row-major scales
 // inside the GEMM (one launch); CTA-pair plans run the scale repack, then
-// the GEMM as a programmatic dependent of it.  With profiling on, events
-// bracket the launches (the middle event keeps the GEMM from starting
-// before the repack ends; with the conversion fused it records no repack
-// time).
+// the GEMM as a programmatic dependent of it.  The one-launch GEMM is itself
+// a programmatic dependent of whatever precedes it: its CTAs set up while a
+// previous GEMM of this library finishes, and read nothing before that GEMM
+// has completed, except B and its scales under the prefetch-B promise.
+// With profiling on, events bracket the launches and nothing overlaps (the
+// middle event keeps the GEMM from starting before the repack ends; with
+// the conversion fused it records no repack time).
 int repack_and_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const uint8_t *SA,
                     const void *B, const uint8_t *SB, void *C, cudaStream_t st)
 {
@@ -191,8 +199,8 @@ int repack_and_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
     }
     if (prof && cudaEventRecord(h->ev[1], st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
-    rc = fused ? do_gemm(h, fmt, M, N, K, A, B, C, st, 0, SA, SB)
-               : do_gemm(h, fmt, M, N, K, A, B, C, st, prof ? 0 : 1);
+    rc = fused ? do_gemm(h, fmt, M, N, K, A, B, C, st, prof ? 0 : 1, h->prefetch_b ? 2 : 0, SA, SB)
+               : do_gemm(h, fmt, M, N, K, A, B, C, st, prof ? 0 : 1, 3);
     if (rc != MXGEMM_OK)
         return rc;
     if (prof) {
@@ -303,7 +311,7 @@ int mxgemm_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const
         rc = enter_device(h);
     if (rc != MXGEMM_OK)
         return rc;
-    return do_gemm(h, fmt, M, N, K, A, B, C, static_cast<cudaStream_t>(stream), 0);
+    return do_gemm(h, fmt, M, N, K, A, B, C, static_cast<cudaStream_t>(stream), 0, 0);
 }
 
 int mxgemm_run(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const uint8_t *A_scales,
@@ -375,6 +383,14 @@ int mxgemm_set_profiling(mxgemm_handle h, int on)
                 return MXGEMM_ERR_CUDA;
     h->profiling = on;
     h->ev_valid = 0;
+    return MXGEMM_OK;
+}
+
+int mxgemm_set_prefetch_b(mxgemm_handle h, int on)
+{
+    if (!h || (on != 0 && on != 1))
+        return MXGEMM_ERR_INVALID_ARG;
+    h->prefetch_b = on;
     return MXGEMM_OK;
 }
 

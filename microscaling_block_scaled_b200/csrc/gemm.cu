@@ -44,6 +44,15 @@
 // Every wait is bounded in time; a wait that runs out records a site code in
 // a device error word, the CTA drains its in-flight copies and MMAs, frees
 // its tensor memory and exits normally.
+//
+// Launch chaining (programmatic dependent launch): mx_gemm_kernel lets the
+// next launch on its stream start as soon as its own CTAs are set up.  A
+// launch that starts early sets up its CTA (barriers, tensor memory, tensor
+// maps) while the previous kernel finishes, and every role waits for that
+// kernel (griddepcontrol.wait) before it touches global memory, except the
+// operand producers named in KParams::early, which may stream their operand
+// into the ring first.  They wait before their first blocking ring wait, so
+// no bounded wait ever spans the previous kernel's run time.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -166,6 +175,12 @@ struct KParams {
     int fused_sf;
     const uint8_t *rawP, *rawQ;   // row-major scales of the row / column operand
     int64_t ldS;                  // K / 32: scale bytes per row
+    // Operands that may be read before the prerequisite grid (the previous
+    // kernel on the stream, when launched as its programmatic dependent) has
+    // completed: bit 0 the row operand (P) with its row-major scales, bit 1
+    // the column operand (Q) with its row-major scales.  Repacked scales and
+    // C are always accessed after it.
+    int early;
 };
 
 // Error site codes written to the device error word.
@@ -395,6 +410,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
 
     const Sched sc{kp.iters, kp.workers, kp.kt, kp.tilesP, kp.dp != 0};
     const uint32_t W = sc.W;
+    // The CTA is set up: a programmatic dependent launch may start.
+    grid_launch_dependents();
 
     if (producer && kp.fused_sf && warp >= 7) {
         // ------------------------------------- scale atoms gathered directly
@@ -412,9 +429,19 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         const uint32_t off = sideP ? C_::kOffSFA : C_::kOffSFB;
         const int nrb = sideP ? 1 : C_::kRBQ;
         const int64_t kblocks = kp.ldS;
+        // scales of an early operand: gathered ahead until the ring is full
+        bool dep_pending = (kp.early & (sideP ? 1 : 2)) != 0;
+        if (!dep_pending)
+            grid_dependency_wait();
+        uint32_t issued = 0;
         int s = 0;
         uint32_t ph = 0;
         for (IterCursor cur(sc, blockIdx.x, gridDim.x); cur.valid(); cur.advance()) {
+            if (dep_pending && issued == static_cast<uint32_t>(S)) {
+                grid_dependency_wait();
+                dep_pending = false;
+            }
+            ++issued;
             int good = 1;
             if (lane == 0)
                 good = mbar_wait_parked(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns);
@@ -456,9 +483,9 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         // MMA row-operand tile, warp 6 the column-operand tile, warps 7 and 8
         // their scale atoms.  Issuing a TMA operation occupies the issuing
         // thread for ~0.1-0.15 us, so one thread per operation keeps the
-        // ring's refill off the critical path.  Operand tiles are never
-        // written by the kernel this one may overlap (the scale repack), so
-        // only the scale producers wait for it.
+        // ring's refill off the critical path.  An operand named in
+        // KParams::early fills the ring before the producer waits for the
+        // prerequisite grid; everything else waits first.
         // L2 policy: in the swapped (decode) form the weights stream through
         // once and the small activation is re-read by every tile; otherwise
         // both operands are re-read across tiles.
@@ -470,7 +497,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
             const uint32_t bytes = scales ? (sideP ? C_::kSFABytes : C_::kSFBBytes)
                                           : (sideP ? C_::kABytes : C_::kBBytes);
             const uint32_t off = scales ? (sideP ? C_::kOffSFA : C_::kOffSFB) : (sideP ? C_::kOffA : C_::kOffB);
-            if (scales)
+            bool dep_pending = !scales && (kp.early & (sideP ? 1 : 2)) != 0;
+            if (!dep_pending)
                 grid_dependency_wait();
             uint32_t armed = 0;         // stages armed so far (round-robin over the ring)
             int skipped_stage = -1;
@@ -478,6 +506,10 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
             int s = 0;
             uint32_t ph = 0;
             for (IterCursor cur(sc, blockIdx.x, gridDim.x); cur.valid(); cur.advance()) {
+                if (dep_pending && armed == static_cast<uint32_t>(S)) {
+                    grid_dependency_wait();
+                    dep_pending = false;
+                }
                 if (!mbar_wait_parked(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns)) {
                     record_error(kp.error, kErrProducerEmpty, s_abort);
                     break;
@@ -540,6 +572,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         const uint32_t t_sfa0 = tmem + C_::kAccCols;
         const uint32_t t_sfb0 = t_sfa0 + S * C_::kSFACols;
         const int a_begin = mma_idx * C_::kAtomsPerMma;
+        grid_dependency_wait();
         int s = 0;
         uint32_t ph = 0;
         int acc = 0;
@@ -1445,6 +1478,8 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     kp.rawP = rawP;
     kp.rawQ = rawQ;
     kp.ldS = pl.K / 32;
+    // bits of b.early are per operand (A, B); the kernel's are per side (P, Q)
+    kp.early = pl.swap ? (((b.early & 1) << 1) | ((b.early >> 1) & 1)) : b.early;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
     cfg.blockDim = dim3(C_::kThreads);
@@ -1514,6 +1549,7 @@ cudaError_t launch_pair_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t lim
     kp.rawP = nullptr;
     kp.rawQ = nullptr;
     kp.ldS = pl.K / 32;
+    kp.early = 3;              // this kernel's operand producers never wait (it follows the repack)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
     cfg.blockDim = dim3(C_::kThreads);

@@ -78,10 +78,15 @@ struct GemmBuffers {
     float *partials;
     uint32_t *counters;
     int *error;
+    // With pdl: operands that may be read before the preceding kernel has
+    // completed (bit 0 A, bit 1 B, each with its row-major scales).  Only
+    // safe where that kernel does not write them: the scale repack, or a
+    // caller's promise that B is constant.
+    int early = 0;
 };
-// pdl: launch as a programmatic dependent of the preceding kernel (the
-// scale repack of mxgemm_run), letting the prologue and the first operand
-// loads overlap it; the kernel waits for it before touching the scales.
+// pdl: launch as a programmatic dependent of the preceding kernel, letting
+// the prologue (and the operands named in buf.early) overlap its tail; every
+// other global access waits for it to complete.
 cudaError_t launch_gemm(const GemmPlan &plan, const GemmBuffers &buf, uint64_t wait_limit_ns, int inject, int pdl,
                         cudaStream_t stream);
 

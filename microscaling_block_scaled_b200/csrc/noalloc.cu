@@ -131,6 +131,7 @@ int mxgemm_run_noalloc(int fmt, int64_t M, int64_t N, int64_t K, const void *A, 
     b.partials = nullptr;      // whole tiles only: never touched
     b.counters = nullptr;
     b.error = err;
+    b.early = 3;               // the preceding kernel is the repack, which writes neither operand
     if (mxg::launch_gemm(pl, b, 2000000000ull, 0, 1, st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
     return MXGEMM_OK;

@@ -49,6 +49,7 @@ SIGNATURES = {
     "mxgemm_run_noalloc": (ctypes.c_int, [ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "mxgemm_set_profiling": (ctypes.c_int, [_vp, ctypes.c_int]),
     "mxgemm_last_timing": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
+    "mxgemm_set_prefetch_b": (ctypes.c_int, [_vp, ctypes.c_int]),
     "mxgemm_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mxgemm_version": (ctypes.c_char_p, []),
 }
@@ -188,6 +189,10 @@ def mxgemm_set_profiling(h, on: int) -> int:
     return load().mxgemm_set_profiling(h, on)
 
 
+def mxgemm_set_prefetch_b(h, on: int) -> int:
+    return load().mxgemm_set_prefetch_b(h, on)
+
+
 def mxgemm_last_timing(h) -> tuple[int, float, float]:
     rep, gem = ctypes.c_float(0.0), ctypes.c_float(0.0)
     st = load().mxgemm_last_timing(h, ctypes.byref(rep), ctypes.byref(gem))
@@ -272,6 +277,11 @@ class Handle:
 
     def set_profiling(self, on: bool):
         _check("mxgemm_set_profiling", mxgemm_set_profiling(self.h, 1 if on else 0))
+
+    def set_prefetch_b(self, on: bool):
+        """Promise that B of later runs is not written by the work queued
+        before them (constant weights); see mxgemm_set_prefetch_b."""
+        _check("mxgemm_set_prefetch_b", mxgemm_set_prefetch_b(self.h, 1 if on else 0))
 
     def last_timing(self) -> tuple[float, float]:
         """(repack_ms, gemm_ms) of the last profiled run on this handle."""

@@ -53,6 +53,7 @@ def test_run_rejects_null_handle(lib):
     assert mxgemm.mxgemm_set_schedule(None, 0, 1, 0) == mxgemm.ERR_INVALID_ARG
     assert mxgemm.mxgemm_debug_inject(None, 1) == mxgemm.ERR_INVALID_ARG
     assert mxgemm.mxgemm_set_profiling(None, 1) == mxgemm.ERR_INVALID_ARG
+    assert mxgemm.mxgemm_set_prefetch_b(None, 1) == mxgemm.ERR_INVALID_ARG
     assert mxgemm.mxgemm_last_timing(None)[0] == mxgemm.ERR_INVALID_ARG
 
 

@@ -63,3 +63,76 @@ def test_reference_arm_rank_other_than_zero_does_no_work(monkeypatch):
         workload = bench.DEFAULT_WORKLOAD
         steps, warmup, gpus, cpu_seconds = 1, 0, 2, 0.01
     assert bench.run_reference(A) == 0
+
+
+class _FakeNVML:
+    """Stands in for pynvml: a GPU at 1965 MHz (max 1965) whose throttle
+    reasons come from a list, one per query."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self, reasons):
+        self.reasons = list(reasons)
+        self.queries = 0
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetHandleByPciBusId(self, bus):
+        raise RuntimeError("no PCI lookup in the fake")
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return ("gpu", i)
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        self.queries += 1
+        return 1965 if self.queries % 2 else 1905
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.reasons.pop(0) if self.reasons else 0
+
+
+def test_clock_sampler_reasons_and_in_region_sample(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    fake = _FakeNVML([0x4 | 0x1, 0x40])          # sw_power_cap (+ idle, ignored), then hw_thermal_slowdown
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    clk = bench.ClockSampler(0, period=10.0)     # the thread never samples within the test
+    assert clk.ok and clk.max_mhz == 1965
+    with clk:
+        clk.active = True
+        clk.sample_now()                         # as the bench does inside the timed region
+        clk.sample_now()
+        clk.active = False
+    s = clk.summary()
+    assert s["samples"] == 2
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert s["sm_mhz"] == (1965 + 1905) / 2 and s["sm_max_mhz"] == 1965
+
+
+def test_clock_sampler_takes_one_sample_when_the_region_had_none(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setitem(sys.modules, "pynvml", _FakeNVML([]))
+    clk = bench.ClockSampler(0, period=10.0)
+    with clk:
+        pass
+    s = clk.summary()
+    assert s["samples"] == 1 and s["reasons"] == [] and s["sm_mhz"] == 1965
+
+
+def test_clock_sampler_without_nvml_reports_nothing(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class Broken:
+        def nvmlInit(self):
+            raise RuntimeError("no driver")
+    monkeypatch.setitem(sys.modules, "pynvml", Broken())
+    clk = bench.ClockSampler(0, period=10.0)
+    assert not clk.ok
+    with clk:
+        clk.sample_now()
+    assert clk.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}

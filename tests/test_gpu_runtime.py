@@ -75,3 +75,49 @@ def test_stalled_stage_times_out_and_handle_recovers(fmt, M, N, K):
     ok, rep = oracle.compare(bits(C), ref, mag)
     assert ok, rep
     h.close()
+
+
+@pytest.mark.parametrize("prefetch_b", [False, True], ids=["plain", "prefetch_b"])
+def test_back_to_back_runs_wait_for_the_previous_gemm(prefetch_b):
+    """Two one-launch runs queued back to back with no synchronisation.  The
+    second starts as a programmatic dependent of the first, so its CTAs can
+    be resident while the first still runs.  It reads the first one's output
+    as its A operand (read after write) and writes its C over the first
+    one's A operand (write after read): both must see the first GEMM
+    complete.  Under the prefetch-B promise only B may be read early.  The
+    second GEMM is MXFP4, whose codes are all finite, so any byte pattern of
+    the first output is a valid operand."""
+    torch.cuda.set_device(0)
+    h = mxgemm.Handle()
+    h.set_prefetch_b(prefetch_b)
+    M, N1, K1 = 32, 512, 16384
+    N2, K2 = 2048, 4 * N1                   # A2 = the bytes of C1, two E2M1 codes per byte
+    assert "scales=fused" in h.describe(F8, M, N1, K1)
+    assert "scales=fused" in h.describe(F4, M, N2, K2)
+    A1f, B1f = synth.operands(M, N1, K1, seed=71, device="cuda")
+    qa1, sa1 = mxgemm.quantize(F8, A1f)
+    qb1, sb1 = mxgemm.quantize(F8, B1f)
+    _, B2f = synth.operands(M, N2, K2, seed=72, device="cuda")
+    qb2, sb2 = mxgemm.quantize(F4, B2f)
+    sa2 = torch.full((M, K2 // 32), 120, dtype=torch.uint8, device="cuda")
+    # the first GEMM alone, on a copy of its A
+    C1_ref = h.run(F8, qa1.clone(), sa1, qb1, sb1, K=K1)
+    torch.cuda.synchronize()
+    # the chain: C1 starts zeroed; C2 is laid over the first half of A1
+    C1 = torch.zeros((M, N1), dtype=torch.bfloat16, device="cuda")
+    C2 = qa1.view(-1)[: M * N2 * 2].view(torch.bfloat16).view(M, N2)
+    h.run(F8, qa1, sa1, qb1, sb1, C=C1, K=K1)
+    h.run(F4, C1.view(torch.uint8), sa2, qb2, sb2, C=C2, K=K2)
+    torch.cuda.synchronize()
+    st, code = h.check_device_error()
+    assert st == mxgemm.OK and code == 0, code
+    assert np.array_equal(bits(C1), bits(C1_ref)), "the second GEMM wrote A1 before the first one read it"
+    # the second GEMM again, alone, from the final C1
+    a2 = C1.view(torch.uint8).clone()
+    C2_ref = h.run(F4, a2, sa2, qb2, sb2, K=K2)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(C2), bits(C2_ref)), "the second GEMM read A before the first one wrote it"
+    ref, _, mag = oracle.gemm(F4, K2, a2.cpu().numpy(), sa2.cpu().numpy(), qb2.cpu().numpy(), sb2.cpu().numpy())
+    ok, rep = oracle.compare(bits(C2_ref), ref, mag)
+    assert ok, rep
+    h.close()

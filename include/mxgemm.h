@@ -174,13 +174,21 @@ MXGEMM_API int mxgemm_set_kchunks(mxgemm_handle h, int kc);
 
 /* Describe the plan mxgemm_gemm would use for a shape: writes up to `cap`
  * bytes of a NUL-terminated text such as
- * "fmt=1 swap=1 pair=0 BN=32 kc=2 stages=4 tiles=112 kt=8 workers=112
+ * "fmt=1 swap=1 pair=0 BN=32 kc=2 stages=5 tiles=112 kt=8 workers=112
  * grid=112 sched=dp partial_bytes=0 scales=fused".  The last field says how
  * mxgemm_run treats the scales for this shape: "fused" (the GEMM converts
  * the row-major scales itself, one launch) or "repack" (scale repack, then
  * the GEMM). */
 MXGEMM_API int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
                          char *buf, size_t cap);
+
+/* The same text for a device with `num_sms` SMs (2 to 4096) and the
+ * automatic schedule, without a handle: it touches no GPU, so the planner
+ * can be queried for capacity planning on any host.  Returns
+ * MXGEMM_ERR_INVALID_ARG for a NULL or empty buffer, an SM count out of
+ * range, or a shape mxgemm_run would reject. */
+MXGEMM_API int mxgemm_describe_plan_for(int num_sms, int fmt, int64_t M, int64_t N, int64_t K,
+                             char *buf, size_t cap);
 
 /* Read and clear the device error word that kernels set when a bounded wait
  * runs out.  Synchronises the device.  *code receives 0 if no kernel gave

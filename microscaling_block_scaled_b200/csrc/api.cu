@@ -442,14 +442,8 @@ int mxgemm_set_kchunks(mxgemm_handle h, int kc)
     return MXGEMM_OK;
 }
 
-int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, char *buf, size_t cap)
+static void format_plan(const mxg::GemmPlan &pl, char *buf, size_t cap)
 {
-    if (!h || !buf || cap == 0)
-        return MXGEMM_ERR_INVALID_ARG;
-    int rc = check_shape(fmt, M, N, K);
-    if (rc != MXGEMM_OK)
-        return rc;
-    const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks);
     static const char *names[] = {"auto", "dp", "splitk", "streamk"};
     snprintf(buf, cap,
              "fmt=%d swap=%d pair=%d BN=%d kc=%d stages=%d tiles=%lld kt=%lld workers=%lld grid=%d sched=%s "
@@ -457,6 +451,27 @@ int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t
              pl.fmt, pl.swap, pl.pair, pl.bn, pl.kc, pl.stages, static_cast<long long>(pl.tiles), static_cast<long long>(pl.kt),
              static_cast<long long>(pl.workers), pl.grid, names[pl.sched & 3],
              static_cast<long long>(pl.partial_bytes), fuse_scales(pl) ? "fused" : "repack");
+}
+
+int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, char *buf, size_t cap)
+{
+    if (!h || !buf || cap == 0)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = check_shape(fmt, M, N, K);
+    if (rc != MXGEMM_OK)
+        return rc;
+    format_plan(mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks), buf, cap);
+    return MXGEMM_OK;
+}
+
+int mxgemm_describe_plan_for(int num_sms, int fmt, int64_t M, int64_t N, int64_t K, char *buf, size_t cap)
+{
+    if (!buf || cap == 0 || num_sms < 2 || num_sms > 4096)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = check_shape(fmt, M, N, K);
+    if (rc != MXGEMM_OK)
+        return rc;
+    format_plan(mxg::make_plan(fmt, M, N, K, num_sms, MXGEMM_SCHED_AUTO, 1, 0, 0), buf, cap);
     return MXGEMM_OK;
 }
 

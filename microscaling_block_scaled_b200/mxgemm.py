@@ -43,6 +43,8 @@ SIGNATURES = {
     "mxgemm_set_schedule": (ctypes.c_int, [_vp, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "mxgemm_set_kchunks": (ctypes.c_int, [_vp, ctypes.c_int]),
     "mxgemm_describe_plan": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, ctypes.c_char_p, ctypes.c_size_t]),
+    "mxgemm_describe_plan_for": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _i64, _i64, _i64, ctypes.c_char_p,
+                                                ctypes.c_size_t]),
     "mxgemm_check_device_error": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_int)]),
     "mxgemm_set_wait_limit": (ctypes.c_int, [_vp, ctypes.c_uint64]),
     "mxgemm_debug_inject": (ctypes.c_int, [_vp, ctypes.c_int]),
@@ -168,6 +170,14 @@ def mxgemm_set_kchunks(h, kc) -> int:
 def mxgemm_describe_plan(h, fmt, M, N, K) -> str:
     buf = ctypes.create_string_buffer(256)
     _check("mxgemm_describe_plan", load().mxgemm_describe_plan(h, fmt, M, N, K, buf, 256))
+    return buf.value.decode()
+
+
+def mxgemm_describe_plan_for(num_sms, fmt, M, N, K) -> str:
+    """The plan text for a device with ``num_sms`` SMs and the automatic
+    schedule; needs no handle and no GPU."""
+    buf = ctypes.create_string_buffer(256)
+    _check("mxgemm_describe_plan_for", load().mxgemm_describe_plan_for(num_sms, fmt, M, N, K, buf, 256))
     return buf.value.decode()
 
 

@@ -125,6 +125,16 @@ def quantize(fmt: int, X: np.ndarray):
     return Q, S
 
 
+def quantize_bf16(fmt: int, C_bits: np.ndarray):
+    """OCP MX quantisation of a BF16 matrix given by its bit patterns [R][K]
+    (uint16): each value widens exactly to FP32, then ``quantize`` applies.
+    This is the form in which a GEMM's BF16 result becomes the MX operand of
+    the next layer (one E8M0 scale per 32 consecutive values of a row, as
+    the 5ulink.com page's support matrix fixes for MX operands)."""
+    b = np.ascontiguousarray(C_bits, dtype=np.uint16).astype(np.uint32) << 16
+    return quantize(fmt, b.view(np.float32))
+
+
 def gemm(fmt: int, K: int, A: np.ndarray, SA: np.ndarray, B: np.ndarray, SB: np.ndarray,
          want_exact: bool = False):
     """C = A * B^T for MX operands.  Returns (C_bf16_bits [M][N] uint16,

@@ -469,3 +469,51 @@ def test_compare_accepts_and_rejects_by_the_rule():
                            (pinf, ninf, False), (qnan, one, False), (one, qnan, False), (pinf, one, False)]:
         ok, rep = oracle.compare(np.array([got], np.uint16), np.array([ref], np.uint16), z)
         assert ok == want, (hex(got), hex(ref), rep)
+
+
+# ------------------------------------------- MX quantisation of BF16 output
+
+def test_quantize_bf16_hand_worked_block():
+    # one block of a row: 1.0, 2.0, then 30 zeros.  amax 2 = 2^1.
+    #  MXFP8: scale exponent 1 - 8 = -7 (byte 120); 1 * 2^7 = 128 = 2^7 -> E4M3
+    #  exponent field 7 + 7 = 14, mantissa 0 -> 0x70; 256 -> field 15 -> 0x78.
+    #  MXFP4: scale exponent 1 - 2 = -1 (byte 126); 1 * 2 = 2.0 -> E2M1 0b0100,
+    #  2 * 2 = 4.0 -> 0b0110; packed low nibble first -> 0x64.
+    bits = np.zeros((1, 32), dtype=np.uint16)
+    bits[0, 0], bits[0, 1] = 0x3F80, 0x4000
+    Q8, S8 = oracle.quantize_bf16(oracle.FMT_MXFP8, bits)
+    assert S8.tolist() == [[120]] and Q8[0, 0] == 0x70 and Q8[0, 1] == 0x78 and not Q8[0, 2:].any()
+    Q4, S4 = oracle.quantize_bf16(oracle.FMT_MXFP4, bits)
+    assert S4.tolist() == [[126]] and Q4[0, 0] == 0x64 and not Q4[0, 1:].any()
+
+
+@pytest.mark.parametrize("fmt", [oracle.FMT_MXFP8, oracle.FMT_MXFP4])
+def test_quantize_bf16_matches_ml_dtypes_widening_and_independent_rule(fmt):
+    rng = np.random.default_rng(31)
+    # BF16 bit patterns of finite values over a wide exponent range, some
+    # blocks zero, some negative zero
+    v = (rng.standard_normal((12, 256)) * np.exp2(rng.integers(-30, 30, (12, 1)))).astype(np.float32)
+    v[3, 64:96] = 0.0
+    v[5, 0:32] = -0.0
+    bits = v.astype(ml_dtypes.bfloat16).view(np.uint16)
+    Q, S = oracle.quantize_bf16(fmt, bits)
+    widened = bits.view(ml_dtypes.bfloat16).astype(np.float32)
+    Qr, Sr = _independent_quantize(fmt, widened)
+    assert np.array_equal(S, Sr) and np.array_equal(Q, Qr)
+
+
+def test_quantize_bf16_exact_round_trip_for_representable_blocks():
+    # BF16 values with at most 3 mantissa bits, within 2^8 of the block's
+    # amax binade and with significand at most 1.75 (the block amax scales to
+    # 2^8 times its significand, and 1.875 * 2^8 = 480 would saturate to 448)
+    # are E4M3 values times the block scale: MXFP8 reproduces them.
+    rng = np.random.default_rng(32)
+    mant = rng.integers(8, 15, (4, 64)).astype(np.float64) / 8.0          # 1.mmm, mmm <= 110
+    expo = rng.integers(-5, 3, (4, 64)).astype(np.float64)
+    sign = np.where(rng.random((4, 64)) < 0.5, -1.0, 1.0)
+    x = (sign * mant * np.exp2(expo)).astype(np.float32)
+    bits = x.astype(ml_dtypes.bfloat16).view(np.uint16)
+    assert np.array_equal(bits.view(ml_dtypes.bfloat16).astype(np.float32), x)   # exact in BF16
+    Q, S = oracle.quantize_bf16(oracle.FMT_MXFP8, bits)
+    dec = e4m3_values()[Q].reshape(4, 2, 32) * e8m0_values()[S][..., None]
+    assert np.array_equal(dec.reshape(4, 64), x.astype(np.float64))

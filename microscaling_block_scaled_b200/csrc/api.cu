@@ -448,7 +448,8 @@ static void format_plan(const mxg::GemmPlan &pl, char *buf, size_t cap)
     snprintf(buf, cap,
              "fmt=%d swap=%d pair=%d BN=%d kc=%d stages=%d tiles=%lld kt=%lld workers=%lld grid=%d sched=%s "
              "partial_bytes=%lld scales=%s",
-             pl.fmt, pl.swap, pl.pair, pl.bn, pl.kc, pl.stages, static_cast<long long>(pl.tiles), static_cast<long long>(pl.kt),
+             pl.fmt, pl.swap, pl.pair, pl.bn, pl.kc, pl.stages, static_cast<long long>(pl.tiles),
+             static_cast<long long>(pl.kt),
              static_cast<long long>(pl.workers), pl.grid, names[pl.sched & 3],
              static_cast<long long>(pl.partial_bytes), fuse_scales(pl) ? "fused" : "repack");
 }

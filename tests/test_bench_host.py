@@ -1,0 +1,70 @@
+"""Host arithmetic of bench.py, on CPU: the roofline's algorithmic bytes
+and flops, the measured-peak lookup and its fallback, and the rule that a
+recorded DRAM traffic figure is used only for the kernel source it was
+captured on."""
+import json
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+# Per-workload totals worked out independently of bench.py (A and B read
+# once, one E8M0 byte per 32 elements of each row, BF16 C written once).
+@pytest.mark.parametrize("fmt,M,N,K,alg_bytes", [
+    (0, 32, 256, 512, 168_448),
+    (1, 32, 14336, 4096, 32_182_272),
+    (0, 64, 4096, 4096, 18_096_128),
+    (1, 64, 4096, 4096, 9_576_448),
+    (0, 2048, 28672, 8192, 376_963_072),
+    (1, 2048, 28672, 8192, 251_133_952),
+    (0, 8192, 8192, 8192, 272_629_760),
+    (1, 8192, 8192, 8192, 205_520_896),
+    (0, 4096, 4096, 14336, 154_664_960),
+    (1, 4096, 4096, 14336, 95_944_704),
+])
+def test_algorithmic_bytes_of_the_workloads(fmt, M, N, K, alg_bytes):
+    assert bench.algorithmic_bytes(fmt, M, N, K) == alg_bytes
+    assert bench.flops(M, N, K) == 2.0 * M * N * K
+
+
+def test_every_named_workload_resolves():
+    from microscaling_block_scaled_b200 import synth
+    for name in synth.WORKLOADS:
+        fmt_name, M, N, K, seed, kind = bench.workload(name)
+        assert fmt_name in ("mxfp8", "mxfp4") and K % 128 == 0 and kind in ("normal", "heavy")
+    assert bench.DEFAULT_WORKLOAD in synth.WORKLOADS
+    with pytest.raises(SystemExit):
+        bench.workload("no_such_workload")
+
+
+def test_measured_peaks_and_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, how = bench.measured_peaks()
+    assert how == "fallback" and peaks["hbm_gbs"] == 6650.0 and peaks["bf16_tflops"] == 1590.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 7000.0, "bf16_tflops": 1700.0}))
+    peaks, how = bench.measured_peaks()
+    assert how == "measured" and peaks["hbm_gbs"] == 7000.0
+
+
+def test_recorded_traffic_only_for_the_captured_source(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("mxfp4_32x14336x4096") is None          # no file
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(
+        {"mxfp4_32x14336x4096": {"kernel_hash": "aaaa", "dram_bytes_per_launch": 123}}))
+    monkeypatch.setattr(bench, "kernel_hash", lambda: "aaaa")
+    assert bench.recorded_traffic("mxfp4_32x14336x4096") == 123
+    assert bench.recorded_traffic("mxfp8_32x256x512") is None               # not captured
+    monkeypatch.setattr(bench, "kernel_hash", lambda: "bbbb")
+    assert bench.recorded_traffic("mxfp4_32x14336x4096") is None            # kernel changed since
+
+
+def test_kernel_hash_covers_the_kernel_sources():
+    h = bench.kernel_hash()
+    assert len(h) == 16 and int(h, 16) >= 0
+    assert any(p.endswith("gemm.cu") for p in bench.KERNEL_SOURCES)

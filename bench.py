@@ -35,7 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MX scaled-GEMM TFLOPS (MXFP8/MXFP4, NT) and % of roofline on 1 B200"
-DEFAULT_WORKLOAD = "mxfp4_32x14336x4096"
+DEFAULT_WORKLOAD = "mxfp8_8192x8192x8192"
 KERNEL_SOURCES = ["microscaling_block_scaled_b200/csrc/gemm.cu", "microscaling_block_scaled_b200/csrc/sm100_ptx.cuh"]
 
 
@@ -59,6 +59,13 @@ def workload(name):
         raise SystemExit("unknown workload %s; one of %s" % (name, sorted(synth.WORKLOADS)))
     fmt_name, M, N, K, seed, kind = synth.WORKLOADS[name]
     return fmt_name, M, N, K, seed, kind
+
+
+def base_config(name):
+    """The workload description both arms print, word for word."""
+    fmt_name, M, N, K, seed, kind = workload(name)
+    return {"workload": name, "fmt": fmt_name, "M": M, "N": N, "K": K, "seed": seed,
+            "inputs": "%s FP32 (torch generator, seed %d), OCP MX quantised, untimed" % (kind, seed)}
 
 
 def flops(M, N, K):
@@ -253,8 +260,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(times) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": fmt_name,
         "data": "synthetic",
-        "config": {"workload": args.workload, "fmt": fmt_name, "M": M, "N": N, "K": K, "seed": seed,
-                   "inputs": kind},
+        "config": base_config(args.workload),
         "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -477,8 +483,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": fmt_name, "data": "synthetic",
-            "config": {"workload": args.workload, "fmt": fmt_name, "M": M, "N": N, "K": K, "seed": seed,
-                       "inputs": "%s FP32 from torch CUDA generator, quantised on device (OCP MX), untimed" % kind,
+            "config": dict(base_config(args.workload), **{
                        "parallelism": "replicas" if world > 1 else "single",
                        "l2": "inputs rotate over %d copies (%.1f MB each, %.0f MB > 2x L2 %.0f MB)" % (
                            nsets, set_bytes / 1e6, nsets * set_bytes / 1e6, l2 / 1e6),
@@ -493,7 +498,7 @@ def run_ours(args):
                                           "min": min(reps) if reps else None, "max": max(reps) if reps else None},
                        "step_kernels": "mx_gemm_kernel with fused scale conversion" if fused
                        else "mx_repack_kernel + " + roof["kernel"],
-                       "gemm_tflops": flops(M, N, K) / (gemm_us * 1e-6) / 1e12},
+                       "gemm_tflops": flops(M, N, K) / (gemm_us * 1e-6) / 1e12}),
             "clocks": clocks,
             "roofline": roof,
             "cpu_baseline": cpu,

@@ -68,7 +68,8 @@ enum {
     MXGEMM_ERR_OOM = 4,                /* workspace allocation failed */
     MXGEMM_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
     MXGEMM_ERR_TIMEOUT = 6,            /* a kernel gave up on a bounded wait */
-    MXGEMM_ERR_TOO_LARGE = 7           /* exceeds mxgemm_run_noalloc's fixed scratch */
+    MXGEMM_ERR_TOO_LARGE = 7,          /* exceeds mxgemm_run_noalloc's fixed scratch */
+    MXGEMM_ERR_CAPTURE = 8             /* the workspace would have to grow during stream capture */
 };
 
 /* Schedules for the GEMM's persistent tile scheduler (mxgemm_set_schedule). */
@@ -82,7 +83,14 @@ enum {
 /* Create a handle bound to the current CUDA device.  The device must be an
  * sm_100 part (B200).  The handle owns a lazily grown device workspace
  * (repacked scales, split-K partials and tile counters).
- * out: receives the handle (host pointer, not NULL). */
+ * out: receives the handle (host pointer, not NULL).
+ *
+ * Workspace and CUDA graphs: the first run of a shape that needs more
+ * workspace than the handle holds grows it with cudaFree + cudaMalloc, which
+ * synchronises the device and cannot be recorded by a stream capture.  Run
+ * each shape once (or call mxgemm_reserve for it) before capturing; a run
+ * that would have to grow the workspace while its stream is capturing
+ * returns MXGEMM_ERR_CAPTURE and launches nothing. */
 MXGEMM_API int mxgemm_create(mxgemm_handle *out);
 
 /* Free the handle and its workspace (synchronises the device first).
@@ -104,6 +112,13 @@ MXGEMM_API int mxgemm_run(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_
                const void *A, const uint8_t *A_scales,
                const void *B, const uint8_t *B_scales,
                void *C, void *stream);
+
+/* Grow the handle's workspace now to what mxgemm_run needs for this shape
+ * under the handle's current schedule settings (an addition; the pages have
+ * no counterpart), so that later runs of this shape or smaller ones allocate
+ * nothing and can be captured into a CUDA graph.  Synchronises the device
+ * when it allocates.  Returns MXGEMM_ERR_OOM when the allocation fails. */
+MXGEMM_API int mxgemm_reserve(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K);
 
 /* The first half of mxgemm_run on its own: the scale repack into the
  * handle's workspace.  Sizes as for mxgemm_run. */

@@ -80,11 +80,22 @@ int check_ptrs(std::initializer_list<const void *> ptrs)
     return MXGEMM_OK;
 }
 
+// Grow a workspace buffer to at least `need` bytes.  Growing allocates
+// device memory (and frees the old buffer), which a stream capture cannot
+// record: while `st` is capturing, a buffer that must grow gives
+// MXGEMM_ERR_CAPTURE and nothing is allocated.
 template <typename T>
-int grow(T **buf, size_t *cap, size_t need, bool zero)
+int grow(T **buf, size_t *cap, size_t need, bool zero, cudaStream_t st)
 {
     if (need <= *cap)
         return MXGEMM_OK;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+        cudaGetLastError();
+        return MXGEMM_ERR_CUDA;
+    }
+    if (cs != cudaStreamCaptureStatusNone)
+        return MXGEMM_ERR_CAPTURE;
     if (*buf) {
         cudaFree(*buf);
         *buf = nullptr;
@@ -117,7 +128,7 @@ int do_repack(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const u
 {
     const int64_t ba = mxg::sf_repacked_bytes(fmt, M, K);
     const int64_t bb = mxg::sf_repacked_bytes(fmt, N, K);
-    int rc = grow(&h->sf, &h->sf_cap, static_cast<size_t>(ba + bb), false);
+    int rc = grow(&h->sf, &h->sf_cap, static_cast<size_t>(ba + bb), false, st);
     if (rc != MXGEMM_OK)
         return rc;
     h->sf_offB = ba;
@@ -148,10 +159,10 @@ int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const voi
     if (!pl.valid)
         return MXGEMM_ERR_INVALID_ARG;
     int rc = grow(&h->partials, &h->partials_cap, static_cast<size_t>(pl.partial_bytes > 0 ? pl.partial_bytes : 16),
-                  false);
+                  false, st);
     if (rc != MXGEMM_OK)
         return rc;
-    rc = grow(&h->counters, &h->counters_cap, static_cast<size_t>(pl.counter_bytes), true);
+    rc = grow(&h->counters, &h->counters_cap, static_cast<size_t>(pl.counter_bytes), true, st);
     if (rc != MXGEMM_OK)
         return rc;
     mxg::GemmBuffers b;
@@ -228,6 +239,8 @@ const char *mxgemm_status_string(int status)
     case MXGEMM_ERR_CUDA: return "CUDA call failed";
     case MXGEMM_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
     case MXGEMM_ERR_TOO_LARGE: return "problem exceeds the fixed scratch of mxgemm_run_noalloc (8 MiB of scales)";
+    case MXGEMM_ERR_CAPTURE:
+        return "the workspace must grow, which cannot happen during stream capture: run or reserve this shape first";
     default: return "unknown status";
     }
 }
@@ -350,10 +363,10 @@ int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
     const size_t nSB = static_cast<size_t>(N) * static_cast<size_t>(K / 32);
     const size_t nC = static_cast<size_t>(M) * static_cast<size_t>(N) * 2;
     const size_t oA = 0, oSA = oA + up16(nA), oB = oSA + up16(nSA), oSB = oB + up16(nB), oC = oSB + up16(nSB);
-    rc = grow(&h->stage, &h->stage_cap, oC + up16(nC), false);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = grow(&h->stage, &h->stage_cap, oC + up16(nC), false, st);
     if (rc != MXGEMM_OK)
         return rc;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *d = h->stage;
     if (cudaMemcpyAsync(d + oA, A_host, nA, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(d + oSA, A_scales_host, nSA, cudaMemcpyHostToDevice, st) != cudaSuccess ||
@@ -368,6 +381,29 @@ int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
     if (cudaStreamSynchronize(st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
     return MXGEMM_OK;
+}
+
+int mxgemm_reserve(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K)
+{
+    if (!h)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = check_shape(fmt, M, N, K);
+    if (rc == MXGEMM_OK)
+        rc = enter_device(h);
+    if (rc != MXGEMM_OK)
+        return rc;
+    const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks);
+    if (!pl.valid)
+        return MXGEMM_ERR_INVALID_ARG;
+    const size_t sf = static_cast<size_t>(mxg::sf_repacked_bytes(fmt, M, K) + mxg::sf_repacked_bytes(fmt, N, K));
+    cudaStream_t st = nullptr;
+    rc = grow(&h->sf, &h->sf_cap, sf, false, st);
+    if (rc == MXGEMM_OK)
+        rc = grow(&h->partials, &h->partials_cap,
+                  static_cast<size_t>(pl.partial_bytes > 0 ? pl.partial_bytes : 16), false, st);
+    if (rc == MXGEMM_OK)
+        rc = grow(&h->counters, &h->counters_cap, static_cast<size_t>(pl.counter_bytes), true, st);
+    return rc;
 }
 
 int mxgemm_set_profiling(mxgemm_handle h, int on)

@@ -28,6 +28,7 @@ ERR_OOM = 4
 ERR_CUDA = 5
 ERR_TIMEOUT = 6
 ERR_TOO_LARGE = 7
+ERR_CAPTURE = 8
 
 # Entry points and their C signatures (restype, argtypes).
 _i64 = ctypes.c_int64
@@ -36,6 +37,7 @@ SIGNATURES = {
     "mxgemm_create": (ctypes.c_int, [ctypes.POINTER(_vp)]),
     "mxgemm_destroy": (ctypes.c_int, [_vp]),
     "mxgemm_run": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "mxgemm_reserve": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64]),
     "mxgemm_repack": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp]),
     "mxgemm_gemm": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
     "mxgemm_run_host": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -123,6 +125,10 @@ def mxgemm_destroy(h: int) -> None:
 
 def mxgemm_run(h, fmt, M, N, K, A, SA, B, SB, C, stream) -> int:
     return load().mxgemm_run(h, fmt, M, N, K, A, SA, B, SB, C, stream)
+
+
+def mxgemm_reserve(h, fmt, M, N, K) -> int:
+    return load().mxgemm_reserve(h, fmt, M, N, K)
 
 
 def mxgemm_repack(h, fmt, M, N, K, SA, SB, stream) -> int:
@@ -246,6 +252,10 @@ class Handle:
 
     def set_schedule(self, schedule: int, splits: int = 1, workers: int = 0):
         _check("mxgemm_set_schedule", mxgemm_set_schedule(self.h, schedule, splits, workers))
+
+    def reserve(self, fmt, M, N, K):
+        """Grow the workspace for this shape now (before a stream capture)."""
+        _check("mxgemm_reserve", mxgemm_reserve(self.h, fmt, M, N, K))
 
     def set_kchunks(self, kc: int):
         _check("mxgemm_set_kchunks", mxgemm_set_kchunks(self.h, kc))

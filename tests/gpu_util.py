@@ -92,6 +92,47 @@ def sampled_case(fmt: int, M: int, N: int, K: int, seed: int, kind: str = "norma
     return rep
 
 
+def rows_cols_points_case(fmt: int, M: int, N: int, K: int, seed: int, kind: str = "normal", n_rows: int = 64,
+                          n_cols: int = 64, n_points: int = 65536, rng_seed: int = 4321):
+    """Full-size run with inputs drawn by the CUDA generator, checked against
+    the oracle on n_rows whole rows of C (every column), n_cols whole columns
+    (every row) and n_points random elements.  The first and last row and
+    column are always among them, so every output tile of the GEMM has
+    checked elements.  Both operands are quantised in full on the host and
+    must agree with the device quantiser bit for bit."""
+    A32, B32 = synth.operands(M, N, K, seed=seed, kind=kind, device="cuda")
+    qa, sa = mxgemm.quantize(fmt, A32)
+    qb, sb = mxgemm.quantize(fmt, B32)
+    h = handle()
+    C = h.run(fmt, qa, sa, qb, sb, K=K)
+    torch.cuda.synchronize()
+    st, code = h.check_device_error()
+    assert st == mxgemm.OK and code == 0, ("device error word", code)
+    plan = h.describe(fmt, M, N, K)
+    got_all = bits(C)
+    assert bool(torch.isfinite(C.float()).all())
+    del C
+    oa, osa = oracle.quantize(fmt, A32.cpu().numpy())
+    assert np.array_equal(qa.cpu().numpy(), oa) and np.array_equal(sa.cpu().numpy(), osa), "A quantiser mismatch"
+    del A32, qa, sa
+    ob, osb = oracle.quantize(fmt, B32.cpu().numpy())
+    assert np.array_equal(qb.cpu().numpy(), ob) and np.array_equal(sb.cpu().numpy(), osb), "B quantiser mismatch"
+    del B32, qb, sb
+    torch.cuda.empty_cache()
+    rng = np.random.default_rng(rng_seed)
+    rm = np.unique(np.concatenate([[0, M - 1], rng.choice(M, min(n_rows, M) - 2, replace=False)]))
+    rn = np.unique(np.concatenate([[0, N - 1], rng.choice(N, min(n_cols, N) - 2, replace=False)]))
+    ref, _, mag = oracle.gemm(fmt, K, oa[rm], osa[rm], ob, osb)
+    assert_parity(got_all[rm], ref, mag, "whole rows fmt=%d %dx%dx%d" % (fmt, M, N, K))
+    ref, _, mag = oracle.gemm(fmt, K, oa, osa, ob[rn], osb[rn])
+    assert_parity(got_all[:, rn], ref, mag, "whole columns fmt=%d %dx%dx%d" % (fmt, M, N, K))
+    pm = rng.integers(0, M, n_points)
+    pn = rng.integers(0, N, n_points)
+    ref, _, mag = oracle.gemm_points(fmt, K, oa, osa, ob, osb, pm, pn)
+    assert_parity(got_all[pm, pn], ref, mag, "random points fmt=%d %dx%dx%d" % (fmt, M, N, K))
+    return plan, len(rm), len(rn)
+
+
 def rows_case(fmt: int, M: int, N: int, K: int, seed: int, n_rows: int = 48, rng_seed: int = 7):
     """CPU-drawn inputs, GPU GEMM through mxgemm_run, oracle on a sample of
     whole output rows (every column of those rows)."""

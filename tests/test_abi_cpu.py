@@ -41,6 +41,7 @@ def test_status_strings(lib):
     assert mxgemm.status_string(mxgemm.OK) == "ok"
     assert "bounded wait" in mxgemm.status_string(mxgemm.ERR_TIMEOUT)
     assert mxgemm.status_string(999) == "unknown status"
+    assert "capture" in mxgemm.status_string(mxgemm.ERR_CAPTURE)
     assert re.match(r"^\d+\.\d+\.\d+$", mxgemm.version())
 
 
@@ -55,6 +56,7 @@ def test_run_rejects_null_handle(lib):
     assert mxgemm.mxgemm_set_profiling(None, 1) == mxgemm.ERR_INVALID_ARG
     assert mxgemm.mxgemm_set_prefetch_b(None, 1) == mxgemm.ERR_INVALID_ARG
     assert mxgemm.mxgemm_last_timing(None)[0] == mxgemm.ERR_INVALID_ARG
+    assert mxgemm.mxgemm_reserve(None, 0, 1, 1, 128) == mxgemm.ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("fmt,R,K,align,expect", [

@@ -11,7 +11,7 @@ import torch
 import oracle
 from microscaling_block_scaled_b200 import mxgemm, synth
 
-from gpu_util import assert_parity, bits, full_case, handle, rows_case, sampled_case
+from gpu_util import assert_parity, bits, full_case, handle, rows_case, rows_cols_points_case, sampled_case
 
 pytestmark = pytest.mark.gpu
 
@@ -127,50 +127,111 @@ def test_gemm_cta_pair_tiles(fmt, kc, M, N, K):
 
 
 # ----------------------------------------------------------- edge cases
+#
+# Every edge case runs through every execution path of the GEMM: the small
+# shape under the automatic plan (one-CTA whole tiles, swapped when M <= 64),
+# a shape that takes the CTA pair (cta_group::2, 256x256 tiles), and forced
+# split-K and stream-K schedules on one-CTA tiles, where the output is the
+# FP32 sum of per-worker partials (last-arriver fixup).  NaN and +-Inf
+# patterns must come out identical on every path.
 
-def _codes_case(fmt, A, SA, B, SB, K):
+PATHS = {
+    # name: (shape override or None, schedule or None)
+    "auto": (None, None),
+    "pair": ((512, 8192, 384), None),
+    "splitk3": ((200, 640, 2048), (mxgemm.SCHED_SPLITK, 3, 0)),
+    "splitk8": ((200, 640, 2048), (mxgemm.SCHED_SPLITK, 8, 0)),
+    "streamk148": ((200, 640, 2048), (mxgemm.SCHED_STREAMK, 1, 148)),
+    "streamk37": ((200, 640, 2048), (mxgemm.SCHED_STREAMK, 1, 37)),
+    "swap-splitk3": ((40, 1024, 2048), (mxgemm.SCHED_SPLITK, 3, 0)),
+    "swap-streamk148": ((40, 1024, 2048), (mxgemm.SCHED_STREAMK, 1, 148)),
+}
+
+
+def _shape(path, default):
+    return PATHS[path][0] or default
+
+
+def _codes_case(fmt, A, SA, B, SB, K, path="auto"):
     h = handle()
     ta = torch.from_numpy(A).cuda()
     tb = torch.from_numpy(B).cuda()
     tsa = torch.from_numpy(SA).cuda()
     tsb = torch.from_numpy(SB).cuda()
-    C = h.run(fmt, ta, tsa, tb, tsb, K=K)
-    torch.cuda.synchronize()
+    M, N = A.shape[0], B.shape[0]
+    sched = PATHS[path][1]
+    if sched is not None:
+        h.set_schedule(*sched)
+    try:
+        plan = h.describe(fmt, M, N, K)
+        C = h.run(fmt, ta, tsa, tb, tsb, K=K)
+        torch.cuda.synchronize()
+    finally:
+        if sched is not None:
+            h.set_schedule(mxgemm.SCHED_AUTO)
+    st, code = h.check_device_error()
+    assert st == mxgemm.OK and code == 0, ("device error word", code)
+    # the path the case is meant to exercise is the one that ran
+    if path == "pair":
+        assert "pair=1" in plan, plan
+    elif path.startswith("split") or path.startswith("swap-split"):
+        assert "sched=splitk" in plan and "pair=0" in plan, plan
+    elif "streamk" in path:
+        assert "sched=streamk" in plan and "pair=0" in plan, plan
+    if path.startswith("swap"):
+        assert "swap=1" in plan, plan
     ref, _, mag = oracle.gemm(fmt, K, A, SA, B, SB)
     return bits(C), ref, mag
 
 
-@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
-def test_gemm_nan_scales_and_zero_blocks(fmt):
-    rng = np.random.default_rng(17)
-    M, N, K = 70, 160, 384
+def _random_codes(rng, fmt, rows, K):
     rb = oracle.row_bytes(fmt, K)
-    A = rng.integers(0, 256, (M, rb), dtype=np.uint8)
-    B = rng.integers(0, 256, (N, rb), dtype=np.uint8)
+    X = rng.integers(0, 256, (rows, rb), dtype=np.uint8)
     if fmt == F8:
-        A[(A & 0x7F) == 0x7F] = 0x35
-        B[(B & 0x7F) == 0x7F] = 0x4A
+        X[(X & 0x7F) == 0x7F] = 0x35       # no NaN codes here
+    return X
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("path", list(PATHS))
+def test_gemm_nan_scales_and_zero_blocks(fmt, path):
+    rng = np.random.default_rng(17)
+    M, N, K = _shape(path, (70, 160, 384))
+    A = _random_codes(rng, fmt, M, K)
+    B = _random_codes(rng, fmt, N, K)
     SA = rng.integers(110, 140, (M, K // 32), dtype=np.uint8)
     SB = rng.integers(110, 140, (N, K // 32), dtype=np.uint8)
+    nan_rows = sorted({3, M - 2})
+    nan_cols = sorted({7, N - 3})
     SA[3, 5] = 0xFF                        # NaN scale in A: row 3 all NaN
+    SA[M - 2, K // 32 - 1] = 0xFF          # ... and a row in the last tile, last K block
     SB[7, 0] = 0xFF                        # NaN scale in B: column 7 all NaN
-    blk = 32 * rb // K
+    SB[N - 3, K // 64] = 0xFF              # ... and a column in the last tile, mid K
+    blk = 32 * oracle.row_bytes(fmt, K) // K
     A[10, 2 * blk:3 * blk] = 0             # an all-zero block
     B[20, :] = 0                           # an all-zero column
-    got, ref, mag = _codes_case(fmt, A, SA, B, SB, K)
-    assert_parity(got, ref, mag, "nan scales")
+    got, ref, mag = _codes_case(fmt, A, SA, B, SB, K, path)
+    assert_parity(got, ref, mag, "nan scales (%s)" % path)
     gv = oracle.bf16_bits_to_f64(got)
-    assert np.isnan(gv[3]).all() and np.isnan(gv[:, 7]).all()
-    assert (gv[np.arange(M) != 3, 20] == 0).all()
+    for r in nan_rows:
+        assert np.isnan(gv[r]).all()
+    for c in nan_cols:
+        assert np.isnan(gv[:, c]).all()
+    keep = np.ones(M, bool)
+    keep[nan_rows] = False
+    assert (gv[keep, 20] == 0).all()
+    assert np.isfinite(gv[np.ix_(keep, [0, 1, 2, 20])]).all()
 
 
 @pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
-def test_gemm_overflow_and_underflow_scales(fmt):
+@pytest.mark.parametrize("path", list(PATHS))
+def test_gemm_overflow_and_underflow_scales(fmt, path):
     """Positive elements (no cancellation) with extreme scales: 2^127 * 2^127
     overflows BF16 to +Inf, 2^-95 * 2^-95 underflows to 0, mixed pairs give
-    normal results."""
+    normal results.  With positive elements every partial sum of a split
+    schedule overflows exactly when the total does."""
     rng = np.random.default_rng(23)
-    M, N, K = 130, 140, 256
+    M, N, K = _shape(path, (130, 140, 256))
     if fmt == F8:
         A = rng.integers(0x08, 0x7F, (M, K), dtype=np.uint8)
         B = rng.integers(0x08, 0x7F, (N, K), dtype=np.uint8)
@@ -185,32 +246,41 @@ def test_gemm_overflow_and_underflow_scales(fmt):
     SA[6, :] = 0x20
     SB[9, :] = 0xFE
     SB[10, :] = 0x20
-    got, ref, mag = _codes_case(fmt, A, SA, B, SB, K)
-    assert_parity(got, ref, mag, "extreme scales")
+    SA[M - 1, :] = 0xFE                    # a row of the last tile (the pair's odd CTA)
+    SB[N - 1, :] = 0xFE                    # a column of the last tile
+    got, ref, mag = _codes_case(fmt, A, SA, B, SB, K, path)
+    assert_parity(got, ref, mag, "extreme scales (%s)" % path)
     gv = oracle.bf16_bits_to_f64(got)
     assert np.isposinf(gv[5, 9]) and np.isposinf(gv[5, 0]) and gv[6, 10] == 0.0
     assert np.isfinite(gv[5, 10]) and gv[5, 10] > 0
+    assert np.isposinf(gv[M - 1, N - 1]) and np.isposinf(gv[M - 1, 0]) and np.isposinf(gv[0, N - 1])
 
 
-def test_gemm_nan_elements_e4m3():
+@pytest.mark.parametrize("path", list(PATHS))
+def test_gemm_nan_elements_e4m3(path):
     rng = np.random.default_rng(5)
-    M, N, K = 40, 72, 256
+    M, N, K = _shape(path, (40, 72, 256))
     A = rng.integers(0, 0x70, (M, K), dtype=np.uint8)
     B = rng.integers(0, 0x70, (N, K), dtype=np.uint8)
     A[5, 17] = 0x7F                        # E4M3 NaN element
-    B[9, 200] = 0xFF
+    B[9, K - 56] = 0xFF
+    A[M - 1, K // 2] = 0xFF                # last row, middle of K
     SA = np.full((M, K // 32), 0x7F, np.uint8)
     SB = np.full((N, K // 32), 0x7F, np.uint8)
-    got, ref, mag = _codes_case(F8, A, SA, B, SB, K)
-    assert_parity(got, ref, mag, "nan elements")
+    got, ref, mag = _codes_case(F8, A, SA, B, SB, K, path)
+    assert_parity(got, ref, mag, "nan elements (%s)" % path)
+    gv = oracle.bf16_bits_to_f64(got)
+    assert np.isnan(gv[5]).all() and np.isnan(gv[:, 9]).all() and np.isnan(gv[M - 1]).all()
 
 
 @pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
-def test_gemm_integer_exact(fmt):
+@pytest.mark.parametrize("path", list(PATHS))
+def test_gemm_integer_exact(fmt, path):
     """All scales 1 and small integer elements: every output is an exact
-    integer (a textbook integer matmul) and must match exactly."""
+    integer (a textbook integer matmul) and must match exactly, whatever the
+    order in which the FP32 partial sums are added."""
     rng = np.random.default_rng(8)
-    M, N, K = 96, 200, 512
+    M, N, K = _shape(path, (96, 200, 512))
     vals = np.arange(-16, 17) if fmt == F8 else np.array([0, 1, 2, 3, 4, 6, -1, -2, -3, -4, -6])
     ai = rng.choice(vals, (M, K))
     bi = rng.choice(vals, (N, K))
@@ -223,11 +293,11 @@ def test_gemm_integer_exact(fmt):
         eb = (eb[:, 0::2] | (eb[:, 1::2] << 4)).astype(np.uint8)
     S1 = np.full((M, K // 32), 0x7F, np.uint8)
     S2 = np.full((N, K // 32), 0x7F, np.uint8)
-    got, ref, mag = _codes_case(fmt, ea, S1, eb, S2, K)
+    got, ref, mag = _codes_case(fmt, ea, S1, eb, S2, K, path)
     exact = ai.astype(np.int64) @ bi.astype(np.int64).T
     small = np.abs(exact) <= 256           # exactly representable in BF16
     assert np.array_equal(oracle.bf16_bits_to_f64(got)[small], exact[small].astype(np.float64))
-    assert_parity(got, ref, mag, "integer")
+    assert np.array_equal(got, ref)        # exact FP32 sums: the one BF16 rounding is the oracle's
 
 
 # -------------------------------------------------------- entry points
@@ -300,8 +370,13 @@ def test_decode_workloads_sampled(fmt, M, N, K, seed):
 
 @pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
 @pytest.mark.parametrize("M,N,K", [(2048, 28672, 8192), (8192, 8192, 8192), (4096, 4096, 14336)])
-def test_prefill_workloads_sampled(fmt, M, N, K):
-    sampled_case(fmt, M, N, K, seed=3, n_rows=96, n_cols=96)
+def test_prefill_workloads_rows_cols_points(fmt, M, N, K):
+    """The prefill workloads at full size, in the launch configuration the
+    benchmark times: 64 whole rows, 64 whole columns and 65 536 random
+    elements of C against the oracle."""
+    plan, nr, nc = rows_cols_points_case(fmt, M, N, K, seed=3)
+    assert "pair=1" in plan, plan
+    assert nr == 64 and nc == 64
 
 
 @pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])

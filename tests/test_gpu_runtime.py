@@ -121,3 +121,34 @@ def test_back_to_back_runs_wait_for_the_previous_gemm(prefetch_b):
     ok, rep = oracle.compare(bits(C2_ref), ref, mag)
     assert ok, rep
     h.close()
+
+
+def test_capture_needs_a_reserved_workspace():
+    """A run whose shape needs a larger workspace than the handle holds cannot
+    grow it inside a stream capture: it returns MXGEMM_ERR_CAPTURE and
+    launches nothing.  After mxgemm_reserve the same run captures, and the
+    replayed graph gives the oracle's result."""
+    torch.cuda.set_device(0)
+    h = mxgemm.Handle()
+    fmt, M, N, K = F8, 512, 8192, 512          # CTA-pair plan: repacked scales in the workspace
+    (qa, sa, qb, sb), (ref, mag) = _operands(fmt, M, N, K, seed=63)
+    C = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        st = mxgemm.mxgemm_run(h.h, fmt, M, N, K, qa.data_ptr(), sa.data_ptr(), qb.data_ptr(), sb.data_ptr(),
+                               C.data_ptr(), s.cuda_stream)
+    assert st == mxgemm.ERR_CAPTURE, st
+    del g
+    h.reserve(fmt, M, N, K)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        st = mxgemm.mxgemm_run(h.h, fmt, M, N, K, qa.data_ptr(), sa.data_ptr(), qb.data_ptr(), sb.data_ptr(),
+                               C.data_ptr(), s.cuda_stream)
+    assert st == mxgemm.OK, st
+    g.replay()
+    torch.cuda.synchronize()
+    ok, rep = oracle.compare(bits(C), ref, mag)
+    assert ok, rep
+    del g
+    h.close()

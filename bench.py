@@ -23,6 +23,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import itertools
 import json
 import math
 import os
@@ -36,7 +37,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MX scaled-GEMM TFLOPS (MXFP8/MXFP4, NT) and % of roofline on 1 B200"
 DEFAULT_WORKLOAD = "mxfp8_8192x8192x8192"
-KERNEL_SOURCES = ["microscaling_block_scaled_b200/csrc/gemm.cu", "microscaling_block_scaled_b200/csrc/sm100_ptx.cuh"]
+KERNEL_SOURCES = ["microscaling_block_scaled_b200/csrc/gemm_kernel.cuh", "microscaling_block_scaled_b200/csrc/sm100_ptx.cuh",
+                  "microscaling_block_scaled_b200/csrc/mx_convert.cuh"]
 
 
 def parse():
@@ -56,16 +58,58 @@ def parse():
 def workload(name):
     from microscaling_block_scaled_b200 import synth
     if name not in synth.WORKLOADS:
-        raise SystemExit("unknown workload %s; one of %s" % (name, sorted(synth.WORKLOADS)))
+        raise SystemExit("unknown workload %s; one of %s" % (name, sorted(synth.WORKLOADS) +
+                                                             sorted(synth.EXTRA_WORKLOADS)))
     fmt_name, M, N, K, seed, kind = synth.WORKLOADS[name]
     return fmt_name, M, N, K, seed, kind
 
 
+def extra_workload(name):
+    """The extension workloads (dense BF16, grouped, fused epilogue,
+    quantised output): their description dict, or None."""
+    from microscaling_block_scaled_b200 import synth
+    w = synth.EXTRA_WORKLOADS.get(name)
+    if w is None:
+        return None
+    w = dict(w)
+    if w["op"] == "grouped":
+        w["M"] = int(sum(w["groups"]))
+    return w
+
+
 def base_config(name):
     """The workload description both arms print, word for word."""
+    w = extra_workload(name)
+    if w is not None:
+        cfg = {"workload": name, "op": w["op"], "fmt": w["fmt"], "M": w["M"], "N": w["N"], "K": w["K"],
+               "seed": w["seed"], "inputs": "normal FP32 (torch generator, seed %d), %s, untimed" % (
+                   w["seed"], "rounded to BF16" if w["fmt"] == "bf16" else "OCP MX quantised")}
+        for k in ("groups", "act", "out_fmt"):
+            if k in w:
+                cfg[k] = list(w[k]) if k == "groups" else w[k]
+        return cfg
     fmt_name, M, N, K, seed, kind = workload(name)
     return {"workload": name, "fmt": fmt_name, "M": M, "N": N, "K": K, "seed": seed,
             "inputs": "%s FP32 (torch generator, seed %d), OCP MX quantised, untimed" % (kind, seed)}
+
+
+def extra_bytes_flops(w):
+    """Algorithmic bytes (every input read once, every output written once)
+    and flops of one extension step."""
+    M, N, K = w["M"], w["N"], w["K"]
+    fl = 2.0 * M * N * K
+    if w["op"] == "bf16":
+        return 2 * M * K + 2 * N * K + 2 * M * N, fl
+    fmt = 0 if w["fmt"] == "mxfp8" else 1
+    rb = K if fmt == 0 else K // 2
+    if w["op"] == "grouped":
+        live = sum(1 for g in w["groups"] if g > 0)
+        return M * (rb + K // 32) + live * N * (rb + K // 32) + 2 * M * N, fl
+    base = M * (rb + K // 32) + N * (rb + K // 32)
+    if w["op"] == "fused":
+        return base + 2 * N + 2 * M * N + 2 * M * N, fl        # bias, residual read, C written
+    orb = N if w["out_fmt"] == 0 else N // 2
+    return base + M * (orb + N // 32), fl                      # codes + scales written
 
 
 def flops(M, N, K):
@@ -204,18 +248,29 @@ class OracleSampler:
         self.oracle = oracle
         self.fmt, self.M, self.N, self.K = fmt, M, N, K
         rng = np.random.default_rng(seed)
-        self.nm = min(M, 32)
-        rm = np.sort(rng.choice(M, self.nm, replace=False))
+        self.nm = min(M, 32, A32.shape[0])
+        rm = np.sort(rng.choice(A32.shape[0], self.nm, replace=False))
         a = A32[torch.from_numpy(rm).to(A32.device)].float().cpu().numpy()
-        self.oa, self.osa = oracle.quantize(fmt, a)
-        self.pool = min(N, 4096)
-        rn = np.sort(rng.choice(N, self.pool, replace=False))
+        self.pool = min(N, 4096, B32.shape[0])
+        rn = np.sort(rng.choice(B32.shape[0], self.pool, replace=False))
         b = B32[torch.from_numpy(rn).to(B32.device)].float().cpu().numpy()
-        self.ob, self.osb = oracle.quantize(fmt, b)
+        if fmt == 2:                       # dense BF16 operands
+            import ml_dtypes
+            self.oa = a.astype(ml_dtypes.bfloat16).view(np.uint16)
+            self.ob = b.astype(ml_dtypes.bfloat16).view(np.uint16)
+            self.osa = self.osb = None
+        else:
+            self.oa, self.osa = oracle.quantize(fmt, a)
+            self.ob, self.osb = oracle.quantize(fmt, b)
         t0 = time.perf_counter()
         nn0 = min(self.pool, 32)
-        oracle.gemm(fmt, K, self.oa, self.osa, self.ob[:nn0], self.osb[:nn0])
+        self._product(nn0)
         self.sec_per_col = max(time.perf_counter() - t0, 1e-5) / nn0
+
+    def _product(self, nn):
+        if self.fmt == 2:
+            return self.oracle.gemm_bf16(self.oa, self.ob[:nn])
+        return self.oracle.gemm(self.fmt, self.K, self.oa, self.osa, self.ob[:nn], self.osb[:nn])
 
     def run(self, target_s):
         """One timed sample: the sampled rows against as many sampled columns as
@@ -225,7 +280,7 @@ class OracleSampler:
         reps = 0
         t0 = time.perf_counter()
         while True:
-            self.oracle.gemm(self.fmt, self.K, self.oa, self.osa, self.ob[:nn], self.osb[:nn])
+            self._product(nn)
             reps += 1
             dt = time.perf_counter() - t0
             if dt >= 0.9 * target_s or nn < self.pool:
@@ -241,11 +296,16 @@ def run_reference(args):
     if rank != 0:
         return 0
     from microscaling_block_scaled_b200 import synth
-    fmt_name, M, N, K, seed, kind = workload(args.workload)
-    fmt = 0 if fmt_name == "mxfp8" else 1
+    w = extra_workload(args.workload)
+    if w is not None:
+        # extension workloads: the oracle's product underneath the op, sampled
+        fmt_name, M, N, K, seed, kind = w["fmt"], w["M"], w["N"], w["K"], w["seed"], "normal"
+    else:
+        fmt_name, M, N, K, seed, kind = workload(args.workload)
+    fmt = 0 if fmt_name == "mxfp8" else (1 if fmt_name == "mxfp4" else 2)
     # the whole run stays within a few minutes: split the budget over the steps
     per_step = max(0.05, min(args.cpu_seconds, 120.0 / max(1, args.steps + args.warmup)))
-    A32, B32 = synth.operands(M, N, K, seed=seed, kind=kind, device="cpu")
+    A32, B32 = synth.operands(min(M, 64), min(N, 4096), K, seed=seed, kind=kind, device="cpu")
     sampler = OracleSampler(fmt, M, N, K, A32, B32)
     times, vals = [], []
     desc = cores = None
@@ -288,6 +348,162 @@ def job_tflops(fmt_flops, world, steps, ms):
     """Whole-job throughput: every rank runs `steps` replicas of the GEMM in
     the slowest rank's `ms` milliseconds."""
     return fmt_flops * world * steps / (ms * 1e-3) / 1e12
+
+
+def run_extra(args, w):
+    """Times one extension op (see extra_workload) as the step: CUDA graph of
+    K steps on rotating inputs, CUDA events on the launch stream; e2e with the
+    inputs copied from pinned host memory and the output copied back in every
+    step."""
+    import torch
+    import torch.distributed as dist
+
+    from microscaling_block_scaled_b200 import mxgemm, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    op, M, N, K = w["op"], w["M"], w["N"], w["K"]
+    fmt = mxgemm.FMT_NAMES[w["fmt"]]
+    Bn = N * len(w["groups"]) if op == "grouped" else N
+    A32, B32 = synth.operands(M, Bn, K, seed=w["seed"], device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w["seed"] + 1000)
+    if op == "bf16":
+        ins = [A32.to(torch.bfloat16), B32.to(torch.bfloat16)]
+    else:
+        qa, sa = mxgemm.quantize(fmt, A32)
+        qb, sb = mxgemm.quantize(fmt, B32)
+        ins = [qa, sa, qb, sb]
+    extra = []
+    if op == "fused":
+        extra = [torch.randn(N, generator=gen, device=dev).to(torch.bfloat16),
+                 torch.randn(M, N, generator=gen, device=dev).to(torch.bfloat16)]
+    if op == "grouped":
+        offs = torch.tensor([0] + list(itertools.accumulate(w["groups"])), dtype=torch.int64, device=dev)
+    del A32, B32
+    abytes, fl = extra_bytes_flops(w)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    nsets = max(2, math.ceil(2 * l2 / abytes) + 1)
+
+    def outputs():
+        if op == "quantized":
+            return [torch.empty((M, mxgemm.row_bytes(w["out_fmt"], N)), dtype=torch.uint8, device=dev),
+                    torch.empty((M, N // 32), dtype=torch.uint8, device=dev)]
+        return [torch.empty((M, N), dtype=torch.bfloat16, device=dev)]
+
+    sets = [([t.clone() for t in ins], [t.clone() for t in extra], outputs()) for _ in range(nsets)]
+    h = mxgemm.Handle()
+    h.set_prefetch_b(True)
+
+    def call(i_set, stream):
+        x, e, o = sets[i_set % nsets]
+        if op == "bf16":
+            h.run_bf16(x[0], x[1], C=o[0], stream=stream)
+        elif op == "grouped":
+            h.run_grouped(fmt, offs, x[0], x[1], x[2].view(len(w["groups"]), N, -1), x[3], C=o[0], K=K,
+                          stream=stream)
+        elif op == "fused":
+            h.run_fused(fmt, x[0], x[1], x[2], x[3], bias=e[0], act=w["act"], residual=e[1], C=o[0], K=K,
+                        stream=stream)
+        else:
+            h.run_quantized(fmt, x[0], x[1], x[2], x[3], w["out_fmt"], out=(o[0], o[1]), K=K, stream=stream)
+
+    for i in range(args.warmup):
+        call(i, None)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        call(0, s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        for i in range(args.steps):
+            call(i, s)
+    g.replay()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        clk.active = True
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        st = torch.cuda.current_stream()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        g.replay()
+        e1.record(st)
+        clk.sample_now()
+        torch.cuda.synchronize()
+        clk.active = False
+        ms = e0.elapsed_time(e1)
+    clocks = clk.summary()
+    del g
+    ms = max_over_ranks([ms], dev)[0]
+    us = ms / args.steps * 1e3
+    peaks, peak_src = measured_peaks()
+    tc_peak = peaks["bf16_tflops"] * (1.0 if op == "bf16" else (2.0 if fmt == 0 else 4.0))
+    hbm = peaks["hbm_gbs"]
+    t_tc, t_hbm = fl / (tc_peak * 1e12), abytes / (hbm * 1e9)
+    if t_hbm >= t_tc:
+        ach = abytes / (us * 1e-6) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm}
+    else:
+        ach = fl / (us * 1e-6) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": tc_peak, "unit": "TFLOP/s", "frac": ach / tc_peak}
+    roof.update({"traffic": None, "peak_source": peak_src, "kernel": "mx_gemm_kernel (one-CTA)",
+                 "algorithmic_bytes": abytes, "flops": fl})
+    # end to end: inputs H2D from pinned memory, the op, output D2H, every step
+    hx = [t.cpu().pin_memory() for t in sets[0][0] + sets[0][1]]
+    ho = [t.cpu().pin_memory() for t in sets[0][2]]
+    dx = sets[0][0] + sets[0][1]
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    st = torch.cuda.current_stream()
+    e0.record(st)
+    for _ in range(args.e2e_steps):
+        for d, hsrc in zip(dx, hx):
+            d.copy_(hsrc, non_blocking=True)
+        call(0, None)
+        for hdst, d in zip(ho, sets[0][2]):
+            hdst.copy_(d, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    e1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dev)[0]
+    st_err, code = h.check_device_error()
+    if st_err != mxgemm.OK:
+        raise SystemExit("device error word set: %d" % code)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": job_tflops(fl, world, args.steps, ms), "unit": "TFLOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w["fmt"], "data": "synthetic",
+            "config": dict(base_config(args.workload), **{
+                "l2": "inputs rotate over %d copies (%.1f MB each)" % (nsets, abytes / 1e6),
+                "timing": "CUDA graph of K steps, CUDA events on the launch stream", "step_us": us,
+                "plan": h.describe(0 if op == "bf16" else fmt, M, N, K) if op != "grouped" else
+                mxgemm.mxgemm_describe_grouped_plan(torch.cuda.get_device_properties(dev).multi_processor_count,
+                                                    fmt, len(w["groups"]), M, N, K)}),
+            "clocks": clocks, "roofline": roof, "cpu_baseline": None,
+            "e2e": {"value": job_tflops(fl, world, args.e2e_steps, e2e_ms), "unit": "TFLOPS",
+                    "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hx),
+                    "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in ho),
+                    "api": "torch copies from pinned host memory around the entry point", "steps": args.e2e_steps},
+            "gpu_launches": args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    h.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
 
 
 def run_ours(args):
@@ -517,6 +733,9 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    w = extra_workload(args.workload)
+    if w is not None:
+        return run_extra(args, w)
     return run_ours(args)
 
 

@@ -53,10 +53,20 @@ extern "C" {
 
 typedef struct mxgemm_ctx *mxgemm_handle;
 
-/* Element formats. */
+/* Element formats.  MXGEMM_FMT_BF16 (dense BF16 operands, no scales) is
+ * taken only where an entry point says so. */
 enum {
     MXGEMM_FMT_MXFP8_E4M3 = 0,
-    MXGEMM_FMT_MXFP4_E2M1 = 1
+    MXGEMM_FMT_MXFP4_E2M1 = 1,
+    MXGEMM_FMT_BF16 = 2
+};
+
+/* Activations of the fused epilogue (mxgemm_run_fused / _quantized). */
+enum {
+    MXGEMM_ACT_NONE = 0,
+    MXGEMM_ACT_RELU = 1,       /* x < 0 ? 0 : x                                  */
+    MXGEMM_ACT_SILU = 2,       /* x * sigmoid(x) = x / (1 + e^-x)                */
+    MXGEMM_ACT_GELU = 3        /* x * Phi(x), Phi the standard normal CDF (erf form) */
 };
 
 /* Status codes.  Every entry point returns one of these. */
@@ -120,6 +130,81 @@ MXGEMM_API int mxgemm_run(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_
  * when it allocates.  Returns MXGEMM_ERR_OOM when the allocation fails. */
 MXGEMM_API int mxgemm_reserve(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K);
 
+/* GEMM epilogue fusion (the roadmap item "GEMM 尾部融合", GEMM epilogue
+ * fusion, at the end of section 怎么用起来 of the 5ulink.com page; an
+ * addition to the operation above): mxgemm_run's product followed, in the
+ * kernel's epilogue and before the one rounding to BF16, by
+ *
+ *     C[m][n] = bf16( act( acc[m][n] + bias[n] ) + residual[m][n] )
+ *
+ * with each step in FP32.  bias: BF16 [N] or NULL (no bias).  residual: BF16
+ * [M][N] or NULL; it may be the same buffer as C (each element is read
+ * before it is written, by the same thread).  act: MXGEMM_ACT_*.  Same
+ * operands, layouts, requirements and stream semantics as mxgemm_run; non-
+ * NULL bias / residual must be 16-byte aligned.  Runs on one-CTA tiles for
+ * every shape (the CTA-pair kernel has no fused epilogue). */
+MXGEMM_API int mxgemm_run_fused(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
+                     const void *A, const uint8_t *A_scales, const void *B, const uint8_t *B_scales,
+                     const void *bias, int act, const void *residual, void *C, void *stream);
+
+/* Quantised output (the next layer's MX operand written by the GEMM's
+ * epilogue instead of a BF16 C, saving the conversion copy the devotd.net
+ * page, section 4, counts against layouts the kernel does not take; an
+ * addition): the fused-epilogue result of mxgemm_run_fused, rounded to BF16,
+ * then MX-quantised by the rule of mxgemm_quantize along n -- one E8M0 scale
+ * per 32 consecutive values of a row of C, as the 5ulink.com support-matrix
+ * note fixes for MX operands (BlockWise1x32).  out_fmt: MXGEMM_FMT_MXFP8_E4M3
+ * or MXGEMM_FMT_MXFP4_E2M1.  C_codes: [M][row_bytes(N)] device; C_scales:
+ * [M][N/32] device.  N % 32 == 0.  bias / residual / act as mxgemm_run_fused
+ * (NULL, NULL, MXGEMM_ACT_NONE for the plain product). */
+MXGEMM_API int mxgemm_run_quantized(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
+                         const void *A, const uint8_t *A_scales, const void *B, const uint8_t *B_scales,
+                         const void *bias, int act, const void *residual, int out_fmt,
+                         void *C_codes, uint8_t *C_scales, void *stream);
+
+/* Dense BF16 NT GEMM on the same kernel and scheduler (the comparison suite
+ * "BF16 稠密 GEMM" of the 内核级成绩 table of the 5ulink.com page, which
+ * calls out 64x4096x4096; the support-matrix row "稠密 GEMM" takes FP16 and
+ * BF16 -- this entry point takes BF16, NT only):
+ *
+ *     C[m][n] = bf16( sum_k A[m][k] * B[n][k] ),  FP32 accumulation
+ *
+ * A: BF16 [M][K], B: BF16 [N][K], C: BF16 [M][N], all device, dense
+ * row-major.  K % 8 == 0 (16-byte rows), M, N >= 1, pointers 16-byte
+ * aligned.  No scales, no repack: one launch.  Stream semantics as
+ * mxgemm_run (programmatic dependent of the work before it). */
+MXGEMM_API int mxgemm_run_bf16(mxgemm_handle h, int64_t M, int64_t N, int64_t K,
+                    const void *A, const void *B, void *C, void *stream);
+
+/* Grouped GEMM (the 5ulink.com page: support-matrix row "Grouped GEMM" --
+ * A rows of uneven length per group, empty groups skipped; the Grouped GEMM
+ * row of the 内核级成绩 table; "MXFP8 Grouped GEMM" on the roadmap at the
+ * end of 怎么用起来).  G groups share N and K; group g owns rows
+ * [off[g], off[g+1]) of A and of C and its own B_g:
+ *
+ *     C[m][n] = sum_k A[m][k] * B[g][n][k]     for off[g] <= m < off[g+1]
+ *
+ * with MX scales as mxgemm_run (fmt MXGEMM_FMT_MXFP8_E4M3 / _MXFP4_E2M1) or
+ * dense BF16 operands (fmt MXGEMM_FMT_BF16; scale pointers ignored, may be
+ * NULL).  group_offsets: int64 [G+1] in DEVICE memory (a router's output
+ * need not come back to the host), off[0] = 0, non-decreasing, off[G] =
+ * M_total; offsets outside [0, M_total] are clamped, and a group whose end
+ * lies before its start is empty (results for such offsets are unspecified,
+ * but no access leaves the buffers).  A: [M_total][row_bytes(K)], A_scales:
+ * [M_total][K/32], B: [G][N][row_bytes(K)], B_scales: [G][N][K/32], C: BF16
+ * [M_total][N].  One launch; a persistent grid walks the groups' 128x128
+ * tiles in order.  1 <= G <= 65536, G * N <= 2^24, M_total >= 0 (0: no
+ * launch). */
+MXGEMM_API int mxgemm_run_grouped(mxgemm_handle h, int fmt, int64_t G, int64_t M_total, int64_t N, int64_t K,
+                       const int64_t *group_offsets, const void *A, const uint8_t *A_scales,
+                       const void *B, const uint8_t *B_scales, void *C, void *stream);
+
+/* The plan text of mxgemm_run_grouped for a device with num_sms SMs, without
+ * a handle or a GPU (as mxgemm_describe_plan_for); `tiles` there is the
+ * upper bound the launch is sized for. */
+MXGEMM_API int mxgemm_describe_grouped_plan(int num_sms, int fmt, int64_t G, int64_t M_total, int64_t N,
+                                 int64_t K, char *buf, size_t cap);
+
 /* The first half of mxgemm_run on its own: the scale repack into the
  * handle's workspace.  Sizes as for mxgemm_run. */
 MXGEMM_API int mxgemm_repack(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
@@ -176,6 +261,14 @@ MXGEMM_API int mxgemm_set_prefetch_b(mxgemm_handle h, int on);
 MXGEMM_API int mxgemm_quantize(int fmt, int64_t R, int64_t K, const float *X,
                     void *Q, uint8_t *scales, void *stream);
 
+/* The same quantisation of BF16 input (bit patterns [R][K], device): each
+ * value widens exactly to FP32, then the rule above applies.  This is the
+ * activation quantiser that turns a layer's BF16 output into the next
+ * layer's MX operand -- the conversion copy of the devotd.net page, section
+ * 4 -- as a stand-alone op (an addition). */
+MXGEMM_API int mxgemm_quantize_bf16(int fmt, int64_t R, int64_t K, const void *X,
+                         void *Q, uint8_t *scales, void *stream);
+
 /* Force a schedule for later mxgemm_run / mxgemm_gemm calls on this handle.
  * splits is used by MXGEMM_SCHED_SPLITK (>= 1); workers by
  * MXGEMM_SCHED_STREAMK (0 = number of SMs). */
@@ -199,7 +292,8 @@ MXGEMM_API int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t
 
 /* The same text for a device with `num_sms` SMs (2 to 4096) and the
  * automatic schedule, without a handle: it touches no GPU, so the planner
- * can be queried for capacity planning on any host.  Returns
+ * can be queried for capacity planning on any host.  fmt MXGEMM_FMT_BF16
+ * describes the plan of mxgemm_run_bf16 (K % 8 == 0).  Returns
  * MXGEMM_ERR_INVALID_ARG for a NULL or empty buffer, an SM count out of
  * range, or a shape mxgemm_run would reject. */
 MXGEMM_API int mxgemm_describe_plan_for(int num_sms, int fmt, int64_t M, int64_t N, int64_t K,

@@ -55,6 +55,7 @@ namespace {
 
 constexpr uint64_t kDefaultLimitNs = 2000000000ull;
 constexpr int64_t kMaxDim = int64_t(1) << 24;
+constexpr int64_t kMaxGroups = int64_t(1) << 16;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -146,17 +147,18 @@ int do_repack(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const u
 // behind the ring); otherwise it runs the separate repack first.
 bool fuse_scales(const mxg::GemmPlan &pl) { return pl.valid && !pl.pair && pl.stages >= 4; }
 
-// GEMM launch.  With raw scales (SA, SB non-NULL) the kernel converts the
-// row-major scales itself; otherwise it reads the last repack's workspace,
-// which must be for this shape.  pdl and early as mxg::launch_gemm and
-// GemmBuffers::early.
-int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const void *B, void *C,
-            cudaStream_t st, int pdl, int early, const uint8_t *SA = nullptr, const uint8_t *SB = nullptr)
+// GEMM launch of plan `pl`.  With raw scales (SA, SB non-NULL) the kernel
+// converts the row-major scales itself; otherwise it reads the last
+// repack's workspace, which must be for this shape (BF16 operands have no
+// scales).  pdl and early as mxg::launch_gemm and GemmBuffers::early.
+int launch_plan(mxgemm_handle h, const mxg::GemmPlan &pl, const void *A, const void *B, void *C, cudaStream_t st,
+                int pdl, int early, const uint8_t *SA, const uint8_t *SB, const mxg::Epilogue &epi,
+                const int64_t *goff = nullptr)
 {
-    if (!SA && (h->last_fmt != fmt || h->last_M != M || h->last_N != N || h->last_K != K))
-        return MXGEMM_ERR_INVALID_ARG;
-    const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks);
     if (!pl.valid)
+        return MXGEMM_ERR_INVALID_ARG;
+    if (pl.fmt != mxg::kFmtBF16 && !SA &&
+        (h->last_fmt != pl.fmt || h->last_M != pl.M || h->last_N != pl.N || h->last_K != pl.K))
         return MXGEMM_ERR_INVALID_ARG;
     int rc = grow(&h->partials, &h->partials_cap, static_cast<size_t>(pl.partial_bytes > 0 ? pl.partial_bytes : 16),
                   false, st);
@@ -177,11 +179,25 @@ int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const voi
     b.rawA = SA;
     b.rawB = SB;
     b.early = early;
+    b.epi = epi;
+    b.group_offsets = goff;
     const int inject = h->inject;
     h->inject = 0;
     if (mxg::launch_gemm(pl, b, h->limit_ns, inject, pdl, st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
     return MXGEMM_OK;
+}
+
+mxg::GemmPlan plan_for(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, bool allow_pair = true)
+{
+    return mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks, allow_pair);
+}
+
+// The GEMM alone on the last repack's workspace (mxgemm_gemm).
+int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const void *B, void *C,
+            cudaStream_t st, int pdl, int early)
+{
+    return launch_plan(h, plan_for(h, fmt, M, N, K), A, B, C, st, pdl, early, nullptr, nullptr, mxg::Epilogue());
 }
 
 // The hot path.  Plans on one CTA per tile convert the row-major scales
@@ -192,13 +208,17 @@ int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const voi
 // has completed, except B and its scales under the prefetch-B promise.
 // With profiling on, events bracket the launches and nothing overlaps (the
 // middle event keeps the GEMM from starting before the repack ends; with
-// the conversion fused it records no repack time).
+// the conversion fused it records no repack time).  A fused epilogue
+// (epi) keeps the plan on one-CTA tiles, whose epilogue implements it.
 int repack_and_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const uint8_t *SA,
-                    const void *B, const uint8_t *SB, void *C, cudaStream_t st)
+                    const void *B, const uint8_t *SB, void *C, cudaStream_t st,
+                    const mxg::Epilogue &epi = mxg::Epilogue(), bool allow_pair = true)
 {
     const bool prof = h->profiling != 0;
     h->ev_valid = 0;
-    const mxg::GemmPlan pl = mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks);
+    const mxg::GemmPlan pl = plan_for(h, fmt, M, N, K, allow_pair);
+    if (!pl.valid)
+        return MXGEMM_ERR_INVALID_ARG;
     const bool fused = fuse_scales(pl);
     if (prof && cudaEventRecord(h->ev[0], st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
@@ -210,8 +230,8 @@ int repack_and_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
     }
     if (prof && cudaEventRecord(h->ev[1], st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
-    rc = fused ? do_gemm(h, fmt, M, N, K, A, B, C, st, prof ? 0 : 1, h->prefetch_b ? 2 : 0, SA, SB)
-               : do_gemm(h, fmt, M, N, K, A, B, C, st, prof ? 0 : 1, 3);
+    rc = fused ? launch_plan(h, pl, A, B, C, st, prof ? 0 : 1, h->prefetch_b ? 2 : 0, SA, SB, epi)
+               : launch_plan(h, pl, A, B, C, st, prof ? 0 : 1, 3, nullptr, nullptr, epi);
     if (rc != MXGEMM_OK)
         return rc;
     if (prof) {
@@ -221,6 +241,23 @@ int repack_and_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
     }
     return MXGEMM_OK;
 }
+
+bool optional_aligned16(const void *p) { return p == nullptr || aligned16(p); }
+
+void format_plan(const mxg::GemmPlan &pl, char *buf, size_t cap)
+{
+    static const char *names[] = {"auto", "dp", "splitk", "streamk"};
+    const char *scales = pl.fmt == mxg::kFmtBF16 ? "none" : ((fuse_scales(pl) || pl.groups > 0) ? "fused" : "repack");
+    int n = snprintf(buf, cap,
+                     "fmt=%d swap=%d pair=%d BN=%d kc=%d stages=%d tiles=%lld kt=%lld workers=%lld grid=%d sched=%s "
+                     "partial_bytes=%lld scales=%s",
+                     pl.fmt, pl.swap, pl.pair, pl.bn, pl.kc, pl.stages, static_cast<long long>(pl.tiles),
+                     static_cast<long long>(pl.kt), static_cast<long long>(pl.workers), pl.grid, names[pl.sched & 3],
+                     static_cast<long long>(pl.partial_bytes), scales);
+    if (pl.groups > 0 && n > 0 && static_cast<size_t>(n) < cap)
+        snprintf(buf + n, cap - n, " groups=%lld", static_cast<long long>(pl.groups));
+}
+
 
 }  // namespace
 
@@ -383,6 +420,132 @@ int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
     return MXGEMM_OK;
 }
 
+int mxgemm_run_fused(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A,
+                     const uint8_t *A_scales, const void *B, const uint8_t *B_scales, const void *bias, int act,
+                     const void *residual, void *C, void *stream)
+{
+    if (!h || act < MXGEMM_ACT_NONE || act > MXGEMM_ACT_GELU)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = check_shape(fmt, M, N, K);
+    if (rc == MXGEMM_OK)
+        rc = check_ptrs({A, A_scales, B, B_scales, C});
+    if (rc == MXGEMM_OK && !(optional_aligned16(bias) && optional_aligned16(residual)))
+        rc = MXGEMM_ERR_ALIGNMENT;
+    if (rc == MXGEMM_OK)
+        rc = enter_device(h);
+    if (rc != MXGEMM_OK)
+        return rc;
+    mxg::Epilogue epi;
+    epi.bias = static_cast<const uint16_t *>(bias);
+    epi.residual = static_cast<const uint16_t *>(residual);
+    epi.act = act;
+    return repack_and_gemm(h, fmt, M, N, K, A, A_scales, B, B_scales, C, static_cast<cudaStream_t>(stream), epi,
+                           false);
+}
+
+int mxgemm_run_quantized(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A,
+                         const uint8_t *A_scales, const void *B, const uint8_t *B_scales, const void *bias, int act,
+                         const void *residual, int out_fmt, void *C_codes, uint8_t *C_scales, void *stream)
+{
+    if (!h || act < MXGEMM_ACT_NONE || act > MXGEMM_ACT_GELU)
+        return MXGEMM_ERR_INVALID_ARG;
+    if (out_fmt != MXGEMM_FMT_MXFP8_E4M3 && out_fmt != MXGEMM_FMT_MXFP4_E2M1)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = check_shape(fmt, M, N, K);
+    if (rc == MXGEMM_OK && N % 32 != 0)
+        rc = MXGEMM_ERR_INVALID_ARG;
+    if (rc == MXGEMM_OK)
+        rc = check_ptrs({A, A_scales, B, B_scales, C_codes, C_scales});
+    if (rc == MXGEMM_OK && !(optional_aligned16(bias) && optional_aligned16(residual)))
+        rc = MXGEMM_ERR_ALIGNMENT;
+    if (rc == MXGEMM_OK)
+        rc = enter_device(h);
+    if (rc != MXGEMM_OK)
+        return rc;
+    mxg::Epilogue epi;
+    epi.bias = static_cast<const uint16_t *>(bias);
+    epi.residual = static_cast<const uint16_t *>(residual);
+    epi.act = act;
+    epi.qfmt = out_fmt;
+    epi.Cq = static_cast<uint8_t *>(C_codes);
+    epi.Cs = C_scales;
+    // C itself is not written; the codes stand in for it in the launch
+    return repack_and_gemm(h, fmt, M, N, K, A, A_scales, B, B_scales, C_codes, static_cast<cudaStream_t>(stream),
+                           epi, false);
+}
+
+int mxgemm_quantize_bf16(int fmt, int64_t R, int64_t K, const void *X, void *Q, uint8_t *scales, void *stream)
+{
+    if (fmt != MXGEMM_FMT_MXFP8_E4M3 && fmt != MXGEMM_FMT_MXFP4_E2M1)
+        return MXGEMM_ERR_INVALID_ARG;
+    if (R < 1 || K < 32 || K % 32 != 0 || R > kMaxDim || K > kMaxDim)
+        return MXGEMM_ERR_INVALID_ARG;
+    if (!X || !Q || !scales)
+        return MXGEMM_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(Q) || !aligned16(scales))
+        return MXGEMM_ERR_ALIGNMENT;
+    if (mxg::launch_quantize(fmt, R, K, nullptr, static_cast<uint8_t *>(Q), scales, static_cast<cudaStream_t>(stream),
+                             static_cast<const uint16_t *>(X)) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    return MXGEMM_OK;
+}
+
+int mxgemm_run_bf16(mxgemm_handle h, int64_t M, int64_t N, int64_t K, const void *A, const void *B, void *C,
+                    void *stream)
+{
+    if (!h)
+        return MXGEMM_ERR_INVALID_ARG;
+    if (M < 1 || N < 1 || K < 8 || K % 8 != 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = check_ptrs({A, B, C});
+    if (rc == MXGEMM_OK)
+        rc = enter_device(h);
+    if (rc != MXGEMM_OK)
+        return rc;
+    h->ev_valid = 0;
+    const mxg::GemmPlan pl = plan_for(h, mxg::kFmtBF16, M, N, K, false);
+    return launch_plan(h, pl, A, B, C, static_cast<cudaStream_t>(stream), 1, h->prefetch_b ? 2 : 0, nullptr, nullptr,
+                       mxg::Epilogue());
+}
+
+int mxgemm_run_grouped(mxgemm_handle h, int fmt, int64_t G, int64_t M_total, int64_t N, int64_t K,
+                       const int64_t *group_offsets, const void *A, const uint8_t *A_scales, const void *B,
+                       const uint8_t *B_scales, void *C, void *stream)
+{
+    if (!h || G < 1 || G > kMaxGroups || M_total < 0)
+        return MXGEMM_ERR_INVALID_ARG;
+    const bool bf16 = fmt == MXGEMM_FMT_BF16;
+    int rc = check_shape(bf16 ? MXGEMM_FMT_MXFP8_E4M3 : fmt, M_total > 0 ? M_total : 1, N, K);
+    if (rc == MXGEMM_OK && G * N > kMaxDim)
+        rc = MXGEMM_ERR_INVALID_ARG;
+    if (rc == MXGEMM_OK)
+        rc = bf16 ? check_ptrs({group_offsets, A, B, C}) : check_ptrs({group_offsets, A, A_scales, B, B_scales, C});
+    if (rc == MXGEMM_OK)
+        rc = enter_device(h);
+    if (rc != MXGEMM_OK)
+        return rc;
+    h->ev_valid = 0;
+    if (M_total == 0)
+        return MXGEMM_OK;                 // every group is empty: nothing to compute
+    const mxg::GemmPlan pl = mxg::make_grouped_plan(fmt, G, M_total, N, K, h->num_sms);
+    if (!pl.valid)
+        return MXGEMM_ERR_INVALID_ARG;
+    return launch_plan(h, pl, A, B, C, static_cast<cudaStream_t>(stream), 1, 0, bf16 ? nullptr : A_scales,
+                       bf16 ? nullptr : B_scales, mxg::Epilogue(), group_offsets);
+}
+
+int mxgemm_describe_grouped_plan(int num_sms, int fmt, int64_t G, int64_t M_total, int64_t N, int64_t K, char *buf,
+                                 size_t cap)
+{
+    if (!buf || cap == 0 || num_sms < 2 || num_sms > 4096 || G < 1 || G > kMaxGroups || M_total < 1)
+        return MXGEMM_ERR_INVALID_ARG;
+    int rc = check_shape(fmt == MXGEMM_FMT_BF16 ? MXGEMM_FMT_MXFP8_E4M3 : fmt, M_total, N, K);
+    if (rc != MXGEMM_OK || G * N > kMaxDim)
+        return MXGEMM_ERR_INVALID_ARG;
+    format_plan(mxg::make_grouped_plan(fmt, G, M_total, N, K, num_sms), buf, cap);
+    return MXGEMM_OK;
+}
+
 int mxgemm_reserve(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K)
 {
     if (!h)
@@ -478,18 +641,6 @@ int mxgemm_set_kchunks(mxgemm_handle h, int kc)
     return MXGEMM_OK;
 }
 
-static void format_plan(const mxg::GemmPlan &pl, char *buf, size_t cap)
-{
-    static const char *names[] = {"auto", "dp", "splitk", "streamk"};
-    snprintf(buf, cap,
-             "fmt=%d swap=%d pair=%d BN=%d kc=%d stages=%d tiles=%lld kt=%lld workers=%lld grid=%d sched=%s "
-             "partial_bytes=%lld scales=%s",
-             pl.fmt, pl.swap, pl.pair, pl.bn, pl.kc, pl.stages, static_cast<long long>(pl.tiles),
-             static_cast<long long>(pl.kt),
-             static_cast<long long>(pl.workers), pl.grid, names[pl.sched & 3],
-             static_cast<long long>(pl.partial_bytes), fuse_scales(pl) ? "fused" : "repack");
-}
-
 int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, char *buf, size_t cap)
 {
     if (!h || !buf || cap == 0)
@@ -505,6 +656,12 @@ int mxgemm_describe_plan_for(int num_sms, int fmt, int64_t M, int64_t N, int64_t
 {
     if (!buf || cap == 0 || num_sms < 2 || num_sms > 4096)
         return MXGEMM_ERR_INVALID_ARG;
+    if (fmt == MXGEMM_FMT_BF16) {           // the plan of mxgemm_run_bf16
+        if (M < 1 || N < 1 || K < 8 || K % 8 != 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
+            return MXGEMM_ERR_INVALID_ARG;
+        format_plan(mxg::make_plan(fmt, M, N, K, num_sms, MXGEMM_SCHED_AUTO, 1, 0, 0, false), buf, cap);
+        return MXGEMM_OK;
+    }
     int rc = check_shape(fmt, M, N, K);
     if (rc != MXGEMM_OK)
         return rc;

@@ -1,1646 +1,43 @@
-// gemm.cu -- the sm_100a MX block-scaled GEMM: C = A * B^T, BF16 out.
+// gemm.cu -- the GEMM's host planner and launch dispatch.
 //
-// Operation: the "MXFP scaled GEMM" of the 5ulink.com page "PyTorch 接上
-// FlyDSL" (support-matrix table; note under it: one E8M0 scale per 32
-// values, FP32 accumulation, BF16 output).  The page's own kernel design
-// (HTI pipeline with staged LDS, MFMA atoms, "operand and scale-factor
-// lifetime pairing", section "三条路") targets another GPU; here the same
-// ideas take Blackwell form: a TMA-fed shared-memory ring whose every stage
-// carries an operand tile pair together with the scale tiles of exactly
-// those K elements, released by one mbarrier.
-//
-// Two kernels.  mx_gemm_kernel: one persistent CTA per SM, 128-row tiles.
-//   warps 0, 6  TMA producers of the row / column operand tile of each stage
-//               (128B-swizzled, KC 128-byte K chunks per 3-D box);
-//   warps 7, 8  their scale atoms: a TMA box of the repacked layout, or, with
-//               the scale conversion fused (mxgemm_run), 4-byte cp.async
-//               gathers from the row-major scales;
-//   warps 1, 9.. MMA warps, up to four: each owns a run of the stage's scale
-//               atoms, copies them into TMEM (tcgen05.cp) and issues the
-//               block-scaled MMAs (kind::mxf8f6f4 K=32 / kind::mxf4 K=64) that
-//               read them into its own FP32 accumulator; its tcgen05.commit
-//               counts toward releasing the stage;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulators, summed in FP32,
-//               BF16 (RNE) through shared memory and TMA stores; for split
-//               tiles an FP32 partial plus a last-arriver fixup.
-// mx_gemm_pair_kernel: a cluster of two CTAs per 256x256 tile
-// (tcgen05.mma.cta_group::2); the leader's warp 7 copies both CTAs' scale
-// atoms, its warp 1 issues the MMAs, the peer's warp 1 relays its landed
-// stages.  Every instruction-issuing role has its own warp because a TMA or
-// tcgen05 instruction holds the issuing thread for tens to hundreds of ns.
-//
-// Work decomposition (stream-K family): the I = tiles * kt K-iterations of
-// all output tiles, tile-major, are cut into W contiguous ranges, one per
-// virtual worker; worker w owns [floor(w*I/W), floor((w+1)*I/W)).  W = tiles
-// gives plain data-parallel tiles, W = tiles*s split-K, W = #SMs stream-K.
-// A tile covered by several workers is reduced by whichever of them arrives
-// last (an atomic counter per tile), summing the partials in worker order so
-// the result does not depend on arrival order.  No CTA ever waits for
-// another CTA.
-//
-// Decode shapes (M <= 64) swap the operands (C^T = B * A^T) so that the N
-// rows of B fill the MMA's 128-row side and the small M becomes the MMA's N.
-//
-// Every wait is bounded in time; a wait that runs out records a site code in
-// a device error word, the CTA drains its in-flight copies and MMAs, frees
-// its tensor memory and exits normally.
-//
-// Launch chaining (programmatic dependent launch): mx_gemm_kernel lets the
-// next launch on its stream start as soon as its own CTAs are set up.  A
-// launch that starts early sets up its CTA (barriers, tensor memory, tensor
-// maps) while the previous kernel finishes, and every role waits for that
-// kernel (griddepcontrol.wait) before it touches global memory, except the
-// operand producers named in KParams::early, which may stream their operand
-// into the ring first.  They wait before their first blocking ring wait, so
-// no bounded wait ever spans the previous kernel's run time.
-#include <cuda.h>
-#include <cuda_bf16.h>
+// The planner picks, from the shape and the SM count alone, the operand
+// swap for decode shapes (M <= 64: C^T = B * A^T), the output tile width,
+// the 128-byte K chunks per pipeline stage, CTA pairs for large M, and the
+// schedule (whole tiles, split-K or stream-K).  The kernels and their launch
+// templates are in gemm_kernel.cuh, instantiated per operand type in
+// gemm_mxfp8.cu, gemm_mxfp4.cu, gemm_bf16.cu and gemm_pair.cu.
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <cstdio>
 #include <cstdlib>
 
 #include "mx_internal.h"
-#include "sm100_ptx.cuh"
 
 namespace mxg {
 
-// ------------------------------------------------------------ configuration
-
-template <int FMT, int BN, int KC>
-struct Cfg {
-    static constexpr int kBM = 128;
-    static constexpr int kAtomsPerChunk = FMT == kFmtMXFP8 ? 1 : 2;   // 512B scale atoms per 128-byte K chunk
-    static constexpr int kAtoms = kAtomsPerChunk * KC;        // scale atoms per 128 rows per stage
-    static constexpr int kRBQ = (BN + 127) / 128;             // 128-row blocks of the column operand
-    static constexpr int kAChunk = kBM * 128;                 // one 128-byte K chunk of the row-operand tile
-    static constexpr int kBChunk = BN * 128;
-    static constexpr int kABytes = kAChunk * KC;
-    static constexpr int kBBytes = kBChunk * KC;
-    static constexpr int kSFABytes = kAtoms * 512;
-    static constexpr int kSFBBytes = kRBQ * kAtoms * 512;
-    static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
-    static constexpr int kCW = BN < 32 ? BN : 32;             // accumulator columns per epilogue chunk
-    // Output staging for TMA stores: two BF16 chunks of the 128-row tile.
-    // Tiles of at most 32 columns (decode, M <= 32) have none of their own
-    // and give the space to a fifth ring stage: a CTA's final tile stages its
-    // output in the then idle first ring stage, an earlier one stores from
-    // registers.
-    static constexpr bool kStaged = BN > 32;
-    static constexpr int kChunkOutBytes = 128 * kCW * 2;      // one BF16 output chunk
-    static constexpr int kOutBytes = kStaged ? kChunkOutBytes : 0;
-    static constexpr int kSmemBudget = 227 * 1024 - 2048 - 2 * kOutBytes;
-    static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
-    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-    static constexpr int kSFACols = kAtoms * 4;
-    static constexpr int kSFBCols = kRBQ * kAtoms * 4;
-    static constexpr int kSFCols = kStages * (kSFACols + kSFBCols);
-    // A tcgen05 instruction holds its issuing thread ~40 ns, so a stage's
-    // scale copies and MMAs are split over kNMma MMA warps, each with its own
-    // accumulator (summed by the epilogue).  Warp m owns a contiguous run of
-    // the stage's scale atoms: it copies them and issues exactly the MMAs
-    // that read them, so no warp's MMA depends on another warp's copy.
-    // Narrow (decode) tiles take up to four warps where TMEM holds one
-    // accumulator set; wider ones keep two accumulator sets.
-    static constexpr int kMmaPerAtom = FMT == kFmtMXFP8 ? 4 : 2;   // MMAs reading one 512B atom
-    static constexpr int pick_nmma()
-    {
-        for (int nm = 4; nm > 1; nm /= 2)
-            if (kAtoms % nm == 0 && (BN <= 64 ? nm * BN : 2 * nm * BN) + kSFCols <= 512)
-                return nm;
-        return 1;
-    }
-    static constexpr int kNMma = pick_nmma();
-    static constexpr int kAtomsPerMma = kAtoms / kNMma;
-    static constexpr int kNumAcc = (2 * kNMma * BN + kSFCols <= 512) ? 2 : 1;
-    static constexpr int kAccCols = kNumAcc * kNMma * BN;
-    static constexpr int kTmemCols = 512;
-    // warps: 0 row-operand TMA, 1 MMA, 2..5 epilogue, 6 column-operand TMA,
-    // 7 row-scale TMA, 8 column-scale TMA, 9.. further MMA warps
-    static constexpr int kWarps = 9 + kNMma - 1;
-    static constexpr int kThreads = 32 * kWarps;
-    static constexpr int kMmaPerChunk = 4;                    // 32 bytes of K per MMA
-    static constexpr uint32_t kTxBytes = kStageBytes;
-    // shared memory layout (offsets from a 1024-aligned base)
-    static constexpr int kOffA = 0;
-    static constexpr int kOffB = kOffA + kStages * kABytes;
-    static constexpr int kOffSFA = kOffB + kStages * kBBytes;
-    static constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
-    static constexpr int kOffOut = (kOffSFB + kStages * kSFBBytes + 1023) / 1024 * 1024;
-    static constexpr int kOffBar = kOffOut + 2 * kOutBytes;
-    static constexpr int kNumBars = 2 * kStages + 2 * kNumAcc + 1;
-    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kSmemBytes = kOffMisc + 64 + 1024;   // + alignment slack
-
-    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be a multiple of 16 in [16, 256]");
-    static_assert(KC == 1 || KC == 2 || KC == 4, "1, 2 or 4 K chunks per stage");
-    static_assert(kStages >= 2, "at least two pipeline stages");
-    static_assert(kAccCols + kSFCols <= kTmemCols, "TMEM budget");
-    static_assert(kBChunk % 1024 == 0, "tiles must keep 1024-byte alignment");
-    static_assert(kStaged || 2 * kChunkOutBytes <= kABytes, "ring stage 0 holds two output chunks");
-    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-};
-
-// Instruction descriptor of the block-scaled MMA (PTX ISA, instruction
-// descriptor for .kind::mxf8f6f4 / .kind::mxf4): A/B type at bits [7,10) and
-// [10,13) (E4M3 = 0 under mxf8f6f4, E2M1 = 1 under mxf4), both K-major (bits
-// 15, 16 = 0), N >> 3 at [17,23), scale type UE8M0 at bit 23, M >> 4 at
-// [24,29); scale-factor ids of B at [4,6) and of A at [29,31) are added per
-// instruction.
-template <int FMT, int BN>
-__host__ __device__ constexpr uint32_t idesc_base()
-{
-    constexpr uint32_t t = FMT == kFmtMXFP8 ? 0u : 1u;
-    return (t << 7) | (t << 10) | (static_cast<uint32_t>(BN >> 3) << 17) | (1u << 23) |
-           (static_cast<uint32_t>(128 >> 4) << 24);
-}
-
-struct KParams {
-    __nv_bfloat16 *C;
-    float *partials;
-    uint32_t *counters;
-    int *error;
-    int64_t P, Q;          // valid rows of the two MMA operands
-    int64_t ldc;           // = N
-    uint32_t tilesP, kt, iters, workers;   // host guarantees iters * workers < 2^32
-    int dp;                // workers == tiles: worker w is exactly tile w
-    uint64_t limit_ns;
-    int swap;
-    int inject;
-    int tma_store;         // 1: epilogue stores C through shared memory with TMA
-    // Fused scale conversion (1-CTA kernel): the scale producers gather each
-    // stage's atoms from the row-major scales [rows][K/32] themselves instead
-    // of loading the repacked layout.
-    int fused_sf;
-    const uint8_t *rawP, *rawQ;   // row-major scales of the row / column operand
-    int64_t ldS;                  // K / 32: scale bytes per row
-    // Operands that may be read before the prerequisite grid (the previous
-    // kernel on the stream, when launched as its programmatic dependent) has
-    // completed: bit 0 the row operand (P) with its row-major scales, bit 1
-    // the column operand (Q) with its row-major scales.  Repacked scales and
-    // C are always accessed after it.
-    int early;
-};
-
-// Error site codes written to the device error word.
-enum : int {
-    kErrProducerEmpty = 1,
-    kErrMmaFull = 2,
-    kErrMmaAccEmpty = 3,
-    kErrEpiAccFull = 4,
-    kErrDrain = 5,
-    kErrLaunch = 6,        // launched with a block size the kernel was not built for
-};
-
-__device__ __forceinline__ void record_error(int *err, int code, volatile int *abort_flag)
-{
-    atomicCAS(err, 0, code);
-    *abort_flag = 1;
-}
-
-// Work decomposition shared by the three roles.  All index arithmetic is
-// 32-bit (64-bit integer division is a long software sequence on the GPU and
-// sat on the critical path of every hand-off); whole-tile schedules take a
-// division-free path.
-struct Sched {
-    uint32_t I, W, KT, tilesP;
-    bool dp;
-    // first K-iteration of worker g: floor(g * I / W)
-    __device__ __forceinline__ uint32_t begin(uint32_t g) const { return dp ? g * KT : (g * I) / W; }
-    // worker owning K-iteration i: the largest g with begin(g) <= i
-    __device__ __forceinline__ uint32_t owner(uint32_t i) const { return dp ? i / KT : ((i + 1) * W - 1) / I; }
-};
-
-// Walks the K-iterations of the workers a CTA owns (blockIdx.x, +gridDim.x,
-// ...) in order, tracking the tile and its K step incrementally.
-struct IterCursor {
-    Sched sc;
-    uint32_t w, step;
-    uint32_t it, end, tile, k;
-    __device__ __forceinline__ IterCursor(const Sched &sc_, uint32_t first, uint32_t step_)
-        : sc(sc_), w(first), step(step_), it(0), end(0), tile(0), k(0)
-    {
-        enter();
-    }
-    __device__ __forceinline__ void enter()
-    {
-        while (w < sc.W) {
-            it = sc.begin(w);
-            end = sc.begin(w + 1);
-            if (it < end)
-                break;
-            w += step;
-        }
-        if (w < sc.W) {
-            tile = sc.dp ? w : it / sc.KT;
-            k = it - tile * sc.KT;
-        }
-    }
-    __device__ __forceinline__ bool valid() const { return w < sc.W; }
-    __device__ __forceinline__ void advance()
-    {
-        ++it;
-        if (it >= end) {
-            w += step;
-            enter();
-            return;
-        }
-        if (++k == sc.KT) {
-            k = 0;
-            ++tile;
-        }
-    }
-    __device__ __forceinline__ uint32_t total() const
-    {
-        uint32_t n = 0;
-        for (uint32_t g = w; g < sc.W; g += step)
-            n += sc.begin(g + 1) - sc.begin(g);
-        return n;
-    }
-};
-
-// One maximal run of a worker's K-iterations inside one tile.
-struct Segment {
-    uint32_t tile, kb, ke, tp, tq;
-};
-
-__device__ __forceinline__ Segment segment_at(const Sched &sc, uint32_t it, uint32_t end)
-{
-    Segment g;
-    g.tile = it / sc.KT;
-    g.kb = it - g.tile * sc.KT;
-    g.ke = (g.kb + (end - it) < sc.KT) ? g.kb + (end - it) : sc.KT;
-    g.tq = g.tile / sc.tilesP;
-    g.tp = g.tile - g.tq * sc.tilesP;
-    return g;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
-{
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-
-// Store CW FP32 values as BF16 into C.  Non-swapped: thread's row p = C row,
-// values are C[p][q0 .. q0+CW).  Swapped: thread's row p = C column, values
-// are C[q0 .. q0+CW)[p].
-struct OutView {
-    __nv_bfloat16 *C;
-    int64_t ldc, P, Q;
-    int swap;
-};
-
-template <int CW>
-__device__ __forceinline__ void store_bf16(const OutView o, int64_t p, int64_t q0, const float (&v)[CW])
-{
-    if (p >= o.P)
-        return;
-    if (!o.swap) {
-        __nv_bfloat16 *dst = o.C + p * o.ldc + q0;
-        const int64_t nvalid = o.Q - q0;
-        if (nvalid >= CW && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
-#pragma unroll
-            for (int j = 0; j < CW / 8; ++j) {
-                uint4 w;
-                w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-                w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-                w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-                w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-                reinterpret_cast<uint4 *>(dst)[j] = w;
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < CW; ++j)
-                if (j < nvalid)
-                    dst[j] = __float2bfloat16_rn(v[j]);
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < CW; ++j) {
-            const int64_t q = q0 + j;
-            if (q < o.Q)
-                o.C[q * o.ldc + p] = __float2bfloat16_rn(v[j]);
-        }
-    }
-}
-
-template <int FMT, int BN, int KC>
-__global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
-    mx_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
-                   const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
-                   const __grid_constant__ CUtensorMap tmC, const KParams kp_in)
-{
-    using C_ = Cfg<FMT, BN, KC>;
-    constexpr int S = C_::kStages;
-    constexpr int CW = C_::kCW;
-    constexpr int NM = C_::kNMma;
-
-    // Work on a register copy of the parameters: the inline-asm memory
-    // clobbers of the pipeline would otherwise force reloads from parameter
-    // space after each TMA / MMA / barrier instruction.
-    const KParams kp = kp_in;
-    const OutView out{kp.C, kp.ldc, kp.P, kp.Q, kp.swap};
-
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~static_cast<uintptr_t>(1023));
-    const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar0 = sbase + C_::kOffBar;
-    auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
-    auto accf_bar = [&](int a) { return bar0 + 8u * (2 * S + a); };
-    auto acce_bar = [&](int a) { return bar0 + 8u * (2 * S + C_::kNumAcc + a); };
-    const uint32_t drain_bar = bar0 + 8u * (2 * S + 2 * C_::kNumAcc);
-    volatile uint32_t *s_tmem = reinterpret_cast<volatile uint32_t *>(smem + C_::kOffMisc);
-    volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C_::kOffMisc + 4);
-    volatile int *s_last = reinterpret_cast<volatile int *>(smem + C_::kOffMisc + 8);
-
-    if (blockDim.x != C_::kThreads) {
-        if (threadIdx.x == 0)
-            atomicCAS(kp.error, 0, kErrLaunch);
-        return;
-    }
-    // Every wait in this kernel parks the thread in the suspending try_wait
-    // at once: the producer and MMA warps share SM sub-partitions, and a
-    // warp spinning on test_wait would take issue slots from an MMA warp.
-    const int warp = threadIdx.x / 32;
-    const int lane = threadIdx.x % 32;
-    const bool producer = warp == 0 || (warp >= 6 && warp <= 8);
-    const int mma_idx = warp == 1 ? 0 : (warp >= 9 ? warp - 8 : -1);
-
-    // Each producer fetches its own tensor map while the CTA sets up.
-    if (lane == 0) {
-        if (warp == 0)
-            tma_prefetch_desc(&tmP);
-        else if (warp == 6)
-            tma_prefetch_desc(&tmQ);
-        else if (warp == 7)
-            tma_prefetch_desc(&tmSP);
-        else if (warp == 8)
-            tma_prefetch_desc(&tmSQ);
-        else if (warp == 2)
-            tma_prefetch_desc(&tmC);
-    }
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            // one arming per producer warp; with fused scales, one async
-            // arrival per lane of the two scale warps
-            mbar_init(full_bar(s), kp.fused_sf ? 2 + 64 : 4);
-            mbar_init(empty_bar(s), NM);        // one commit per MMA warp
-        }
-        for (int a = 0; a < C_::kNumAcc; ++a) {
-            mbar_init(accf_bar(a), NM);
-            mbar_init(acce_bar(a), 4);
-        }
-        mbar_init(drain_bar, NM);
-        *s_abort = 0;
-        *s_last = 0;
-        fence_mbar_init();
-        fence_proxy_async_smem();
-    }
-    if (warp == 1) {
-        tmem_alloc(sbase + C_::kOffMisc, C_::kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *s_tmem;
-
-    const Sched sc{kp.iters, kp.workers, kp.kt, kp.tilesP, kp.dp != 0};
-    const uint32_t W = sc.W;
-    // The CTA is set up: a programmatic dependent launch may start.
-    grid_launch_dependents();
-
-    if (producer && kp.fused_sf && warp >= 7) {
-        // ------------------------------------- scale atoms gathered directly
-        // Warp 7 (row operand) and warp 8 (column operand) build each stage's
-        // scale atoms in shared memory from the row-major scales: atom a of a
-        // 128-row block holds, for row r and K block 4a + j, the byte at
-        // (r % 32) * 16 + (r / 32) * 4 + j.  Lane l moves rows l, l+32, l+64,
-        // l+96 with 4-byte cp.async copies (rows past the operand and K
-        // blocks past K are zero-filled) and arrives on the stage's full
-        // barrier once its copies have landed.
-        const bool sideP = warp == 7;
-        const uint8_t *raw = sideP ? kp.rawP : kp.rawQ;
-        const int64_t nrows = sideP ? kp.P : kp.Q;
-        const uint32_t bytes = sideP ? C_::kSFABytes : C_::kSFBBytes;
-        const uint32_t off = sideP ? C_::kOffSFA : C_::kOffSFB;
-        const int nrb = sideP ? 1 : C_::kRBQ;
-        const int64_t kblocks = kp.ldS;
-        // scales of an early operand: gathered ahead until the ring is full
-        bool dep_pending = (kp.early & (sideP ? 1 : 2)) != 0;
-        if (!dep_pending)
-            grid_dependency_wait();
-        uint32_t issued = 0;
-        int s = 0;
-        uint32_t ph = 0;
-        for (IterCursor cur(sc, blockIdx.x, gridDim.x); cur.valid(); cur.advance()) {
-            if (dep_pending && issued == static_cast<uint32_t>(S)) {
-                grid_dependency_wait();
-                dep_pending = false;
-            }
-            ++issued;
-            int good = 1;
-            if (lane == 0)
-                good = mbar_wait_parked(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns);
-            good = __shfl_sync(0xffffffffu, good, 0);
-            if (!good) {
-                if (lane == 0)
-                    record_error(kp.error, kErrProducerEmpty, s_abort);
-                break;
-            }
-            const uint32_t tq = cur.tile / sc.tilesP, tp = cur.tile - tq * sc.tilesP;
-            const int64_t rb0 = sideP ? static_cast<int64_t>(tp) : static_cast<int64_t>((tq * BN) / 128);
-            const int64_t kb0 = static_cast<int64_t>(cur.k) * C_::kAtoms * 4;
-            const uint32_t dst0 = sbase + off + s * bytes + lane * 16;
-            for (int rb = 0; rb < nrb; ++rb) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int64_t row = (rb0 + rb) * 128 + i * 32 + lane;
-                    const bool rv = row < nrows;
-#pragma unroll
-                    for (int a = 0; a < C_::kAtoms; ++a) {
-                        const int64_t kb = kb0 + 4 * a;
-                        const bool v = rv && kb < kblocks;
-                        cp_async_4(dst0 + (rb * C_::kAtoms + a) * 512 + i * 4, v ? raw + row * kblocks + kb : raw,
-                                   v ? 4u : 0u);
-                    }
-                }
-            }
-            cp_async_arrive_noinc(full_bar(s));
-            if (++s == S) {
-                s = 0;
-                ph ^= 1u;
-            }
-        }
-        cp_async_wait_all();
-        __syncwarp();
-    } else if (producer) {
-        // ----------------------------------------------------- TMA producers
-        // Four producer warps, one TMA operation each per stage: warp 0 the
-        // MMA row-operand tile, warp 6 the column-operand tile, warps 7 and 8
-        // their scale atoms.  Issuing a TMA operation occupies the issuing
-        // thread for ~0.1-0.15 us, so one thread per operation keeps the
-        // ring's refill off the critical path.  An operand named in
-        // KParams::early fills the ring before the producer waits for the
-        // prerequisite grid; everything else waits first.
-        // L2 policy: in the swapped (decode) form the weights stream through
-        // once and the small activation is re-read by every tile; otherwise
-        // both operands are re-read across tiles.
-        if (lane == 0) {
-            const bool sideP = warp == 0 || warp == 7;
-            const bool scales = warp >= 7;
-            const uint64_t pol = sideP ? (kp.swap ? policy_evict_first() : policy_evict_normal())
-                                       : (kp.swap ? policy_evict_last() : policy_evict_normal());
-            const uint32_t bytes = scales ? (sideP ? C_::kSFABytes : C_::kSFBBytes)
-                                          : (sideP ? C_::kABytes : C_::kBBytes);
-            const uint32_t off = scales ? (sideP ? C_::kOffSFA : C_::kOffSFB) : (sideP ? C_::kOffA : C_::kOffB);
-            bool dep_pending = !scales && (kp.early & (sideP ? 1 : 2)) != 0;
-            if (!dep_pending)
-                grid_dependency_wait();
-            uint32_t armed = 0;         // stages armed so far (round-robin over the ring)
-            int skipped_stage = -1;
-            bool inject = warp == 0 && kp.inject == 1;
-            int s = 0;
-            uint32_t ph = 0;
-            for (IterCursor cur(sc, blockIdx.x, gridDim.x); cur.valid(); cur.advance()) {
-                if (dep_pending && armed == static_cast<uint32_t>(S)) {
-                    grid_dependency_wait();
-                    dep_pending = false;
-                }
-                if (!mbar_wait_parked(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns)) {
-                    record_error(kp.error, kErrProducerEmpty, s_abort);
-                    break;
-                }
-                const uint32_t tq = cur.tile / sc.tilesP, tp = cur.tile - tq * sc.tilesP;
-                const uint32_t fb = full_bar(s);
-                const uint32_t dst = sbase + off + s * bytes;
-                if (inject) {
-                    inject = false;             // test hook: leave this stage unarmed
-                    skipped_stage = s;
-                } else {
-                    mbar_arrive_expect_tx(fb, bytes);
-                    if (warp == 0) {
-                        const int32_t row = static_cast<int32_t>(tp) * 128;
-                        if constexpr (KC == 1)      // 2-D maps: x = byte offset along K
-                            tma_load_2d(dst, &tmP, static_cast<int32_t>(cur.k * 128), row, fb, pol);
-                        else                        // 3-D maps: {byte in chunk, row, 128-byte K chunk}
-                            tma_load_3d(dst, &tmP, 0, row, static_cast<int32_t>(cur.k * KC), fb, pol);
-                    } else if (warp == 6) {
-                        const int32_t row = static_cast<int32_t>(tq) * BN;
-                        if constexpr (KC == 1)
-                            tma_load_2d(dst, &tmQ, static_cast<int32_t>(cur.k * 128), row, fb, pol);
-                        else
-                            tma_load_3d(dst, &tmQ, 0, row, static_cast<int32_t>(cur.k * KC), fb, pol);
-                    } else if (warp == 7) {
-                        tma_load_3d(dst, &tmSP, 0, static_cast<int32_t>(cur.k * C_::kAtoms),
-                                    static_cast<int32_t>(tp), fb, pol);
-                    } else {
-                        tma_load_3d(dst, &tmSQ, 0, static_cast<int32_t>(cur.k * C_::kAtoms),
-                                    static_cast<int32_t>((tq * BN) / 128), fb, pol);
-                    }
-                }
-                ++armed;
-                if (++s == S) {
-                    s = 0;
-                    ph ^= 1u;
-                }
-            }
-            // Let every armed copy land before the CTA can exit: wait for the
-            // latest armed phase of each stage (already complete on the normal
-            // path, where the MMA warps consumed every stage).
-            for (int st = 0; st < S; ++st) {
-                const uint32_t n = armed / S + (static_cast<uint32_t>(st) < armed % S ? 1u : 0u);
-                if (n == 0 || (st == skipped_stage && n == 1))
-                    continue;
-                const uint32_t parity = static_cast<uint32_t>((n - 1) & 1);
-                int dummy_abort = 0;
-                if (!mbar_wait_parked(full_bar(st), parity, &dummy_abort, kp.limit_ns))
-                    atomicCAS(kp.error, 0, kErrDrain);
-            }
-        }
-        __syncwarp();
-    } else if (mma_idx >= 0) {
-        // ------------------------------------------------------ MMA issuers
-        // MMA warp m takes scale atoms [m * kAtomsPerMma, (m + 1) * kAtomsPerMma)
-        // of every stage: their scale copies into TMEM and their block-scaled
-        // MMAs, into its own accumulator.  Each commit releases the stage once
-        // that warp's MMAs have read it; the stage is free after all NM commits.
-        constexpr uint32_t kIdesc = idesc_base<FMT, BN>();
-        const uint32_t t_sfa0 = tmem + C_::kAccCols;
-        const uint32_t t_sfb0 = t_sfa0 + S * C_::kSFACols;
-        const int a_begin = mma_idx * C_::kAtomsPerMma;
-        grid_dependency_wait();
-        int s = 0;
-        uint32_t ph = 0;
-        int acc = 0;
-        uint32_t acc_ph = 0;
-        bool ok = true;
-        for (uint32_t w = blockIdx.x; w < W && ok; w += gridDim.x) {
-            uint32_t it = sc.begin(w);
-            const uint32_t end = sc.begin(w + 1);
-            while (it < end && ok) {
-                const Segment sg = segment_at(sc, it, end);
-                const uint32_t kb = sg.kb, ke = sg.ke;
-                int good = 1;
-                if (lane == 0)
-                    good = mbar_wait_parked(acce_bar(acc), acc_ph ^ 1u, s_abort, kp.limit_ns);
-                good = __shfl_sync(0xffffffffu, good, 0);
-                if (!good) {
-                    if (lane == 0)
-                        record_error(kp.error, kErrMmaAccEmpty, s_abort);
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t t_acc = tmem + (acc * NM + mma_idx) * BN;
-                for (uint32_t k = kb; k < ke; ++k) {
-                    good = 1;
-                    if (lane == 0)
-                        good = mbar_wait_parked(full_bar(s), ph, s_abort, kp.limit_ns);
-                    good = __shfl_sync(0xffffffffu, good, 0);
-                    if (!good) {
-                        if (lane == 0)
-                            record_error(kp.error, kErrMmaFull, s_abort);
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (lane == 0) {
-                        if (kp.fused_sf)            // scale atoms written by cp.async (generic proxy)
-                            fence_proxy_async_smem();
-                        const uint32_t t_sfa = t_sfa0 + s * C_::kSFACols;
-                        const uint32_t t_sfb = t_sfb0 + s * C_::kSFBCols;
-                        const uint32_t s_sfa = sbase + C_::kOffSFA + s * C_::kSFABytes;
-                        const uint32_t s_sfb = sbase + C_::kOffSFB + s * C_::kSFBBytes;
-#pragma unroll
-                        for (int a = a_begin; a < a_begin + C_::kAtomsPerMma; ++a)
-                            tmem_cp_32x128b_x4(t_sfa + 4 * a, sdesc_rows16(s_sfa + 512 * a));
-#pragma unroll
-                        for (int rb = 0; rb < C_::kRBQ; ++rb)
-#pragma unroll
-                            for (int a = a_begin; a < a_begin + C_::kAtomsPerMma; ++a)
-                                tmem_cp_32x128b_x4(t_sfb + a * 4 * C_::kRBQ + 4 * rb,
-                                                   sdesc_rows16(s_sfb + (rb * C_::kAtoms + a) * 512));
-                        // MMA q of the stage (chunk q / 4, 32-byte step q % 4) reads atom
-                        // q / kMmaPerAtom: MXFP8 one scale block per MMA (byte q % 4 of
-                        // the chunk's atom), MXFP4 two (byte pair 2 * (q % 2)).
-#pragma unroll
-                        for (int q = a_begin * C_::kMmaPerAtom; q < (a_begin + C_::kAtomsPerMma) * C_::kMmaPerAtom;
-                             ++q) {
-                            const int c = q / C_::kMmaPerChunk, j = q % C_::kMmaPerChunk;
-                            const int atom = q / C_::kMmaPerAtom;
-                            const uint64_t adesc =
-                                sdesc_sw128_kmajor(sbase + C_::kOffA + s * C_::kABytes + c * C_::kAChunk);
-                            const uint64_t bdesc =
-                                sdesc_sw128_kmajor(sbase + C_::kOffB + s * C_::kBBytes + c * C_::kBChunk);
-                            const uint32_t sf_id = FMT == kFmtMXFP8 ? j : 2 * (j % 2);
-                            const uint32_t idesc = kIdesc | (sf_id << 4) | (sf_id << 29);
-                            const uint32_t acc_flag = (k > kb || q > a_begin * C_::kMmaPerAtom) ? 1u : 0u;
-                            const uint64_t koff = static_cast<uint64_t>(j * 32) >> 4;
-                            if (FMT == kFmtMXFP8)
-                                mma_mxf8f6f4(t_acc, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
-                                             t_sfb + atom * 4 * C_::kRBQ, acc_flag);
-                            else
-                                mma_mxf4(t_acc, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
-                                         t_sfb + atom * 4 * C_::kRBQ, acc_flag);
-                        }
-                        tc_commit(empty_bar(s));
-                    }
-                    __syncwarp();
-                    if (++s == S) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
-                }
-                if (!ok)
-                    break;
-                if (lane == 0)
-                    tc_commit(accf_bar(acc));
-                __syncwarp();
-                if (++acc == C_::kNumAcc) {
-                    acc = 0;
-                    acc_ph ^= 1u;
-                }
-                it += ke - kb;
-            }
-        }
-        // Drain: every tcgen05 operation of every MMA warp has completed.
-        if (lane == 0) {
-            tc_commit(drain_bar);
-            int dummy_abort = 0;
-            if (!mbar_wait_parked(drain_bar, 0, &dummy_abort, kp.limit_ns))
-                atomicCAS(kp.error, 0, kErrDrain);
-        }
-        __syncwarp();
-    } else if (warp >= 2 && warp <= 5) {
-        // ---------------------------------------------------------- epilogue
-        grid_dependency_wait();
-        const int quad = warp & 3;             // TMEM lanes 32*quad .. +31
-        const int row = quad * 32 + lane;      // accumulator row = MMA row in tile
-        const int etid = threadIdx.x - 64;     // 0..127
-        int acc = 0;
-        uint32_t acc_ph = 0;
-        uint32_t out_chunks = 0;               // BF16 chunks staged so far (buffer = parity)
-        bool stop = false;
-        bool ring_out = false;                 // this segment may stage its output in ring stage 0
-
-        // The tile's accumulator is the sum of the NM MMA warps' accumulators.
-        auto load_acc = [&](uint32_t t_acc, int c, float (&v)[CW]) {
-            uint32_t r[CW];
-            tmem_ld_cols<CW>(t_acc + c, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < CW; ++j)
-                v[j] = __uint_as_float(r[j]);
-#pragma unroll
-            for (int m = 1; m < NM; ++m) {
-                tmem_ld_cols<CW>(t_acc + m * BN + c, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < CW; ++j)
-                    v[j] += __uint_as_float(r[j]);
-            }
-        };
-
-        // Convert one CW-column chunk of the tile (this thread's row) to BF16
-        // and write it to C: through shared memory and a TMA store when the
-        // output layout allows, else with predicated global stores.
-        auto emit = [&](const float (&v)[CW], int64_t tp, int64_t qcol) {
-            const int64_t p = tp * 128 + row;
-            if (!kp.tma_store || !(C_::kStaged || ring_out)) {
-                store_bf16<CW>(out, p, qcol, v);
-                return;
-            }
-            const int b = static_cast<int>(out_chunks & 1u);
-            uint8_t *buf = C_::kStaged ? smem + C_::kOffOut + b * C_::kOutBytes
-                                       : smem + C_::kOffA + b * C_::kChunkOutBytes;
-            if (etid == 0)
-                bulk_wait_group_read<1>();      // the store that last read this buffer is done
-            named_bar_sync(1, 128);
-            if (!kp.swap) {                     // [128 rows][CW] row-major, this thread's row
-                uint4 *dst = reinterpret_cast<uint4 *>(buf + row * CW * 2);
-#pragma unroll
-                for (int j = 0; j < CW / 8; ++j) {
-                    uint4 w;
-                    w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-                    w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-                    w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-                    w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-                    dst[j] = w;
-                }
-            } else {                            // [CW rows of C][128 columns of C]
-                __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(buf) + row;
-#pragma unroll
-                for (int j = 0; j < CW; ++j)
-                    dst[j * 128] = __float2bfloat16_rn(v[j]);
-            }
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (etid == 0) {
-                if (!kp.swap)
-                    tma_store_2d(&tmC, smem_u32(buf), static_cast<int32_t>(qcol), static_cast<int32_t>(tp * 128));
-                else
-                    tma_store_2d(&tmC, smem_u32(buf), static_cast<int32_t>(tp * 128), static_cast<int32_t>(qcol));
-                bulk_commit_group();
-            }
-            ++out_chunks;
-        };
-
-        for (uint32_t w = blockIdx.x; w < W && !stop; w += gridDim.x) {
-            uint32_t it = sc.begin(w);
-            const uint32_t end = sc.begin(w + 1);
-            bool first = true;
-            while (it < end) {
-                const Segment sg = segment_at(sc, it, end);
-                const uint32_t tile = sg.tile, kb = sg.kb, ke = sg.ke;
-                const int64_t tp = sg.tp, tq = sg.tq;
-                // the CTA's final segment: once its accumulator is complete every
-                // stage has been consumed and no further loads are coming
-                ring_out = (w + gridDim.x >= W) && (it + (ke - kb) >= end);
-                int good = 1;
-                if (lane == 0)
-                    good = mbar_wait_parked(accf_bar(acc), acc_ph, s_abort, kp.limit_ns);
-                good = __shfl_sync(0xffffffffu, good, 0);
-                if (!good && lane == 0)
-                    record_error(kp.error, kErrEpiAccFull, s_abort);
-                // One decision for all four epilogue warps.
-                if (named_bar_or(1, 128, (!good || *s_abort) ? 1 : 0)) {
-                    stop = true;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t t_acc = tmem + acc * NM * BN + (static_cast<uint32_t>(quad * 32) << 16);
-                const uint32_t g_first = sc.dp ? tile : sc.owner(tile * sc.KT);
-                const uint32_t g_last = sc.dp ? tile : sc.owner(tile * sc.KT + sc.KT - 1);
-                bool released = false;
-                if (g_first == g_last) {
-                    // Drain the accumulator row into registers as BF16 pairs and
-                    // hand the accumulator back before any store, so the next
-                    // tile's MMAs overlap this tile's output traffic.
-                    uint32_t packed[BN / 2];
-#pragma unroll
-                    for (int c = 0; c < BN; c += CW) {
-                        float v[CW];
-                        load_acc(t_acc, c, v);
-#pragma unroll
-                        for (int j = 0; j < CW / 2; ++j)
-                            packed[c / 2 + j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(acce_bar(acc));
-                    released = true;
-#pragma unroll
-                    for (int c = 0; c < BN; c += CW) {
-                        float v[CW];     // BF16 values widened back exactly
-#pragma unroll
-                        for (int j = 0; j < CW / 2; ++j) {
-                            v[2 * j] = __uint_as_float(packed[c / 2 + j] << 16);
-                            v[2 * j + 1] = __uint_as_float(packed[c / 2 + j] & 0xFFFF0000u);
-                        }
-                        emit(v, tp, tq * BN + c);
-                    }
-                } else {
-                    const int64_t slot = 2 * static_cast<int64_t>(w) + (first ? 0 : 1);
-                    float *mine = kp.partials + (slot * 128 + row) * BN;
-#pragma unroll 1
-                    for (int c = 0; c < BN; c += CW) {
-                        float v[CW];
-                        load_acc(t_acc, c, v);
-#pragma unroll
-                        for (int j = 0; j < CW / 4; ++j)
-                            reinterpret_cast<float4 *>(mine + c)[j] =
-                                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                    }
-                    __threadfence();
-                    named_bar_sync(1, 128);
-                    if (etid == 0) {
-                        const uint32_t nseg = g_last - g_first + 1;
-                        const uint32_t old = atomicAdd(kp.counters + tile, 1u);
-                        const int last = (old == nseg - 1) ? 1 : 0;
-                        if (last)
-                            kp.counters[tile] = 0u;
-                        *s_last = last;
-                    }
-                    named_bar_sync(1, 128);
-                    if (*s_last) {
-                        __threadfence();
-#pragma unroll 1
-                        for (int c = 0; c < BN; c += CW) {
-                            float own[CW];
-                            load_acc(t_acc, c, own);
-                            float v[CW];
-#pragma unroll
-                            for (int j = 0; j < CW; ++j)
-                                v[j] = 0.0f;
-                            for (uint32_t g = g_first; g <= g_last; ++g) {
-                                if (g == w) {
-#pragma unroll
-                                    for (int j = 0; j < CW; ++j)
-                                        v[j] += own[j];
-                                } else {
-                                    const int64_t gslot =
-                                        2 * static_cast<int64_t>(g) + ((sc.begin(g) / sc.KT == tile) ? 0 : 1);
-                                    const float4 *src = reinterpret_cast<const float4 *>(
-                                        kp.partials + (gslot * 128 + row) * BN + c);
-#pragma unroll
-                                    for (int j = 0; j < CW / 4; ++j) {
-                                        const float4 x = __ldcg(src + j);
-                                        v[4 * j + 0] += x.x;
-                                        v[4 * j + 1] += x.y;
-                                        v[4 * j + 2] += x.z;
-                                        v[4 * j + 3] += x.w;
-                                    }
-                                }
-                            }
-                            emit(v, tp, tq * BN + c);
-                        }
-                    }
-                }
-                if (!released) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(acce_bar(acc));
-                }
-                if (++acc == C_::kNumAcc) {
-                    acc = 0;
-                    acc_ph ^= 1u;
-                }
-                first = false;
-                it += ke - kb;
-            }
-        }
-        // Output stores must finish reading shared memory before the CTA exits.
-        if (etid == 0)
-            bulk_wait_group<0>();
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 1)
-        tmem_dealloc(tmem, C_::kTmemCols);
-}
-
-// ------------------------------------------------------ CTA-pair kernel
-//
-// Large-M form: a cluster of two CTAs computes a 256x256 output tile with
-// tcgen05.mma.cta_group::2 (M = 256, N = 256).  Each CTA loads its own 128
-// rows of A and its own 128 rows of B (no multicast), the scale atoms of its
-// A rows and of all 256 B rows; the even CTA (the leader) issues the scale
-// copies and MMAs for both and its commits arrive in both CTAs.  Per CTA this
-// halves the operand bytes per MMA against a 128x256 tile on one SM.
-//
-// Hand-offs across the pair: the odd CTA's MMA warp is idle, so it relays
-// "my stage has landed" to the leader (wait on its own full barrier, then a
-// cluster-scope remote arrive); both CTAs' epilogues tell the leader when the
-// accumulator may be reused with remote arrives as well.
-
-template <int FMT, int KC>
-struct PairCfg {
-    static constexpr int kAtomsPerChunk = FMT == kFmtMXFP8 ? 1 : 2;
-    static constexpr int kAtoms = kAtomsPerChunk * KC;
-    static constexpr int kChunk = 128 * 128;                  // 128 rows x 128 bytes of K
-    static constexpr int kABytes = kChunk * KC;               // this CTA's 128 rows of A
-    static constexpr int kBBytes = kChunk * KC;               // this CTA's 128 rows of B
-    static constexpr int kSFABytes = kAtoms * 512;            // scales of this CTA's A rows
-    static constexpr int kSFBBytes = 2 * kAtoms * 512;        // scales of all 256 B rows
-    static constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
-    // output staging: two BF16 chunks of 128 rows x kCW columns; 16-column
-    // chunks when the smaller staging buys the ring another stage
-    static constexpr int stages_with(int cw)
-    {
-        return (227 * 1024 - 2048 - 2 * 128 * cw * 2) / kStageBytes;
-    }
-    static constexpr int kCW = stages_with(16) > stages_with(32) ? 16 : 32;
-    static constexpr int kOutBytes = 128 * kCW * 2;
-    static constexpr int kSmemBudget = 227 * 1024 - 2048 - 2 * kOutBytes;
-    static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
-    static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-    static constexpr int kSFACols = kAtoms * 4;
-    static constexpr int kSFBCols = 2 * kAtoms * 4;
-    static constexpr int kAccCols = 256;
-    static constexpr int kTmemCols = 512;
-    static constexpr uint32_t kTxBytes = kStageBytes;
-    static constexpr int kOffA = 0;
-    static constexpr int kOffB = kOffA + kStages * kABytes;
-    static constexpr int kOffSFA = kOffB + kStages * kBBytes;
-    static constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
-    static constexpr int kOffOut = (kOffSFB + kStages * kSFBBytes + 1023) / 1024 * 1024;
-    static constexpr int kOffBar = kOffOut + 2 * kOutBytes;
-    static constexpr int kNumBars = 4 * kStages + 3;   // full, empty, pair_full, scales-ready; accf, acce, drain
-    static constexpr int kThreads = 256;                 // warps 0..6 as the 1-CTA kernel, 7 scale copies
-    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
-
-    static_assert(kStages >= 2, "at least two pipeline stages");
-    static_assert(kAccCols + kStages * (kSFACols + kSFBCols) <= kTmemCols, "TMEM budget");
-    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-};
-
-template <int FMT>
-__host__ __device__ constexpr uint32_t idesc_pair()
-{
-    constexpr uint32_t t = FMT == kFmtMXFP8 ? 0u : 1u;
-    return (t << 7) | (t << 10) | (static_cast<uint32_t>(256 >> 3) << 17) | (1u << 23) |
-           (static_cast<uint32_t>(256 >> 4) << 24);
-}
-
-template <int FMT, int KC>
-__global__ void __launch_bounds__(256, 1)
-    mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
-                        const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
-                        const __grid_constant__ CUtensorMap tmC, const KParams kp_in)
-{
-    using C_ = PairCfg<FMT, KC>;
-    constexpr int S = C_::kStages;
-    constexpr int CW = C_::kCW;
-    const KParams kp = kp_in;
-
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~static_cast<uintptr_t>(1023));
-    const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar0 = sbase + C_::kOffBar;
-    auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
-    auto pfull_bar = [&](int s) { return bar0 + 8u * (2 * S + s); };
-    auto sfr_bar = [&](int s) { return bar0 + 8u * (3 * S + s); };     // leader: stage's scales in TMEM
-    const uint32_t accf_bar = bar0 + 8u * (4 * S);
-    const uint32_t acce_bar = bar0 + 8u * (4 * S + 1);
-    const uint32_t drain_bar = bar0 + 8u * (4 * S + 2);
-    volatile uint32_t *s_tmem = reinterpret_cast<volatile uint32_t *>(smem + C_::kOffMisc);
-    volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C_::kOffMisc + 4);
-
-    if (blockDim.x != C_::kThreads) {     // uniform over the cluster: both CTAs return
-        if (threadIdx.x == 0)
-            atomicCAS(kp.error, 0, kErrLaunch);
-        return;
-    }
-    const int warp = threadIdx.x / 32;
-    const int lane = threadIdx.x % 32;
-    const uint32_t rank = cluster_ctarank();
-    const bool leader = rank == 0;
-    const uint32_t pair = blockIdx.x / 2, npairs = gridDim.x / 2;
-    const uint32_t tiles = kp.workers, tilesP = kp.tilesP, KT = kp.kt;
-
-    if (threadIdx.x == 0) {
-        tma_prefetch_desc(&tmP);
-        tma_prefetch_desc(&tmQ);
-        tma_prefetch_desc(&tmSP);
-        tma_prefetch_desc(&tmSQ);
-        tma_prefetch_desc(&tmC);
-        for (int s = 0; s < S; ++s) {
-            mbar_init(full_bar(s), 2);          // one arming per producer warp
-            mbar_init(empty_bar(s), 1);
-            mbar_init(pfull_bar(s), 1);
-            mbar_init(sfr_bar(s), 1);
-        }
-        mbar_init(accf_bar, 1);
-        mbar_init(acce_bar, 8);
-        mbar_init(drain_bar, 2);            // MMA warp and scale-copy warp of the leader
-        *s_abort = 0;
-        fence_mbar_init();
-        fence_proxy_async_smem();
-    }
-    if (warp == 1) {
-        tmem_alloc_pair(sbase + C_::kOffMisc, C_::kTmemCols);
-        tmem_relinquish_pair();
-    }
-    tc_fence_before();
-    cluster_sync_all();
-    tc_fence_after();
-    const uint32_t tmem = *s_tmem;
-
-    if (warp != 0 && warp != 6)
-        grid_dependency_wait();
-
-    if (warp == 0 || warp == 6) {
-        // ----------------------------------------------------- TMA producers
-        // Warp 0: this CTA's 128 rows of A and their scale atoms; warp 6: its
-        // 128 rows of B and the scale atoms of all 256 B rows of the tile.
-        const bool sideA = warp == 0;
-        if (lane == 0) {
-            const uint64_t pol = policy_evict_normal();
-            const CUtensorMap *tmOp = sideA ? &tmP : &tmQ;
-            const CUtensorMap *tmSf = sideA ? &tmSP : &tmSQ;
-            const uint32_t opBytes = sideA ? C_::kABytes : C_::kBBytes;
-            const uint32_t sfBytes = sideA ? C_::kSFABytes : C_::kSFBBytes;
-            const uint32_t offOp = sideA ? C_::kOffA : C_::kOffB;
-            const uint32_t offSf = sideA ? C_::kOffSFA : C_::kOffSFB;
-            uint32_t armed = 0;
-            int skipped_stage = -1;
-            bool inject = sideA && kp.inject == 1;
-            int s = 0;
-            uint32_t ph = 0;
-            bool first = true;
-            for (uint32_t tile = pair; tile < tiles; tile += npairs) {
-                const uint32_t tq = tile / tilesP, tp = tile - tq * tilesP;
-                const int32_t row = static_cast<int32_t>((sideA ? tp : tq) * 256 + rank * 128);
-                const int32_t sf_rb = sideA ? static_cast<int32_t>(tp * 2 + rank) : static_cast<int32_t>(tq * 2);
-                bool ok = true;
-                for (uint32_t k = 0; k < KT; ++k) {
-                    if (!mbar_wait_parked(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns)) {
-                        record_error(kp.error, kErrProducerEmpty, s_abort);
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t fb = full_bar(s);
-                    if (inject) {
-                        inject = false;
-                        skipped_stage = s;
-                    } else {
-                        mbar_arrive_expect_tx(fb, opBytes + sfBytes);
-                        if constexpr (KC == 1)
-                            tma_load_2d(sbase + offOp + s * opBytes, tmOp, static_cast<int32_t>(k * 128), row, fb, pol);
-                        else
-                            tma_load_3d(sbase + offOp + s * opBytes, tmOp, 0, row, static_cast<int32_t>(k * KC), fb,
-                                        pol);
-                        if (first) {            // operands of stage 0 may overlap the preceding kernel
-                            grid_dependency_wait();
-                            first = false;
-                        }
-                        tma_load_3d(sbase + offSf + s * sfBytes, tmSf, 0, static_cast<int32_t>(k * C_::kAtoms),
-                                    sf_rb, fb, pol);
-                    }
-                    ++armed;
-                    if (++s == S) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
-                }
-                if (!ok)
-                    break;
-            }
-            if (first)
-                grid_dependency_wait();
-            for (int st = 0; st < S; ++st) {
-                const uint32_t n = armed / S + (static_cast<uint32_t>(st) < armed % S ? 1u : 0u);
-                if (n == 0 || (st == skipped_stage && n == 1))
-                    continue;
-                int dummy_abort = 0;
-                if (!mbar_wait_parked(full_bar(st), (n - 1) & 1u, &dummy_abort, kp.limit_ns))
-                    atomicCAS(kp.error, 0, kErrDrain);
-            }
-        }
-        __syncwarp();
-    } else if (warp == 1 && !leader) {
-        // ------------------------------------- relay: this CTA's stages landed
-        if (lane == 0) {
-            int s = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            for (uint32_t tile = pair; tile < tiles && ok; tile += npairs) {
-                for (uint32_t k = 0; k < KT; ++k) {
-                    if (!mbar_wait_parked(full_bar(s), ph, s_abort, kp.limit_ns)) {
-                        record_error(kp.error, kErrMmaFull, s_abort);
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_remote(pfull_bar(s), 0);
-                    if (++s == S) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
-                }
-            }
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------- MMA issuer (leader CTA)
-        constexpr uint32_t kIdesc = idesc_pair<FMT>();
-        const uint32_t t_sfa0 = tmem + C_::kAccCols;
-        const uint32_t t_sfb0 = t_sfa0 + S * C_::kSFACols;
-        int s = 0;
-        uint32_t ph = 0;
-        uint32_t acc_ph = 0;
-        bool ok = true;
-        for (uint32_t tile = pair; tile < tiles && ok; tile += npairs) {
-            int good = 1;
-            if (lane == 0)
-                good = mbar_wait_cluster_bounded(acce_bar, acc_ph ^ 1u, s_abort, kp.limit_ns);
-            good = __shfl_sync(0xffffffffu, good, 0);
-            if (!good) {
-                if (lane == 0)
-                    record_error(kp.error, kErrMmaAccEmpty, s_abort);
-                break;
-            }
-            tc_fence_after();
-            for (uint32_t k = 0; k < KT; ++k) {
-                good = 1;
-                if (lane == 0)
-                    // the MMA warp alone spins: it feeds the tensor pipe
-                    good = mbar_wait_bounded(sfr_bar(s), ph, s_abort, kp.limit_ns);
-                good = __shfl_sync(0xffffffffu, good, 0);
-                if (!good) {
-                    if (lane == 0)
-                        record_error(kp.error, kErrMmaFull, s_abort);
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t t_sfa = t_sfa0 + s * C_::kSFACols;
-                    const uint32_t t_sfb = t_sfb0 + s * C_::kSFBCols;
-#pragma unroll
-                    for (int c = 0; c < KC; ++c) {
-                        const uint64_t adesc = sdesc_sw128_kmajor(sbase + C_::kOffA + s * C_::kABytes + c * C_::kChunk);
-                        const uint64_t bdesc = sdesc_sw128_kmajor(sbase + C_::kOffB + s * C_::kBBytes + c * C_::kChunk);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int atom = FMT == kFmtMXFP8 ? c : 2 * c + j / 2;
-                            const uint32_t sf_id = FMT == kFmtMXFP8 ? j : 2 * (j % 2);
-                            const uint32_t idesc = kIdesc | (sf_id << 4) | (sf_id << 29);
-                            const uint32_t acc_flag = (k > 0 || c > 0 || j > 0) ? 1u : 0u;
-                            const uint64_t koff = static_cast<uint64_t>(j * 32) >> 4;
-                            if (FMT == kFmtMXFP8)
-                                mma_mxf8f6f4_pair(tmem, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
-                                                  t_sfb + atom * 8, acc_flag);
-                            else
-                                mma_mxf4_pair(tmem, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
-                                              t_sfb + atom * 8, acc_flag);
-                        }
-                    }
-                    tc_commit_pair(empty_bar(s), 0x3);
-                }
-                __syncwarp();
-                if (++s == S) {
-                    s = 0;
-                    ph ^= 1u;
-                }
-            }
-            if (!ok)
-                break;
-            if (lane == 0)
-                tc_commit_pair(accf_bar, 0x3);
-            __syncwarp();
-            acc_ph ^= 1u;
-        }
-        if (lane == 0) {
-            tc_commit_pair(drain_bar, 0x1);
-            int dummy_abort = 0;
-            if (!mbar_wait_parked(drain_bar, 0, &dummy_abort, kp.limit_ns))
-                atomicCAS(kp.error, 0, kErrDrain);
-        }
-        __syncwarp();
-    } else if (warp == 7 && leader) {
-        // ------------------------------ scale copies into TMEM (leader CTA)
-        // Once both CTAs' stage has landed, copy the scale atoms of both
-        // CTAs' A rows and of the tile's B rows into the stage's TMEM slots
-        // (cta_group::2 copies write both CTAs' TMEM), then signal the MMA
-        // warp.  Issuing the copies beside the MMAs keeps them off the MMA
-        // warp's issue stream, where they would add to every stage.
-        const uint32_t t_sfa0 = tmem + C_::kAccCols;
-        const uint32_t t_sfb0 = t_sfa0 + S * C_::kSFACols;
-        int s = 0;
-        uint32_t ph = 0;
-        bool ok = true;
-        for (uint32_t tile = pair; tile < tiles && ok; tile += npairs) {
-            for (uint32_t k = 0; k < KT; ++k) {
-                int good = 1;
-                if (lane == 0) {
-                    good = mbar_wait_parked(full_bar(s), ph, s_abort, kp.limit_ns);
-                    if (good)
-                        good = mbar_wait_cluster_bounded(pfull_bar(s), ph, s_abort, kp.limit_ns);
-                }
-                good = __shfl_sync(0xffffffffu, good, 0);
-                if (!good) {
-                    if (lane == 0)
-                        record_error(kp.error, kErrMmaFull, s_abort);
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t t_sfa = t_sfa0 + s * C_::kSFACols;
-                    const uint32_t t_sfb = t_sfb0 + s * C_::kSFBCols;
-                    const uint32_t s_sfa = sbase + C_::kOffSFA + s * C_::kSFABytes;
-                    const uint32_t s_sfb = sbase + C_::kOffSFB + s * C_::kSFBBytes;
-#pragma unroll
-                    for (int a = 0; a < C_::kAtoms; ++a)
-                        tmem_cp_32x128b_x4_pair(t_sfa + 4 * a, sdesc_rows16(s_sfa + 512 * a));
-#pragma unroll
-                    for (int rb = 0; rb < 2; ++rb)
-#pragma unroll
-                        for (int a = 0; a < C_::kAtoms; ++a)
-                            tmem_cp_32x128b_x4_pair(t_sfb + a * 8 + 4 * rb,
-                                                    sdesc_rows16(s_sfb + (rb * C_::kAtoms + a) * 512));
-                    tc_commit_pair(sfr_bar(s), 0x1);
-                }
-                __syncwarp();
-                if (++s == S) {
-                    s = 0;
-                    ph ^= 1u;
-                }
-            }
-        }
-        if (lane == 0) {
-            tc_commit_pair(drain_bar, 0x1);
-            int dummy_abort = 0;
-            if (!mbar_wait_parked(drain_bar, 0, &dummy_abort, kp.limit_ns))
-                atomicCAS(kp.error, 0, kErrDrain);
-        }
-        __syncwarp();
-    } else if (warp >= 2 && warp <= 5) {
-        // ---------------------------------------------------------- epilogue
-        const int quad = warp & 3;
-        const int row = quad * 32 + lane;
-        const int etid = threadIdx.x - 64;
-        uint32_t acc_ph = 0;
-        uint32_t out_chunks = 0;
-        for (uint32_t tile = pair; tile < tiles; tile += npairs) {
-            const uint32_t tq = tile / tilesP, tp = tile - tq * tilesP;
-            int good = 1;
-            if (lane == 0)
-                good = mbar_wait_parked(accf_bar, acc_ph, s_abort, kp.limit_ns);
-            good = __shfl_sync(0xffffffffu, good, 0);
-            if (!good && lane == 0)
-                record_error(kp.error, kErrEpiAccFull, s_abort);
-            if (named_bar_or(1, 128, (!good || *s_abort) ? 1 : 0))
-                break;
-            tc_fence_after();
-            const uint32_t t_acc = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-            // Drain the whole accumulator row into registers (BF16 pairs) and
-            // hand the accumulator back to the MMA warp before any store, so
-            // the next tile's MMAs overlap this tile's output traffic.
-            uint32_t packed[128];
-#pragma unroll
-            for (int c = 0; c < 256; c += CW) {
-                uint32_t r[CW];
-                tmem_ld_cols<CW>(t_acc + c, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < CW / 2; ++j)
-                    packed[c / 2 + j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if (leader)
-                    mbar_arrive(acce_bar);
-                else
-                    mbar_arrive_remote(acce_bar, 0);
-            }
-#pragma unroll
-            for (int c = 0; c < 256; c += CW) {
-                const int b = static_cast<int>(out_chunks & 1u);
-                uint8_t *buf = smem + C_::kOffOut + b * C_::kOutBytes;
-                if (etid == 0)
-                    bulk_wait_group_read<1>();
-                named_bar_sync(1, 128);
-                uint4 *dst = reinterpret_cast<uint4 *>(buf + row * CW * 2);
-#pragma unroll
-                for (int j = 0; j < CW / 8; ++j)
-                    dst[j] = make_uint4(packed[c / 2 + 4 * j], packed[c / 2 + 4 * j + 1], packed[c / 2 + 4 * j + 2],
-                                        packed[c / 2 + 4 * j + 3]);
-                fence_proxy_async_smem();
-                named_bar_sync(1, 128);
-                if (etid == 0) {
-                    tma_store_2d(&tmC, smem_u32(buf), static_cast<int32_t>(tq * 256 + c),
-                                 static_cast<int32_t>(tp * 256 + rank * 128));
-                    bulk_commit_group();
-                }
-                ++out_chunks;
-            }
-            acc_ph ^= 1u;
-        }
-        if (etid == 0)
-            bulk_wait_group<0>();
-    }
-
-    tc_fence_before();
-    cluster_sync_all();
-    tc_fence_after();
-    if (warp == 1)
-        tmem_dealloc_pair(tmem, C_::kTmemCols);
-}
-
-// ------------------------------------------------------------------- host
-
 namespace {
-
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
-                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                   CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// 2-D uint8 map over [rows][row_bytes] with a box of 128 bytes x box_rows,
-// 128-byte swizzle, zero fill out of bounds.
-bool make_operand_map(CUtensorMap *map, const void *base, int64_t rows, int64_t rbytes, int box_rows)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn)
-        return false;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(rbytes), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(rbytes)};
-    cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(box_rows)};
-    cuuint32_t estr[2] = {1u, 1u};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-// 3-D uint8 map viewing [rows][row_bytes] as {128-byte piece, row, chunk}
-// (strides: row_bytes between rows, 128 bytes between chunks) with a box of
-// 128 bytes x box_rows x kc chunks, 128-byte swizzle, zero fill out of
-// bounds.  Needs row_bytes % 128 == 0.
-bool make_operand_map_3d(CUtensorMap *map, const void *base, int64_t rows, int64_t rbytes, int box_rows, int kc)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn || rbytes % 128 != 0)
-        return false;
-    cuuint64_t dims[3] = {128u, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(rbytes / 128)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(rbytes), 128u};
-    cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(kc)};
-    cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-// 3-D uint32 map over a repacked scale buffer [row blocks][ka][512 bytes]:
-// {128 words of an atom, atom, 128-row block}, box {128, atoms, row blocks}.
-bool make_sf_map(CUtensorMap *map, const uint8_t *base, int64_t ka, int64_t row_blocks, int atoms, int rbs)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn)
-        return false;
-    cuuint64_t dims[3] = {128u, static_cast<cuuint64_t>(ka), static_cast<cuuint64_t>(row_blocks)};
-    cuuint64_t strides[2] = {512u, static_cast<cuuint64_t>(ka) * 512u};
-    cuuint32_t box[3] = {128u, static_cast<cuuint32_t>(atoms), static_cast<cuuint32_t>(rbs)};
-    cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-inline int64_t sf_row_blocks(int64_t rows) { return (rows + 255) / 256 * 2; }
-
-template <int FMT, int BN, int KC>
-cudaError_t set_attrs()
-{
-    return cudaFuncSetAttribute(mx_gemm_kernel<FMT, BN, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Cfg<FMT, BN, KC>::kSmemBytes);
-}
-
-// 2-D BF16 map over C [M][N] with a box of box_x (inner, along N) x box_y
-// rows, no swizzle; used by the epilogue's TMA stores.
-bool make_output_map(CUtensorMap *map, void *C, int64_t M, int64_t N, int box_x, int box_y)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn)
-        return false;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * 2};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_x), static_cast<cuuint32_t>(box_y)};
-    cuuint32_t estr[2] = {1u, 1u};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, C, dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-template <int FMT, int BN, int KC>
-cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
-                     cudaStream_t st)
-{
-    using C_ = Cfg<FMT, BN, KC>;
-    const int64_t rbytes = row_bytes(FMT, pl.K);
-    const void *Pptr = pl.swap ? b.B : b.A;
-    const void *Qptr = pl.swap ? b.A : b.B;
-    CUtensorMap tmP, tmQ, tmC;
-    if (KC == 1) {
-        if (!make_operand_map(&tmP, Pptr, pl.P, rbytes, 128) || !make_operand_map(&tmQ, Qptr, pl.Q, rbytes, BN))
-            return cudaErrorInvalidValue;
-    } else {
-        if (!make_operand_map_3d(&tmP, Pptr, pl.P, rbytes, 128, KC) ||
-            !make_operand_map_3d(&tmQ, Qptr, pl.Q, rbytes, BN, KC))
-            return cudaErrorInvalidValue;
-    }
-    // TMA stores need 16-byte row pitch; other widths take the predicated
-    // store path (the map is then a never-used placeholder over C).
-    const int tma_store = (pl.N % 8 == 0) ? 1 : 0;
-    const bool okC = tma_store ? (pl.swap ? make_output_map(&tmC, b.C, pl.M, pl.N, 128, C_::kCW)
-                                          : make_output_map(&tmC, b.C, pl.M, pl.N, C_::kCW, 128))
-                               : make_output_map(&tmC, b.C, 1, 8, 8, 1);
-    if (!okC)
-        return cudaErrorInvalidValue;
-    CUtensorMap tmSP, tmSQ;
-    const bool fused = b.rawA != nullptr;
-    const uint8_t *rawP = pl.swap ? b.rawB : b.rawA;
-    const uint8_t *rawQ = pl.swap ? b.rawA : b.rawB;
-    // with fused scales the repacked maps are never read: encode them over
-    // the row-major scales so they are valid
-    const uint8_t *sfP = fused ? rawP : (pl.swap ? b.sfB : b.sfA);
-    const uint8_t *sfQ = fused ? rawQ : (pl.swap ? b.sfA : b.sfB);
-    if (!make_sf_map(&tmSP, sfP, pl.kaP, sf_row_blocks(pl.P), C_::kAtoms, 1) ||
-        !make_sf_map(&tmSQ, sfQ, pl.kaQ, sf_row_blocks(pl.Q), C_::kAtoms, C_::kRBQ))
-        return cudaErrorInvalidValue;
-    KParams kp;
-    kp.C = reinterpret_cast<__nv_bfloat16 *>(b.C);
-    kp.partials = b.partials;
-    kp.counters = b.counters;
-    kp.error = b.error;
-    kp.P = pl.P;
-    kp.Q = pl.Q;
-    kp.ldc = pl.N;
-    kp.tilesP = static_cast<uint32_t>(pl.tilesP);
-    kp.kt = static_cast<uint32_t>(pl.kt);
-    kp.iters = static_cast<uint32_t>(pl.iters);
-    kp.workers = static_cast<uint32_t>(pl.workers);
-    kp.dp = pl.workers == pl.tiles ? 1 : 0;
-    kp.limit_ns = limit_ns;
-    kp.swap = pl.swap;
-    kp.inject = inject;
-    kp.tma_store = tma_store;
-    kp.fused_sf = fused ? 1 : 0;
-    kp.rawP = rawP;
-    kp.rawQ = rawQ;
-    kp.ldS = pl.K / 32;
-    // bits of b.early are per operand (A, B); the kernel's are per side (P, Q)
-    kp.early = pl.swap ? (((b.early & 1) << 1) | ((b.early >> 1) & 1)) : b.early;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
-    cfg.blockDim = dim3(C_::kThreads);
-    cfg.dynamicSmemBytes = C_::kSmemBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, mx_gemm_kernel<FMT, BN, KC>, tmP, tmQ, tmSP, tmSQ, tmC, kp);
-}
-
-template <int FMT, int KC>
-cudaError_t dispatch_bn(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
-                        cudaStream_t st)
-{
-    switch (pl.bn) {
-    case 16: return launch_t<FMT, 16, KC>(pl, b, limit_ns, inject, pdl, st);
-    case 32: return launch_t<FMT, 32, KC>(pl, b, limit_ns, inject, pdl, st);
-    case 64: return launch_t<FMT, 64, KC>(pl, b, limit_ns, inject, pdl, st);
-    case 128: return launch_t<FMT, 128, KC>(pl, b, limit_ns, inject, pdl, st);
-    case 256: return launch_t<FMT, 256, KC>(pl, b, limit_ns, inject, pdl, st);
-    default: return cudaErrorInvalidValue;
-    }
-}
-
-template <int FMT, int KC>
-cudaError_t launch_pair_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
-                          cudaStream_t st)
-{
-    using C_ = PairCfg<FMT, KC>;
-    const int64_t rbytes = row_bytes(FMT, pl.K);
-    CUtensorMap tmP, tmQ, tmC;
-    if (KC == 1) {
-        if (!make_operand_map(&tmP, b.A, pl.M, rbytes, 128) || !make_operand_map(&tmQ, b.B, pl.N, rbytes, 128))
-            return cudaErrorInvalidValue;
-    } else {
-        if (!make_operand_map_3d(&tmP, b.A, pl.M, rbytes, 128, KC) ||
-            !make_operand_map_3d(&tmQ, b.B, pl.N, rbytes, 128, KC))
-            return cudaErrorInvalidValue;
-    }
-    if (!make_output_map(&tmC, b.C, pl.M, pl.N, C_::kCW, 128))
-        return cudaErrorInvalidValue;
-    CUtensorMap tmSP, tmSQ;
-    if (!make_sf_map(&tmSP, b.sfA, pl.kaP, sf_row_blocks(pl.M), C_::kAtoms, 1) ||
-        !make_sf_map(&tmSQ, b.sfB, pl.kaQ, sf_row_blocks(pl.N), C_::kAtoms, 2))
-        return cudaErrorInvalidValue;
-    KParams kp;
-    kp.C = reinterpret_cast<__nv_bfloat16 *>(b.C);
-    kp.partials = nullptr;
-    kp.counters = nullptr;
-    kp.error = b.error;
-    kp.P = pl.M;
-    kp.Q = pl.N;
-    kp.ldc = pl.N;
-    kp.tilesP = static_cast<uint32_t>(pl.tilesP);
-    kp.kt = static_cast<uint32_t>(pl.kt);
-    kp.iters = static_cast<uint32_t>(pl.iters);
-    kp.workers = static_cast<uint32_t>(pl.tiles);
-    kp.dp = 1;
-    kp.limit_ns = limit_ns;
-    kp.swap = 0;
-    kp.inject = inject;
-    kp.tma_store = 1;
-    kp.fused_sf = 0;
-    kp.rawP = nullptr;
-    kp.rawQ = nullptr;
-    kp.ldS = pl.K / 32;
-    kp.early = 3;              // this kernel's operand producers never wait (it follows the repack)
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
-    cfg.blockDim = dim3(C_::kThreads);
-    cfg.dynamicSmemBytes = C_::kSmemBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, mx_gemm_pair_kernel<FMT, KC>, tmP, tmQ, tmSP, tmSQ, tmC, kp);
-}
-
-template <int FMT>
-cudaError_t dispatch_bn4(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
-                         cudaStream_t st)
-{
-    switch (pl.bn) {
-    case 16: return launch_t<FMT, 16, 4>(pl, b, limit_ns, inject, pdl, st);
-    case 32: return launch_t<FMT, 32, 4>(pl, b, limit_ns, inject, pdl, st);
-    case 64: return launch_t<FMT, 64, 4>(pl, b, limit_ns, inject, pdl, st);
-    default: return cudaErrorInvalidValue;
-    }
-}
-
-template <int FMT, int KC>
-int stages_kc(int bn)
-{
-    switch (bn) {
-    case 16: return Cfg<FMT, 16, KC>::kStages;
-    case 32: return Cfg<FMT, 32, KC>::kStages;
-    case 64: return Cfg<FMT, 64, KC>::kStages;
-    case 128: return Cfg<FMT, 128, KC>::kStages;
-    case 256: return Cfg<FMT, 256, KC>::kStages;
-    default: return 0;
-    }
-}
-
-template <int FMT>
-int stages_kc4(int bn)
-{
-    switch (bn) {
-    case 16: return Cfg<FMT, 16, 4>::kStages;
-    case 32: return Cfg<FMT, 32, 4>::kStages;
-    case 64: return Cfg<FMT, 64, 4>::kStages;
-    default: return 0;
-    }
-}
 
 int stages_for(int fmt, int bn, int kc)
 {
-    if (kc == 4)
-        return fmt == kFmtMXFP8 ? stages_kc4<0>(bn) : stages_kc4<1>(bn);
-    if (fmt == kFmtMXFP8)
-        return kc == 1 ? stages_kc<0, 1>(bn) : stages_kc<0, 2>(bn);
-    return kc == 1 ? stages_kc<1, 1>(bn) : stages_kc<1, 2>(bn);
+    return fmt == kFmtMXFP8 ? stages_mxfp8(bn, kc) : (fmt == kFmtMXFP4 ? stages_mxfp4(bn, kc) : stages_bf16(bn, kc));
 }
 
 }  // namespace
 
 cudaError_t prepare_gemm_kernels()
 {
-    cudaError_t e = cudaSuccess;
-#define MXG_ATTR(F, B)                                                  \
-    if (e == cudaSuccess)                                               \
-        e = set_attrs<F, B, 1>();                                       \
-    if (e == cudaSuccess)                                               \
-        e = set_attrs<F, B, 2>();
-    MXG_ATTR(0, 16) MXG_ATTR(0, 32) MXG_ATTR(0, 64) MXG_ATTR(0, 128) MXG_ATTR(0, 256)
-    MXG_ATTR(1, 16) MXG_ATTR(1, 32) MXG_ATTR(1, 64) MXG_ATTR(1, 128) MXG_ATTR(1, 256)
-#undef MXG_ATTR
-#define MXG_ATTRP(F, KCV)                                               \
-    if (e == cudaSuccess)                                               \
-        e = cudaFuncSetAttribute(mx_gemm_pair_kernel<F, KCV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                 PairCfg<F, KCV>::kSmemBytes);
-    MXG_ATTRP(0, 1) MXG_ATTRP(0, 2) MXG_ATTRP(1, 1) MXG_ATTRP(1, 2)
-#undef MXG_ATTRP
-#define MXG_ATTR4(F, B)                                                 \
-    if (e == cudaSuccess)                                               \
-        e = set_attrs<F, B, 4>();
-    MXG_ATTR4(0, 16) MXG_ATTR4(0, 32) MXG_ATTR4(0, 64) MXG_ATTR4(1, 16) MXG_ATTR4(1, 32) MXG_ATTR4(1, 64)
-#undef MXG_ATTR4
+    cudaError_t e = prepare_mxfp8();
+    if (e == cudaSuccess)
+        e = prepare_mxfp4();
+    if (e == cudaSuccess)
+        e = prepare_bf16();
+    if (e == cudaSuccess)
+        e = prepare_pair();
     return e;
 }
 
 GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sched, int splits, int workers,
-                   int force_kc)
+                   int force_kc, bool allow_pair)
 {
     GemmPlan pl;
     pl.fmt = fmt;
@@ -1677,7 +74,7 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
     {
         const int64_t ptiles = ((M + 255) / 256) * ((N + 255) / 256);
         const char *e = getenv("MXGEMM_PAIR");
-        const bool allow = !(e && atoi(e) == 0);
+        const bool allow = allow_pair && fmt != kFmtBF16 && !(e && atoi(e) == 0);
         if (allow && !pl.swap && M >= 512 && N >= 256 && N % 8 == 0 && ptiles >= 64)
             pl.pair = 1;
     }
@@ -1687,13 +84,17 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
             pl.kc = (whole && chunks >= 2) ? 2 : 1;
         else
             pl.kc = (force_kc == 2 && whole) ? 2 : 1;
-        pl.stages = fmt == kFmtMXFP8 ? (pl.kc == 1 ? PairCfg<0, 1>::kStages : PairCfg<0, 2>::kStages)
-                                     : (pl.kc == 1 ? PairCfg<1, 1>::kStages : PairCfg<1, 2>::kStages);
+        pl.stages = stages_pair(fmt, pl.kc);
         pl.tilesP = (M + 255) / 256;
         pl.tilesQ = (N + 255) / 256;
         pl.kt = (chunks + pl.kc - 1) / pl.kc;
         pl.tiles = pl.tilesP * pl.tilesQ;
         pl.iters = pl.tiles * pl.kt;
+        // tile order: bands of tile rows (measurement knob MXGEMM_BAND)
+        pl.band = pl.tilesP;
+        if (const char *e = getenv("MXGEMM_BAND"))
+            if (atoi(e) > 0)
+                pl.band = atoi(e) < pl.tilesP ? atoi(e) : pl.tilesP;
         const int64_t pairs = (num_sms > 0 ? num_sms : 2) / 2;
         pl.workers = pl.tiles;
         pl.grid = static_cast<int>(2 * (pl.tiles < pairs ? pl.tiles : pairs));
@@ -1762,24 +163,50 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
     return pl;
 }
 
+GemmPlan make_grouped_plan(int fmt, int64_t G, int64_t M_total, int64_t N, int64_t K, int num_sms)
+{
+    GemmPlan pl;
+    pl.fmt = fmt;
+    pl.M = M_total;
+    pl.N = N;
+    pl.K = K;
+    pl.swap = 0;
+    pl.pair = 0;
+    pl.bn = 128;
+    pl.P = M_total;
+    pl.Q = N;
+    const int64_t chunks = (row_bytes(fmt, K) + 127) / 128;
+    const bool whole = row_bytes(fmt, K) % 128 == 0;
+    pl.kc = (whole && chunks >= 2) ? 2 : 1;
+    pl.stages = stages_for(fmt, pl.bn, pl.kc);
+    pl.tilesQ = (N + pl.bn - 1) / pl.bn;
+    pl.tilesP = (M_total + 127) / 128 + G;        // each group adds at most one partial row tile
+    pl.kt = (chunks + pl.kc - 1) / pl.kc;
+    pl.tiles = pl.tilesP * pl.tilesQ;
+    pl.iters = pl.tiles * pl.kt;
+    pl.workers = pl.tiles;
+    pl.sched = 1;
+    const int64_t sms = num_sms > 0 ? num_sms : 1;
+    pl.grid = static_cast<int>(pl.tiles < sms ? pl.tiles : sms);
+    pl.kaP = sf_atoms_per_rowblock(fmt, K);
+    pl.kaQ = pl.kaP;
+    pl.partial_bytes = 0;
+    pl.counter_bytes = 4;
+    pl.groups = G;
+    pl.valid = pl.iters < (int64_t(1) << 31) && pl.tiles < (int64_t(1) << 31);
+    return pl;
+}
+
 cudaError_t launch_gemm(const GemmPlan &plan, const GemmBuffers &buf, uint64_t wait_limit_ns, int inject, int pdl,
                         cudaStream_t stream)
 {
-    if (plan.pair) {
-        if (plan.fmt == kFmtMXFP8)
-            return plan.kc == 1 ? launch_pair_t<0, 1>(plan, buf, wait_limit_ns, inject, pdl, stream)
-                                : launch_pair_t<0, 2>(plan, buf, wait_limit_ns, inject, pdl, stream);
-        return plan.kc == 1 ? launch_pair_t<1, 1>(plan, buf, wait_limit_ns, inject, pdl, stream)
-                            : launch_pair_t<1, 2>(plan, buf, wait_limit_ns, inject, pdl, stream);
-    }
-    if (plan.kc == 4)
-        return plan.fmt == kFmtMXFP8 ? dispatch_bn4<0>(plan, buf, wait_limit_ns, inject, pdl, stream)
-                                     : dispatch_bn4<1>(plan, buf, wait_limit_ns, inject, pdl, stream);
+    if (plan.pair)
+        return launch_gemm_pair(plan, buf, wait_limit_ns, inject, pdl, stream);
     if (plan.fmt == kFmtMXFP8)
-        return plan.kc == 1 ? dispatch_bn<0, 1>(plan, buf, wait_limit_ns, inject, pdl, stream)
-                            : dispatch_bn<0, 2>(plan, buf, wait_limit_ns, inject, pdl, stream);
-    return plan.kc == 1 ? dispatch_bn<1, 1>(plan, buf, wait_limit_ns, inject, pdl, stream)
-                        : dispatch_bn<1, 2>(plan, buf, wait_limit_ns, inject, pdl, stream);
+        return launch_gemm_mxfp8(plan, buf, wait_limit_ns, inject, pdl, stream);
+    if (plan.fmt == kFmtMXFP4)
+        return launch_gemm_mxfp4(plan, buf, wait_limit_ns, inject, pdl, stream);
+    return launch_gemm_bf16(plan, buf, wait_limit_ns, inject, pdl, stream);
 }
 
 }  // namespace mxg

@@ -9,14 +9,16 @@ namespace mxg {
 
 constexpr int kFmtMXFP8 = 0;
 constexpr int kFmtMXFP4 = 1;
+constexpr int kFmtBF16 = 2;     // dense BF16 operands, no scales (kind::f16 MMA)
 
 // Bytes of one operand row of K elements.
-inline int64_t row_bytes(int fmt, int64_t K) { return fmt == kFmtMXFP8 ? K : K / 2; }
+inline int64_t row_bytes(int fmt, int64_t K) { return fmt == kFmtMXFP8 ? K : (fmt == kFmtMXFP4 ? K / 2 : 2 * K); }
 
 // 512-byte scale atoms per 128-row block per 128-byte K chunk of the
 // operands (128 E4M3 elements = 4 scale blocks, or 256 E2M1 elements = 8
-// scale blocks); a pipeline stage holds 1, 2 or 4 chunks.
-inline int atoms_per_stage(int fmt) { return fmt == kFmtMXFP8 ? 1 : 2; }
+// scale blocks; BF16 operands carry none); a pipeline stage holds 1, 2 or 4
+// chunks.
+inline int atoms_per_stage(int fmt) { return fmt == kFmtMXFP8 ? 1 : (fmt == kFmtMXFP4 ? 2 : 0); }
 
 // Repacked scale layout of one operand with R rows: [ceil(R/256)*2][ka][512]
 // (row blocks of 128, padded to an even count so a 256-row tile never reads
@@ -27,6 +29,8 @@ inline int atoms_per_stage(int fmt) { return fmt == kFmtMXFP8 ? 1 : 2; }
 // expects for block-scale factors.
 inline int64_t sf_atoms_per_rowblock(int fmt, int64_t K)
 {
+    if (fmt == kFmtBF16)
+        return 0;
     const int64_t a = K / 128, s = 4 * atoms_per_stage(fmt);   // room for up to 4 chunks per stage
     return (a + s - 1) / s * s;
 }
@@ -39,9 +43,10 @@ inline int64_t sf_repacked_bytes(int fmt, int64_t R, int64_t K)
 cudaError_t launch_repack(int fmt, int64_t M, int64_t N, int64_t K, const uint8_t *sa, const uint8_t *sb,
                           uint8_t *sa_out, uint8_t *sb_out, cudaStream_t stream);
 
-// Launch the OCP MX quantiser.
+// Launch the OCP MX quantiser (FP32 input, or BF16 input when X_bf16 is set
+// and X is NULL).
 cudaError_t launch_quantize(int fmt, int64_t R, int64_t K, const float *X, uint8_t *Q, uint8_t *S,
-                            cudaStream_t stream);
+                            cudaStream_t stream, const uint16_t *X_bf16 = nullptr);
 
 // Scheduling plan of one GEMM.
 struct GemmPlan {
@@ -61,11 +66,34 @@ struct GemmPlan {
     int64_t partial_bytes = 0;  // workspace for split partials
     bool valid = true;          // false: the shape exceeds the kernel's 32-bit scheduler range
     int64_t counter_bytes = 0;
+    int64_t groups = 0;         // > 0: grouped plan (make_grouped_plan)
+    int64_t band = 0;           // CTA-pair plans: tile rows per band of the tile order (0: all)
 };
 
 // Build the plan for a shape.  sched/splits/workers as mxgemm_set_schedule.
+// allow_pair = false keeps the plan on one-CTA tiles (the paths whose
+// epilogue or tile walk only the one-CTA kernel implements).
 GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sched, int splits,
-                   int workers, int force_kc = 0);
+                   int workers, int force_kc = 0, bool allow_pair = true);
+
+// Plan of a grouped GEMM: G groups sharing N and K, group g owning rows
+// [off[g], off[g+1]) of A and C (M_total rows in all) and rows [g*N, g*N+N)
+// of B.  Whole 128 x 128 tiles, never swapped; W is an upper bound on the
+// number of tiles ((ceil(M_total/128) + G) * ceil(N/128)), the kernel skips
+// what the group sizes leave empty.
+GemmPlan make_grouped_plan(int fmt, int64_t G, int64_t M_total, int64_t N, int64_t K, int num_sms);
+
+// Fused epilogue of the one-CTA kernel: out = act(acc + bias[n]) +
+// residual[m][n], then either BF16 C or the next layer's MX operand (codes
+// plus E8M0 scales, one per 32 consecutive n of a row).
+struct Epilogue {
+    const uint16_t *bias = nullptr;       // BF16 [N] or NULL
+    const uint16_t *residual = nullptr;   // BF16 [M][N] or NULL
+    int act = 0;                          // 0 none, 1 ReLU, 2 SiLU, 3 GELU (erf form)
+    int qfmt = -1;                        // -1 BF16 C; kFmtMXFP8 / kFmtMXFP4 quantised output
+    uint8_t *Cq = nullptr;                // codes [M][row_bytes(qfmt, N)]
+    uint8_t *Cs = nullptr;                // E8M0 scales [M][N/32]
+};
 
 // Launch the GEMM kernel for `plan`.
 struct GemmBuffers {
@@ -83,6 +111,8 @@ struct GemmBuffers {
     // safe where that kernel does not write them: the scale repack, or a
     // caller's promise that B is constant.
     int early = 0;
+    Epilogue epi;
+    const int64_t *group_offsets = nullptr;   // grouped plans: device [G+1]
 };
 // pdl: launch as a programmatic dependent of the preceding kernel, letting
 // the prologue (and the operands named in buf.early) overlap its tail; every
@@ -92,5 +122,26 @@ cudaError_t launch_gemm(const GemmPlan &plan, const GemmBuffers &buf, uint64_t w
 
 // Per-(fmt, BN) kernel attribute setup; returns cudaSuccess once done.
 cudaError_t prepare_gemm_kernels();
+
+// The kernel instantiations, one translation unit per operand type
+// (gemm_mxfp8.cu, gemm_mxfp4.cu, gemm_bf16.cu: one-CTA kernel;
+// gemm_pair.cu: CTA-pair kernel): ring depth of a configuration, launch,
+// and shared-memory attribute setup.
+int stages_mxfp8(int bn, int kc);
+int stages_mxfp4(int bn, int kc);
+int stages_bf16(int bn, int kc);
+int stages_pair(int fmt, int kc);
+cudaError_t launch_gemm_mxfp8(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
+                              cudaStream_t st);
+cudaError_t launch_gemm_mxfp4(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
+                              cudaStream_t st);
+cudaError_t launch_gemm_bf16(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
+                             cudaStream_t st);
+cudaError_t launch_gemm_pair(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
+                             cudaStream_t st);
+cudaError_t prepare_mxfp8();
+cudaError_t prepare_mxfp4();
+cudaError_t prepare_bf16();
+cudaError_t prepare_pair();
 
 }  // namespace mxg

@@ -16,7 +16,10 @@ LIB_PATH = os.path.join(HERE, "libmxgemm.so")
 
 FMT_MXFP8 = 0
 FMT_MXFP4 = 1
-FMT_NAMES = {"mxfp8": FMT_MXFP8, "mxfp4": FMT_MXFP4}
+FMT_BF16 = 2
+FMT_NAMES = {"mxfp8": FMT_MXFP8, "mxfp4": FMT_MXFP4, "bf16": FMT_BF16}
+
+ACT_NONE, ACT_RELU, ACT_SILU, ACT_GELU = 0, 1, 2, 3
 
 SCHED_AUTO, SCHED_DP, SCHED_SPLITK, SCHED_STREAMK = 0, 1, 2, 3
 
@@ -50,6 +53,16 @@ SIGNATURES = {
     "mxgemm_check_device_error": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_int)]),
     "mxgemm_set_wait_limit": (ctypes.c_int, [_vp, ctypes.c_uint64]),
     "mxgemm_debug_inject": (ctypes.c_int, [_vp, ctypes.c_int]),
+    "mxgemm_run_fused": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, ctypes.c_int,
+                                        _vp, _vp, _vp]),
+    "mxgemm_run_quantized": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp,
+                                            ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, _vp]),
+    "mxgemm_quantize_bf16": (ctypes.c_int, [ctypes.c_int, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "mxgemm_run_bf16": (ctypes.c_int, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "mxgemm_run_grouped": (ctypes.c_int, [_vp, ctypes.c_int, _i64, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
+                                          _vp]),
+    "mxgemm_describe_grouped_plan": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, _i64, _i64, _i64, _i64,
+                                                    ctypes.c_char_p, ctypes.c_size_t]),
     "mxgemm_run_noalloc": (ctypes.c_int, [ctypes.c_int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "mxgemm_set_profiling": (ctypes.c_int, [_vp, ctypes.c_int]),
     "mxgemm_last_timing": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
@@ -97,7 +110,7 @@ def _check(fn: str, status: int) -> None:
 
 
 def row_bytes(fmt: int, K: int) -> int:
-    return K if fmt == FMT_MXFP8 else K // 2
+    return K if fmt == FMT_MXFP8 else (K // 2 if fmt == FMT_MXFP4 else 2 * K)
 
 
 def _stream_ptr(stream) -> int:
@@ -159,6 +172,33 @@ def run_noalloc(fmt, A, SA, B, SB, C=None, K=None, stream=None):
     _check("mxgemm_run_noalloc", mxgemm_run_noalloc(fmt, M, N, K, _ptr(A), _ptr(SA), _ptr(B), _ptr(SB), _ptr(C),
                                                     _stream_ptr(stream)))
     return C
+
+
+def mxgemm_run_fused(h, fmt, M, N, K, A, SA, B, SB, bias, act, residual, C, stream) -> int:
+    return load().mxgemm_run_fused(h, fmt, M, N, K, A, SA, B, SB, bias, act, residual, C, stream)
+
+
+def mxgemm_run_quantized(h, fmt, M, N, K, A, SA, B, SB, bias, act, residual, out_fmt, Cq, Cs, stream) -> int:
+    return load().mxgemm_run_quantized(h, fmt, M, N, K, A, SA, B, SB, bias, act, residual, out_fmt, Cq, Cs, stream)
+
+
+def mxgemm_quantize_bf16(fmt, R, K, X, Q, S, stream) -> int:
+    return load().mxgemm_quantize_bf16(fmt, R, K, X, Q, S, stream)
+
+
+def mxgemm_run_bf16(h, M, N, K, A, B, C, stream) -> int:
+    return load().mxgemm_run_bf16(h, M, N, K, A, B, C, stream)
+
+
+def mxgemm_run_grouped(h, fmt, G, M_total, N, K, offsets, A, SA, B, SB, C, stream) -> int:
+    return load().mxgemm_run_grouped(h, fmt, G, M_total, N, K, offsets, A, SA, B, SB, C, stream)
+
+
+def mxgemm_describe_grouped_plan(num_sms, fmt, G, M_total, N, K) -> str:
+    buf = ctypes.create_string_buffer(256)
+    _check("mxgemm_describe_grouped_plan",
+           load().mxgemm_describe_grouped_plan(num_sms, fmt, G, M_total, N, K, buf, 256))
+    return buf.value.decode()
 
 
 def mxgemm_quantize(fmt, R, K, X, Q, S, stream) -> int:
@@ -233,6 +273,25 @@ def quantize(fmt: int, X, stream=None, out=None):
     return Q, S
 
 
+def quantize_bf16(fmt: int, X, stream=None, out=None):
+    """OCP MX quantisation of a BF16 CUDA tensor [R][K] (the activation
+    quantiser).  Returns (codes uint8 [R][row_bytes], scales uint8 [R][K/32])."""
+    import torch
+    assert X.is_cuda and X.dtype == torch.bfloat16 and X.is_contiguous()
+    R, K = X.shape
+    if out is None:
+        Q = torch.empty((R, row_bytes(fmt, K)), dtype=torch.uint8, device=X.device)
+        S = torch.empty((R, K // 32), dtype=torch.uint8, device=X.device)
+    else:
+        Q, S = out
+    _check("mxgemm_quantize_bf16", mxgemm_quantize_bf16(fmt, R, K, _ptr(X), _ptr(Q), _ptr(S), _stream_ptr(stream)))
+    return Q, S
+
+
+def _optr(t) -> int:
+    return 0 if t is None else _ptr(t)
+
+
 class Handle:
     """Owns one ``mxgemm_handle`` (workspace, schedule) on the current device."""
 
@@ -273,6 +332,64 @@ class Handle:
             C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
         _check("mxgemm_run", mxgemm_run(self.h, fmt, M, N, K, _ptr(A), _ptr(SA), _ptr(B), _ptr(SB), _ptr(C),
                                         _stream_ptr(stream)))
+        return C
+
+    def run_fused(self, fmt, A, SA, B, SB, bias=None, act=ACT_NONE, residual=None, C=None, K=None, stream=None):
+        """C = bf16(act(A * B^T + bias) + residual) with the operations in the
+        GEMM's epilogue; bias BF16 [N] / residual BF16 [M][N] or None."""
+        import torch
+        M, N = A.shape[0], B.shape[0]
+        if K is None:
+            K = SA.shape[1] * 32
+        if C is None:
+            C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+        _check("mxgemm_run_fused", mxgemm_run_fused(self.h, fmt, M, N, K, _ptr(A), _ptr(SA), _ptr(B), _ptr(SB),
+                                                    _optr(bias), act, _optr(residual), _ptr(C), _stream_ptr(stream)))
+        return C
+
+    def run_quantized(self, fmt, A, SA, B, SB, out_fmt, bias=None, act=ACT_NONE, residual=None, out=None, K=None,
+                      stream=None):
+        """The fused-epilogue product written as the next layer's MX operand:
+        returns (codes uint8 [M][row_bytes(out_fmt, N)], scales uint8 [M][N/32])."""
+        import torch
+        M, N = A.shape[0], B.shape[0]
+        if K is None:
+            K = SA.shape[1] * 32
+        if out is None:
+            Cq = torch.empty((M, row_bytes(out_fmt, N)), dtype=torch.uint8, device=A.device)
+            Cs = torch.empty((M, N // 32), dtype=torch.uint8, device=A.device)
+        else:
+            Cq, Cs = out
+        _check("mxgemm_run_quantized",
+               mxgemm_run_quantized(self.h, fmt, M, N, K, _ptr(A), _ptr(SA), _ptr(B), _ptr(SB), _optr(bias), act,
+                                    _optr(residual), out_fmt, _ptr(Cq), _ptr(Cs), _stream_ptr(stream)))
+        return Cq, Cs
+
+    def run_bf16(self, A, B, C=None, stream=None):
+        """Dense BF16 C = A * B^T (A [M][K], B [N][K] bfloat16 CUDA tensors)."""
+        import torch
+        M, K = A.shape
+        N = B.shape[0]
+        if C is None:
+            C = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+        _check("mxgemm_run_bf16", mxgemm_run_bf16(self.h, M, N, K, _ptr(A), _ptr(B), _ptr(C), _stream_ptr(stream)))
+        return C
+
+    def run_grouped(self, fmt, offsets, A, SA, B, SB, C=None, K=None, stream=None):
+        """Grouped GEMM: offsets int64 [G+1] CUDA tensor, A [M_total][..], B
+        [G][N][..]; C[off[g]:off[g+1]] = A[off[g]:off[g+1]] * B[g]^T.  SA / SB
+        are ignored (may be None) for fmt FMT_BF16."""
+        import torch
+        G = offsets.shape[0] - 1
+        M_total = A.shape[0]
+        N = B.shape[1]
+        if K is None:
+            K = SA.shape[1] * 32 if fmt != FMT_BF16 else A.shape[1]
+        if C is None:
+            C = torch.empty((M_total, N), dtype=torch.bfloat16, device=A.device)
+        _check("mxgemm_run_grouped",
+               mxgemm_run_grouped(self.h, fmt, G, M_total, N, K, _ptr(offsets), _ptr(A), _optr(SA), _ptr(B),
+                                  _optr(SB), _ptr(C), _stream_ptr(stream)))
         return C
 
     def repack(self, fmt, M, N, K, SA, SB, stream=None):

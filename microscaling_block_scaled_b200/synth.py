@@ -65,6 +65,19 @@ WORKLOADS = {
     "mxfp4_4096x4096x14336": ("mxfp4", 4096, 4096, 14336, 3, "normal"),
 }
 
+# Workloads of the extensions beyond the MX product, by name: op and sizes.
+#  bf16:      dense BF16 GEMM (A, B drawn N(0,1) in FP32 then rounded to BF16)
+#  grouped:   grouped GEMM, `groups` rows of A per group (uneven, one empty)
+#  fused:     MX GEMM with bias + activation + residual in the epilogue
+#  quantized: MX GEMM whose epilogue writes the next layer's MX operand
+EXTRA_WORKLOADS = {
+    "bf16_64x4096x4096": dict(op="bf16", fmt="bf16", M=64, N=4096, K=4096, seed=2),
+    "mxfp8_grouped_8x4096x4096_uneven": dict(op="grouped", fmt="mxfp8", groups=(1024, 0, 512, 768, 256, 1280, 128, 128),
+                                             N=4096, K=4096, seed=5),
+    "mxfp4_32x14336x4096_bias_gelu_residual": dict(op="fused", fmt="mxfp4", M=32, N=14336, K=4096, seed=1, act=3),
+    "mxfp4_32x14336x4096_to_mxfp8": dict(op="quantized", fmt="mxfp4", M=32, N=14336, K=4096, seed=1, out_fmt=0),
+}
+
 SWEEP_M = (16, 32, 64, 128, 256, 1024, 4096, 8192)
 SWEEP_NK = ((4096, 4096), (14336, 4096), (4096, 14336), (8192, 8192), (28672, 8192))
 SWEEP_SEED = 4

@@ -22,6 +22,7 @@ _LIB = os.path.join(_HERE, "libmx_oracle.so")
 
 FMT_MXFP8 = 0
 FMT_MXFP4 = 1
+FMT_BF16 = 2
 
 _lib = None
 
@@ -67,6 +68,16 @@ def _load():
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+        lib.mxo_decode_bf16.restype = ctypes.c_double
+        lib.mxo_decode_bf16.argtypes = [ctypes.c_uint16]
+        lib.mxo_gemm_bf16.restype = None
+        lib.mxo_gemm_bf16.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+        lib.mxo_activation.restype = ctypes.c_double
+        lib.mxo_activation.argtypes = [ctypes.c_int, ctypes.c_double]
+        lib.mxo_epilogue.restype = None
+        lib.mxo_epilogue.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
         lib.mxo_num_threads.restype = ctypes.c_int
         lib.mxo_num_threads.argtypes = []
         del u8p
@@ -174,6 +185,107 @@ def gemm_points(fmt: int, K: int, A, SA, B, SB, im: np.ndarray, in_: np.ndarray,
                             n, _ptr(im), _ptr(in_), _ptr(C),
                             _ptr(ex) if ex is not None else None, _ptr(mag))
     return C, ex, mag
+
+
+ACT_NONE, ACT_RELU, ACT_SILU, ACT_GELU = 0, 1, 2, 3
+
+
+def decode_bf16(bits: int) -> float:
+    return _load().mxo_decode_bf16(bits)
+
+
+def activation(act: int, x: float) -> float:
+    return _load().mxo_activation(act, x)
+
+
+def gemm_bf16(A_bits: np.ndarray, B_bits: np.ndarray, want_exact: bool = False):
+    """C = A * B^T for dense BF16 operands given as bit patterns (uint16 [M][K],
+    [N][K]).  Returns (C_bf16_bits [M][N], exact FP64 or None, sum|a*b|)."""
+    A = np.ascontiguousarray(A_bits, dtype=np.uint16)
+    B = np.ascontiguousarray(B_bits, dtype=np.uint16)
+    M, K = A.shape
+    N = B.shape[0]
+    assert B.shape[1] == K
+    C = np.zeros((M, N), dtype=np.uint16)
+    ex = np.zeros((M, N), dtype=np.float64) if want_exact else None
+    mag = np.zeros((M, N), dtype=np.float64)
+    _load().mxo_gemm_bf16(M, N, K, _ptr(A), _ptr(B), _ptr(C), _ptr(ex) if ex is not None else None, _ptr(mag))
+    return C, ex, mag
+
+
+def epilogue(exact: np.ndarray, bias_bits=None, act: int = ACT_NONE, residual_bits=None):
+    """The fused epilogue from the unrounded product: C = bf16(act(exact +
+    bias) + residual), one rounding.  Returns (C_bits, pre) with pre =
+    exact + bias (FP64)."""
+    exact = np.ascontiguousarray(exact, dtype=np.float64)
+    M, N = exact.shape
+    b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+    r = None if residual_bits is None else np.ascontiguousarray(residual_bits, dtype=np.uint16)
+    assert b is None or b.shape == (N,)
+    assert r is None or r.shape == (M, N)
+    C = np.zeros((M, N), dtype=np.uint16)
+    pre = np.zeros((M, N), dtype=np.float64)
+    _load().mxo_epilogue(M, N, _ptr(exact), _ptr(b) if b is not None else None, act,
+                         _ptr(r) if r is not None else None, _ptr(C), _ptr(pre))
+    return C, pre
+
+
+def gemm_grouped(fmt: int, K: int, offsets, A, SA, B, SB):
+    """Grouped product: group g's rows [off[g], off[g+1]) of A times its own
+    B[g] (one plain product per group; empty groups contribute nothing).
+    fmt FMT_BF16 takes BF16 bit patterns and ignores SA / SB.  Returns
+    (C_bits [M_total][N], sum|a*b| [M_total][N])."""
+    off = [int(x) for x in offsets]
+    G = len(off) - 1
+    M_total, N = A.shape[0], B.shape[1]
+    C = np.zeros((M_total, N), dtype=np.uint16)
+    mag = np.zeros((M_total, N), dtype=np.float64)
+    for g in range(G):
+        r0, r1 = off[g], off[g + 1]
+        if r1 <= r0:
+            continue
+        if fmt == FMT_BF16:
+            c, _, m = gemm_bf16(A[r0:r1], B[g])
+        else:
+            c, _, m = gemm(fmt, K, A[r0:r1], SA[r0:r1], B[g], SB[g])
+        C[r0:r1] = c
+        mag[r0:r1] = m
+    return C, mag
+
+
+def tolerance_fused(ref_bits: np.ndarray, abssum: np.ndarray, pre: np.ndarray, residual_bits=None) -> np.ndarray:
+    """Per-element bound for the fused epilogue: 1 BF16 ulp of the result +
+    the product's bound 2^-18 * sum|a b| carried through the activation (whose
+    slope is at most 1.13 for GELU, 1.1 for SiLU, 1 for ReLU; 1.25 here) +
+    2^-19 * (|pre| + |residual|) for the FP32 rounding of the bias add, the
+    activation's evaluation and the residual add (each a few FP32 ulps)."""
+    res = 0.0 if residual_bits is None else np.abs(bf16_bits_to_f64(residual_bits))
+    with np.errstate(invalid="ignore"):
+        extra = (2.0 ** -19) * (np.abs(pre) + res)
+    extra = np.where(np.isfinite(extra), extra, 0.0)
+    return bf16_ulp(ref_bits) + 1.25 * (2.0 ** -18) * abssum + extra
+
+
+def compare_with_tolerance(got_bits: np.ndarray, ref_bits: np.ndarray, tol: np.ndarray):
+    """compare() with an explicit per-element tolerance."""
+    got = bf16_bits_to_f64(got_bits)
+    ref = bf16_bits_to_f64(ref_bits)
+    nan_g, nan_r = np.isnan(got), np.isnan(ref)
+    inf_g, inf_r = np.isinf(got), np.isinf(ref)
+    pattern_ok = bool(np.array_equal(nan_g, nan_r)) and bool(
+        np.array_equal(inf_g & (got > 0), inf_r & (ref > 0))) and bool(
+        np.array_equal(inf_g & (got < 0), inf_r & (ref < 0)))
+    fin = ~(nan_r | inf_r) & ~(nan_g | inf_g)
+    with np.errstate(invalid="ignore"):
+        err = np.abs(got - ref)
+    bad = fin & ~(err <= tol)
+    rep = {"n": int(got.size), "pattern_ok": pattern_ok, "n_bad": int(bad.sum()),
+           "max_err_over_tol": float((err[fin] / tol[fin]).max()) if fin.any() else 0.0}
+    if bad.any():
+        idx = np.argwhere(bad)[:5]
+        rep["first_bad"] = [(tuple(int(x) for x in i), float(got[tuple(i)]), float(ref[tuple(i)]),
+                             float(tol[tuple(i)])) for i in idx]
+    return pattern_ok and not bad.any(), rep
 
 
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:

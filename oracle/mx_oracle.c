@@ -334,6 +334,88 @@ void mxo_gemm_points(int fmt, int64_t M, int64_t N, int64_t K,
     }
 }
 
+/* --------------------------------------------------------- dense BF16 GEMM */
+
+/* A BF16 value from its bit pattern: the upper half of a binary32, widened
+ * exactly to binary64.                                                     */
+double mxo_decode_bf16(uint16_t bits)
+{
+    uint32_t w = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &w, sizeof f);
+    return (double)f;
+}
+
+/* C = A * B^T for dense BF16 operands (the dense-GEMM comparison suite of
+ * the 5ulink.com page, table 内核级成绩): A [M][K], B [N][K] BF16 bits, C
+ * BF16 bits [M][N].  Every product of two BF16 values is exact in binary64;
+ * the products are summed in FP64 in k order and the sum is rounded to BF16
+ * once.  `exact` / `abssum` as in mxo_gemm (may be NULL).                   */
+void mxo_gemm_bf16(int64_t M, int64_t N, int64_t K,
+                   const uint16_t *A, const uint16_t *B,
+                   uint16_t *C, double *exact, double *abssum)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double p = mxo_decode_bf16(A[m * K + k]) * mxo_decode_bf16(B[n * K + k]);
+                acc += p;
+                mag += fabs(p);
+            }
+            C[m * N + n] = mxo_bf16_rne(acc);
+            if (exact) exact[m * N + n] = acc;
+            if (abssum) abssum[m * N + n] = mag;
+        }
+    }
+}
+
+/* ------------------------------------------------------- fused epilogue */
+
+/* The activations of the fused epilogue, in binary64, from their
+ * definitions: ReLU max(x, 0) (NaN stays NaN), SiLU x * sigmoid(x) =
+ * x / (1 + e^-x), GELU x * Phi(x) with the standard normal CDF
+ * Phi(x) = erfc(-x / sqrt(2)) / 2.                                          */
+double mxo_activation(int act, double x)
+{
+    switch (act) {
+    case 1:
+        return x < 0.0 ? 0.0 : x;
+    case 2:
+        return x / (1.0 + exp(-x));
+    case 3:
+        return 0.5 * x * erfc(-x / sqrt(2.0));
+    default:
+        return x;
+    }
+}
+
+/* Epilogue fusion (the roadmap's "GEMM 尾部融合" on the 5ulink.com page,
+ * section 怎么用起来): from the unrounded product `exact` [M][N] (binary64,
+ * as mxo_gemm returns it), out = act(exact + bias[n]) + residual[m][n] in
+ * binary64, rounded to BF16 once.  bias: BF16 bits [N] or NULL; residual:
+ * BF16 bits [M][N] or NULL.  `pre` (may be NULL) receives exact + bias.    */
+void mxo_epilogue(int64_t M, int64_t N, const double *exact,
+                  const uint16_t *bias, int act, const uint16_t *residual,
+                  uint16_t *C, double *pre)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double v = exact[m * N + n];
+            if (bias)
+                v += mxo_decode_bf16(bias[n]);
+            if (pre)
+                pre[m * N + n] = v;
+            v = mxo_activation(act, v);
+            if (residual)
+                v += mxo_decode_bf16(residual[m * N + n]);
+            C[m * N + n] = mxo_bf16_rne(v);
+        }
+    }
+}
+
 /* Number of OpenMP threads the oracle runs with (1 without OpenMP).        */
 int mxo_num_threads(void)
 {

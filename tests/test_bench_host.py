@@ -67,4 +67,4 @@ def test_recorded_traffic_only_for_the_captured_source(tmp_path, monkeypatch):
 def test_kernel_hash_covers_the_kernel_sources():
     h = bench.kernel_hash()
     assert len(h) == 16 and int(h, 16) >= 0
-    assert any(p.endswith("gemm.cu") for p in bench.KERNEL_SOURCES)
+    assert any(p.endswith("gemm_kernel.cuh") for p in bench.KERNEL_SOURCES)

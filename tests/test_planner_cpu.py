@@ -148,7 +148,8 @@ def test_describe_plan_for_rejects_bad_arguments():
     assert lib.mxgemm_describe_plan_for(1, F8, 32, 256, 512, buf, 256) == mxgemm.ERR_INVALID_ARG
     assert lib.mxgemm_describe_plan_for(148, F8, 32, 256, 500, buf, 256) == mxgemm.ERR_INVALID_ARG
     assert lib.mxgemm_describe_plan_for(148, F8, 0, 256, 512, buf, 256) == mxgemm.ERR_INVALID_ARG
-    assert lib.mxgemm_describe_plan_for(148, 2, 32, 256, 512, buf, 256) == mxgemm.ERR_INVALID_ARG
+    assert lib.mxgemm_describe_plan_for(148, 3, 32, 256, 512, buf, 256) == mxgemm.ERR_INVALID_ARG
+    assert lib.mxgemm_describe_plan_for(148, mxgemm.FMT_BF16, 32, 256, 100, buf, 256) == mxgemm.ERR_INVALID_ARG
     assert lib.mxgemm_describe_plan_for(148, F8, 32, 256, 512, buf, 0) == mxgemm.ERR_INVALID_ARG
     assert lib.mxgemm_describe_plan_for(148, F8, 32, 256, 512, None, 256) == mxgemm.ERR_INVALID_ARG
     # a short buffer is filled and NUL-terminated

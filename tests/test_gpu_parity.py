@@ -300,6 +300,44 @@ def test_gemm_integer_exact(fmt, path):
     assert np.array_equal(got, ref)        # exact FP32 sums: the one BF16 rounding is the oracle's
 
 
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("path", list(PATHS))
+def test_gemm_fp32_subnormal_results(fmt, path):
+    """Results, partial sums and single products in the FP32-subnormal range
+    (below 2^-126): the tensor pipe's FP32 accumulation keeps them (no flush
+    to zero), so they match the oracle exactly and fall under the ordinary
+    pass rule."""
+    M, N, K = _shape(path, (64, 256, 256))
+    enc = oracle.encode_e4m3 if fmt == F8 else oracle.encode_e2m1
+    one, neg1 = enc(1.0), enc(-1.0)
+    big = enc(1.125) if fmt == F8 else enc(1.5)
+    tiny = 0x01                                     # smallest subnormal code: 2^-9 (E4M3), 0.5 (E2M1)
+    A = np.zeros((M, K), np.uint8)
+    B = np.zeros((N, K), np.uint8)
+    SA = np.full((M, K // 32), 62, np.uint8)
+    SB = np.full((N, K // 32), 62, np.uint8)
+    B[:, 0] = one
+    B[:, 32] = one
+    B[:, 64] = tiny
+    A[0, 0] = one                                   # one product of 2^-130
+    A[1, 0], A[1, 32] = big, neg1                   # (1.125 - 1) 2^-125 or (1.5 - 1) 2^-126: a subnormal difference
+    SA[1, :] = 67 if fmt == F8 else 66
+    A[2, 64] = tiny                                 # smallest elements: 2^-18 * 2^-112 / 0.25 * 2^-130
+    SA[2, :] = 80 if fmt == F8 else 62
+    A[3, 0], A[3, K - 32] = one, one                # a subnormal part added to a normal one
+    SA[3, K // 32 - 1] = 167
+    B[:, K - 32] = one
+    A[4, 0], A[4, 32], A[4, 64] = one, one, one     # subnormal products summed
+    if fmt == F4:
+        A = (A[:, 0::2] | (A[:, 1::2] << 4)).astype(np.uint8)
+        B = (B[:, 0::2] | (B[:, 1::2] << 4)).astype(np.uint8)
+    got, ref, mag = _codes_case(fmt, A, SA, B, SB, K, path)
+    assert_parity(got, ref, mag, "subnormal results (%s)" % path)
+    rv = oracle.bf16_bits_to_f64(ref)
+    assert (np.abs(rv[[0, 1, 2, 4], 0]) < 2.0 ** -126).all() and (rv[[0, 1, 2, 4], 0] != 0).all()
+    assert np.array_equal(got[:5], ref[:5])
+
+
 # -------------------------------------------------------- entry points
 
 @pytest.mark.parametrize("fmt,M,N,K", [(F4, 48, 512, 1024), (F4, 32, 512, 1024), (F8, 16, 384, 512)],

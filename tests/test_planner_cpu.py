@@ -85,7 +85,8 @@ def test_pair_grid_on_a_small_device():
     (F8, 128, 128, 1),      # one 128-byte chunk
     (F8, 128, 256, 2),
     (F4, 128, 512, 2),
-    (F8, 64, 512, 4),       # 64-column decode tiles take four chunks when rows have them
+    (F8, 64, 512, 4),       # 64-column MXFP8 decode tiles take four chunks when rows have them
+    (F4, 64, 4096, 2),      # ... MXFP4 ones two
     (F8, 64, 384, 2),       # ... and two with fewer than four
     (F4, 32, 4096, 2),
 ])

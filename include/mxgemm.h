@@ -283,10 +283,13 @@ MXGEMM_API int mxgemm_set_kchunks(mxgemm_handle h, int kc);
 /* Describe the plan mxgemm_gemm would use for a shape: writes up to `cap`
  * bytes of a NUL-terminated text such as
  * "fmt=1 swap=1 pair=0 BN=32 kc=2 stages=5 tiles=112 kt=8 workers=112
- * grid=112 sched=dp partial_bytes=0 scales=fused".  The last field says how
+ * grid=112 sched=dp partial_bytes=0 scales=fused".  "scales" says how
  * mxgemm_run treats the scales for this shape: "fused" (the GEMM converts
  * the row-major scales itself, one launch) or "repack" (scale repack, then
- * the GEMM). */
+ * the GEMM).  sched is dp (whole tiles), splitk, streamk, or for CTA-pair
+ * plans dptail: whole tiles, except that the tiles of the last, partial wave
+ * (from tail_first on, fields appended) are split into tail_split K ranges
+ * over the pairs that wave would leave idle. */
 MXGEMM_API int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
                          char *buf, size_t cap);
 

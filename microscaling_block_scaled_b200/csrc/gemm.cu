@@ -98,13 +98,34 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
             if (atoi(e) > 0)
                 pl.band = atoi(e) < pl.tilesP ? atoi(e) : pl.tilesP;
         const int64_t pairs = (num_sms > 0 ? num_sms : 2) / 2;
+        const int64_t npairs = pl.tiles < pairs ? pl.tiles : pairs;
         pl.workers = pl.tiles;
-        pl.grid = static_cast<int>(2 * (pl.tiles < pairs ? pl.tiles : pairs));
+        pl.grid = static_cast<int>(2 * npairs);
         pl.sched = 1;
         pl.kaP = sf_atoms_per_rowblock(fmt, K);
         pl.kaQ = pl.kaP;
         pl.partial_bytes = 0;
         pl.counter_bytes = 4;
+        pl.tail_first = pl.tiles;
+        pl.tail_split = 1;
+        // Automatic schedule: when the last wave of whole tiles would leave
+        // pairs idle, split each of its tiles into up to four K ranges over
+        // them; the split tiles' FP32 partials (128 KB per CTA and range)
+        // are summed by the range that finishes last.
+        if (sched == 0) {
+            const int64_t full = pl.tiles / npairs * npairs, rest = pl.tiles - full;
+            int64_t sp = rest > 0 ? npairs / rest : 1;
+            sp = sp > 4 ? 4 : sp;
+            sp = sp > pl.kt ? pl.kt : sp;
+            if (rest > 0 && sp >= 2) {
+                pl.tail_first = full;
+                pl.tail_split = sp;
+                pl.workers = full + rest * sp;
+                pl.sched = 4;
+                pl.partial_bytes = rest * sp * 2 * 128 * 256 * 4;
+                pl.counter_bytes = rest * 2 * 4;
+            }
+        }
         pl.valid = pl.iters < (int64_t(1) << 31);
         return pl;
     }

@@ -220,6 +220,9 @@ struct KParams {
     uint32_t groups;
     uint32_t tilesQ;       // column tiles (grouped: per group), ceil(N / BN)
     uint32_t band;         // CTA-pair plans: tile rows per band of the tile order
+    // CTA-pair plans: tiles from tail_first on (the last, partial wave) are
+    // split into tail_split K ranges, each its own work unit (1: no split)
+    uint32_t tail_first, tail_split;
 };
 
 // Where one output tile lives: rows [prow, prow+128) of the row operand
@@ -1316,6 +1319,36 @@ __device__ __forceinline__ void pair_tile(uint32_t t, uint32_t tilesP, uint32_t 
     tp = b * band + (w - tq * rows);
 }
 
+// Work unit w of a pair plan: whole tiles first; then, for the tiles of the
+// last, partial wave, `split` units per tile, each a contiguous range of its
+// K iterations.  A split tile's units write FP32 partials to slots
+// [slot0, slot0 + nseg) and the last to finish sums them in slot order.
+struct PairUnit {
+    uint32_t tile, kb, ke, seg, nseg, slot0;
+};
+
+__device__ __forceinline__ PairUnit pair_unit(uint32_t w, uint32_t first, uint32_t split, uint32_t KT)
+{
+    PairUnit u;
+    if (w < first || split <= 1) {
+        u.tile = w;
+        u.kb = 0;
+        u.ke = KT;
+        u.seg = 0;
+        u.nseg = 1;
+        u.slot0 = 0;
+    } else {
+        const uint32_t v = w - first, ti = v / split;
+        u.tile = first + ti;
+        u.seg = v - ti * split;
+        u.kb = u.seg * KT / split;
+        u.ke = (u.seg + 1) * KT / split;
+        u.nseg = split;
+        u.slot0 = ti * split;
+    }
+    return u;
+}
+
 template <int FMT, int KC>
 __global__ void __launch_bounds__(256, 1)
     mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
@@ -1339,6 +1372,7 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t drain_bar = bar0 + 8u * (3 * S + 2);
     volatile uint32_t *s_tmem = reinterpret_cast<volatile uint32_t *>(smem + C_::kOffMisc);
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C_::kOffMisc + 4);
+    volatile int *s_last = reinterpret_cast<volatile int *>(smem + C_::kOffMisc + 8);
 
     if (blockDim.x != C_::kThreads) {     // uniform over the cluster: both CTAs return
         if (threadIdx.x == 0)
@@ -1350,8 +1384,8 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
     const uint32_t pair = blockIdx.x / 2, npairs = gridDim.x / 2;
-    const uint32_t tiles = kp.workers, tilesP = kp.tilesP, tilesQ = kp.tilesQ, KT = kp.kt;
-    const uint32_t band = kp.band;
+    const uint32_t units = kp.workers, tilesP = kp.tilesP, tilesQ = kp.tilesQ, KT = kp.kt;
+    const uint32_t band = kp.band, tail_first = kp.tail_first, tail_split = kp.tail_split;
 
     if (threadIdx.x == 0) {
         tma_prefetch_desc(&tmP);
@@ -1404,13 +1438,14 @@ __global__ void __launch_bounds__(256, 1)
             int s = 0;
             uint32_t ph = 0;
             bool first = true;
-            for (uint32_t tile = pair; tile < tiles; tile += npairs) {
+            for (uint32_t w = pair; w < units; w += npairs) {
+                const PairUnit un = pair_unit(w, tail_first, tail_split, KT);
                 uint32_t tp, tq;
-                pair_tile(tile, tilesP, tilesQ, band, tp, tq);
+                pair_tile(un.tile, tilesP, tilesQ, band, tp, tq);
                 const int32_t row = static_cast<int32_t>((sideA ? tp : tq) * 256 + rank * 128);
                 const int32_t sf_rb = sideA ? static_cast<int32_t>(tp * 2 + rank) : static_cast<int32_t>(tq * 2);
                 bool ok = true;
-                for (uint32_t k = 0; k < KT; ++k) {
+                for (uint32_t k = un.kb; k < un.ke; ++k) {
                     if (!mbar_wait_parked(empty_bar(s), ph ^ 1u, s_abort, kp.limit_ns)) {
                         record_error(kp.error, kErrProducerEmpty, s_abort);
                         ok = false;
@@ -1472,7 +1507,8 @@ __global__ void __launch_bounds__(256, 1)
         uint32_t ph = 0;
         uint32_t acc_ph = 0;
         bool ok = true;
-        for (uint32_t tile = pair; tile < tiles && ok; tile += npairs) {
+        for (uint32_t w = pair; w < units && ok; w += npairs) {
+            const PairUnit un = pair_unit(w, tail_first, tail_split, KT);
             int good = 1;
             if (lane == 0)
                 good = mbar_wait_cluster_bounded(acce_bar, acc_ph ^ 1u, s_abort, kp.limit_ns);
@@ -1483,7 +1519,7 @@ __global__ void __launch_bounds__(256, 1)
                 break;
             }
             tc_fence_after();
-            for (uint32_t k = 0; k < KT; ++k) {
+            for (uint32_t k = un.kb; k < un.ke; ++k) {
                 good = 1;
                 if (lane == 0)
                     // the MMA warp alone spins: it feeds the tensor pipe
@@ -1508,7 +1544,7 @@ __global__ void __launch_bounds__(256, 1)
                             const int atom = FMT == kFmtMXFP8 ? c : 2 * c + j / 2;
                             const uint32_t sf_id = FMT == kFmtMXFP8 ? j : 2 * (j % 2);
                             const uint32_t idesc = kIdesc | (sf_id << 4) | (sf_id << 29);
-                            const uint32_t acc_flag = (k > 0 || c > 0 || j > 0) ? 1u : 0u;
+                            const uint32_t acc_flag = (k > un.kb || c > 0 || j > 0) ? 1u : 0u;
                             const uint64_t koff = static_cast<uint64_t>(j * 32) >> 4;
                             if (FMT == kFmtMXFP8)
                                 mma_mxf8f6f4_pair(tmem, adesc + koff, bdesc + koff, idesc, t_sfa + 4 * atom,
@@ -1552,8 +1588,9 @@ __global__ void __launch_bounds__(256, 1)
         int s = 0;
         uint32_t ph = 0;
         bool ok = true;
-        for (uint32_t tile = pair; tile < tiles && ok; tile += npairs) {
-            for (uint32_t k = 0; k < KT; ++k) {
+        for (uint32_t w = pair; w < units && ok; w += npairs) {
+            const PairUnit un = pair_unit(w, tail_first, tail_split, KT);
+            for (uint32_t k = un.kb; k < un.ke; ++k) {
                 int good = 1;
                 if (lane == 0)
                     good = mbar_wait_cluster_parked(full_bar(s), ph, s_abort, kp.limit_ns);
@@ -1603,9 +1640,30 @@ __global__ void __launch_bounds__(256, 1)
         const int etid = threadIdx.x - 64;
         uint32_t acc_ph = 0;
         uint32_t out_chunks = 0;
-        for (uint32_t tile = pair; tile < tiles; tile += npairs) {
+        // one CW-column chunk of BF16 pairs to C through shared memory and a TMA store
+        auto store_chunk = [&](const uint32_t *pk, uint32_t tp, uint32_t tq, int c) {
+            const int b = static_cast<int>(out_chunks & 1u);
+            uint8_t *buf = smem + C_::kOffOut + b * C_::kOutBytes;
+            if (etid == 0)
+                bulk_wait_group_read<1>();
+            named_bar_sync(1, 128);
+            uint4 *dst = reinterpret_cast<uint4 *>(buf + row * CW * 2);
+#pragma unroll
+            for (int j = 0; j < CW / 8; ++j)
+                dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (etid == 0) {
+                tma_store_2d(&tmC, smem_u32(buf), static_cast<int32_t>(tq * 256 + c),
+                             static_cast<int32_t>(tp * 256 + rank * 128));
+                bulk_commit_group();
+            }
+            ++out_chunks;
+        };
+        for (uint32_t w = pair; w < units; w += npairs) {
+            const PairUnit un = pair_unit(w, tail_first, tail_split, KT);
             uint32_t tp, tq;
-            pair_tile(tile, tilesP, tilesQ, band, tp, tq);
+            pair_tile(un.tile, tilesP, tilesQ, band, tp, tq);
             int good = 1;
             if (lane == 0)
                 good = mbar_wait_parked(accf_bar, acc_ph, s_abort, kp.limit_ns);
@@ -1616,48 +1674,94 @@ __global__ void __launch_bounds__(256, 1)
                 break;
             tc_fence_after();
             const uint32_t t_acc = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-            // Drain the whole accumulator row into registers (BF16 pairs), 64
-            // columns per TMEM load, and hand the accumulator back to the MMA
-            // warp before any store, so the next tile's MMAs overlap this
-            // tile's output traffic.
-            uint32_t packed[128];
+            if (un.nseg == 1) {
+                // Drain the whole accumulator row into registers (BF16 pairs), 64
+                // columns per TMEM load, and hand the accumulator back to the MMA
+                // warp before any store, so the next tile's MMAs overlap this
+                // tile's output traffic.
+                uint32_t packed[128];
 #pragma unroll
-            for (int c = 0; c < 256; c += 64) {
-                uint32_t r[64];
-                tmem_ld_32x32b_x64(t_acc + c, r);
-                tmem_ld_wait();
+                for (int c = 0; c < 256; c += 64) {
+                    uint32_t r[64];
+                    tmem_ld_32x32b_x64(t_acc + c, r);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    packed[c / 2 + j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if (leader)
-                    mbar_arrive(acce_bar);
-                else
-                    mbar_arrive_remote(acce_bar, 0);
-            }
+                    for (int j = 0; j < 32; ++j)
+                        packed[c / 2 + j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (leader)
+                        mbar_arrive(acce_bar);
+                    else
+                        mbar_arrive_remote(acce_bar, 0);
+                }
 #pragma unroll
-            for (int c = 0; c < 256; c += CW) {
-                const int b = static_cast<int>(out_chunks & 1u);
-                uint8_t *buf = smem + C_::kOffOut + b * C_::kOutBytes;
-                if (etid == 0)
-                    bulk_wait_group_read<1>();
-                named_bar_sync(1, 128);
-                uint4 *dst = reinterpret_cast<uint4 *>(buf + row * CW * 2);
+                for (int c = 0; c < 256; c += CW)
+                    store_chunk(packed + c / 2, tp, tq, c);
+            } else {
+                // A K range of a split tile: its FP32 partial (this CTA's 128
+                // rows) goes to its slot; the unit that completes the tile
+                // sums all slots in order and stores C.
+                float *mine = kp.partials + ((static_cast<int64_t>(un.slot0 + un.seg) * 2 + rank) * 128 + row) * 256;
+#pragma unroll 1
+                for (int c = 0; c < 256; c += 64) {
+                    uint32_t r[64];
+                    tmem_ld_32x32b_x64(t_acc + c, r);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < CW / 8; ++j)
-                    dst[j] = make_uint4(packed[c / 2 + 4 * j], packed[c / 2 + 4 * j + 1], packed[c / 2 + 4 * j + 2],
-                                        packed[c / 2 + 4 * j + 3]);
-                fence_proxy_async_smem();
+                    for (int j = 0; j < 16; ++j)
+                        reinterpret_cast<float4 *>(mine + c)[j] =
+                            make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (leader)
+                        mbar_arrive(acce_bar);
+                    else
+                        mbar_arrive_remote(acce_bar, 0);
+                }
+                __threadfence();
                 named_bar_sync(1, 128);
                 if (etid == 0) {
-                    tma_store_2d(&tmC, smem_u32(buf), static_cast<int32_t>(tq * 256 + c),
-                                 static_cast<int32_t>(tp * 256 + rank * 128));
-                    bulk_commit_group();
+                    uint32_t *ctr = kp.counters + (un.tile - tail_first) * 2 + rank;
+                    const uint32_t old = atomicAdd(ctr, 1u);
+                    const int last = (old == un.nseg - 1) ? 1 : 0;
+                    if (last)
+                        *ctr = 0u;          // counters stay zero between launches
+                    *s_last = last;
                 }
-                ++out_chunks;
+                named_bar_sync(1, 128);
+                if (*s_last) {
+                    __threadfence();
+#pragma unroll 1
+                    for (int c = 0; c < 256; c += CW) {
+                        float v[CW];
+#pragma unroll
+                        for (int j = 0; j < CW; ++j)
+                            v[j] = 0.0f;
+                        for (uint32_t g = 0; g < un.nseg; ++g) {
+                            const float4 *src = reinterpret_cast<const float4 *>(
+                                kp.partials + ((static_cast<int64_t>(un.slot0 + g) * 2 + rank) * 128 + row) * 256 + c);
+#pragma unroll
+                            for (int j = 0; j < CW / 4; ++j) {
+                                const float4 x = __ldcg(src + j);
+                                v[4 * j + 0] += x.x;
+                                v[4 * j + 1] += x.y;
+                                v[4 * j + 2] += x.z;
+                                v[4 * j + 3] += x.w;
+                            }
+                        }
+                        uint32_t pk[CW / 2];
+#pragma unroll
+                        for (int j = 0; j < CW / 2; ++j)
+                            pk[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                        store_chunk(pk, tp, tq, c);
+                    }
+                }
             }
             acc_ph ^= 1u;
         }
@@ -1857,6 +1961,8 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     kp.groups = static_cast<uint32_t>(pl.groups);
     kp.tilesQ = static_cast<uint32_t>(pl.tilesQ);
     kp.band = 0;
+    kp.tail_first = 0;
+    kp.tail_split = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
     cfg.blockDim = dim3(C_::kThreads);
@@ -1907,8 +2013,8 @@ cudaError_t launch_pair_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t lim
         return cudaErrorInvalidValue;
     KParams kp;
     kp.C = reinterpret_cast<__nv_bfloat16 *>(b.C);
-    kp.partials = nullptr;
-    kp.counters = nullptr;
+    kp.partials = b.partials;
+    kp.counters = b.counters;
     kp.error = b.error;
     kp.P = pl.M;
     kp.Q = pl.N;
@@ -1916,7 +2022,7 @@ cudaError_t launch_pair_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t lim
     kp.tilesP = static_cast<uint32_t>(pl.tilesP);
     kp.kt = static_cast<uint32_t>(pl.kt);
     kp.iters = static_cast<uint32_t>(pl.iters);
-    kp.workers = static_cast<uint32_t>(pl.tiles);
+    kp.workers = static_cast<uint32_t>(pl.workers);
     kp.dp = 1;
     kp.limit_ns = limit_ns;
     kp.swap = 0;
@@ -1938,6 +2044,8 @@ cudaError_t launch_pair_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t lim
     kp.groups = 0;
     kp.tilesQ = static_cast<uint32_t>(pl.tilesQ);
     kp.band = static_cast<uint32_t>(pl.band > 0 ? pl.band : pl.tilesP);
+    kp.tail_first = static_cast<uint32_t>(pl.tail_first);
+    kp.tail_split = static_cast<uint32_t>(pl.tail_split > 1 ? pl.tail_split : 1);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
     cfg.blockDim = dim3(C_::kThreads);

@@ -112,6 +112,18 @@ def test_gemm_k_chunks_per_stage(fmt, kc, M, N, K):
 
 
 @pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("M,N,K", [(1024, 5120, 1024), (1000, 5000, 2048), (2048, 4864, 1024)])
+def test_gemm_cta_pair_last_wave_split(fmt, M, N, K):
+    """CTA-pair plans whose last wave of whole tiles would leave pairs idle
+    split that wave's tiles into K ranges; the FP32 partials are summed by
+    the range that finishes last."""
+    _, plan = rows_case(fmt, M, N, K, seed=M + K)
+    assert "pair=1" in plan and "sched=dptail" in plan, plan
+    # the same shape again: the tile counters were left at zero
+    _, plan = rows_case(fmt, M, N, K, seed=M + K + 1, n_rows=16)
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
 @pytest.mark.parametrize("kc", [0, 1, 2])
 @pytest.mark.parametrize("M,N,K", [(512, 8192, 256), (640, 8448, 384), (1000, 4104, 512)])
 def test_gemm_cta_pair_tiles(fmt, kc, M, N, K):
@@ -139,6 +151,7 @@ PATHS = {
     # name: (shape override or None, schedule or None)
     "auto": (None, None),
     "pair": ((512, 8192, 384), None),
+    "pair-tail": ((1024, 5120, 1024), None),      # 80 pair tiles: the last wave's 6 tiles split in K
     "splitk3": ((200, 640, 2048), (mxgemm.SCHED_SPLITK, 3, 0)),
     "splitk8": ((200, 640, 2048), (mxgemm.SCHED_SPLITK, 8, 0)),
     "streamk148": ((200, 640, 2048), (mxgemm.SCHED_STREAMK, 1, 148)),
@@ -174,6 +187,8 @@ def _codes_case(fmt, A, SA, B, SB, K, path="auto"):
     # the path the case is meant to exercise is the one that ran
     if path == "pair":
         assert "pair=1" in plan, plan
+    elif path == "pair-tail":
+        assert "pair=1" in plan and "sched=dptail" in plan, plan
     elif path.startswith("split") or path.startswith("swap-split"):
         assert "sched=splitk" in plan and "pair=0" in plan, plan
     elif "streamk" in path:

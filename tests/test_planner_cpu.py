@@ -70,9 +70,28 @@ def test_cta_pairs_for_large_M(M, N, pair):
     p = plan(F8, M, N, 1024)
     assert p["pair"] == pair
     if pair:
-        assert p["BN"] == 256 and p["scales"] == "repack" and p["sched"] == "dp"
+        assert p["BN"] == 256 and p["scales"] == "repack" and p["sched"] in ("dp", "dptail")
         assert p["tiles"] == cdiv(M, 256) * cdiv(N, 256)
         assert p["grid"] == 2 * min(p["tiles"], B200_SMS // 2)
+
+
+@pytest.mark.parametrize("M,N,full,split", [
+    (4096, 4096, 222, 2),      # 256 tiles on 74 pairs: 3 whole waves, 34 tiles split in two
+    (2048, 28672, 888, 4),     # 896 tiles: 12 waves, 8 tiles split in four (at most four)
+    (8192, 8192, None, 1),     # 1024 tiles: the last wave has 62 of 74 pairs busy: whole tiles
+    (512, 8192, None, 1),      # 64 tiles, one wave
+])
+def test_pair_plans_split_the_last_wave(M, N, full, split):
+    p = plan(F8, M, N, 8192)
+    tiles, pairs = p["tiles"], B200_SMS // 2
+    if split == 1:
+        assert p["sched"] == "dp" and p["workers"] == tiles and p["partial_bytes"] == 0
+        return
+    rest = tiles - full
+    assert p["sched"] == "dptail" and p["tail_first"] == full and p["tail_split"] == split
+    assert full == tiles // pairs * pairs and rest * split <= pairs
+    assert p["workers"] == full + rest * split
+    assert p["partial_bytes"] == rest * split * 2 * 128 * 256 * 4
 
 
 def test_pair_grid_on_a_small_device():
@@ -130,6 +149,12 @@ def test_plan_invariants_over_random_shapes():
         if p["pair"]:
             assert p["tiles"] == cdiv(M, 256) * cdiv(N, 256) and p["grid"] % 2 == 0
             assert p["scales"] == "repack"
+            if p["sched"] == "dptail":
+                rest = p["tiles"] - p["tail_first"]
+                assert 0 < rest and p["workers"] == p["tail_first"] + rest * p["tail_split"]
+                assert rest * p["tail_split"] <= p["grid"] // 2 and 2 <= p["tail_split"] <= 4
+                assert p["partial_bytes"] == rest * p["tail_split"] * 2 * 128 * 256 * 4
+                continue
         else:
             P, Q = (N, M) if p["swap"] else (M, N)
             assert p["swap"] == (1 if M <= 64 else 0)

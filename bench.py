@@ -481,6 +481,7 @@ def run_extra(args, w):
     st_err, code = h.check_device_error()
     if st_err != mxgemm.OK:
         raise SystemExit("device error word set: %d" % code)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     if rank == 0:
         line = {
             "metric": METRIC, "value": job_tflops(fl, world, args.steps, ms), "unit": "TFLOPS", "n_gpus": world,
@@ -489,9 +490,9 @@ def run_extra(args, w):
             "config": dict(base_config(args.workload), **{
                 "l2": "inputs rotate over %d copies (%.1f MB each)" % (nsets, abytes / 1e6),
                 "timing": "CUDA graph of K steps, CUDA events on the launch stream", "step_us": us,
-                "plan": h.describe(0 if op == "bf16" else fmt, M, N, K) if op != "grouped" else
-                mxgemm.mxgemm_describe_grouped_plan(torch.cuda.get_device_properties(dev).multi_processor_count,
-                                                    fmt, len(w["groups"]), M, N, K)}),
+                "plan": (mxgemm.mxgemm_describe_grouped_plan(sms, fmt, len(w["groups"]), M, N, K) if op == "grouped"
+                         else mxgemm.mxgemm_describe_plan_for(sms, fmt, M, N, K) if op == "bf16"
+                         else h.describe(fmt, M, N, K))}),
             "clocks": clocks, "roofline": roof, "cpu_baseline": None,
             "e2e": {"value": job_tflops(fl, world, args.e2e_steps, e2e_ms), "unit": "TFLOPS",
                     "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hx),
@@ -601,7 +602,11 @@ def run_ours(args):
     torch.cuda.synchronize()
     g_gemm, s_gemm = capture(gemm_only, args.steps)
     g_gemm.replay()
-    ms_gemm = timed(g_gemm, s_gemm)
+    with ClockSampler(local) as clk_k:
+        clk_k.active = True
+        ms_gemm = timed(g_gemm, s_gemm, probe=clk_k.sample_now)
+        clk_k.active = False
+    clocks_kernel = clk_k.summary()
     g_rep, s_rep = capture(repack_only, args.steps)
     g_rep.replay()
     ms_rep = timed(g_rep, s_rep)
@@ -655,6 +660,13 @@ def run_ours(args):
         roof["note"] = ("latency-bound: %d bytes per launch take ~%.0f ns at HBM speed, far below a launch; "
                         "the fraction is not meaningful, the us are" % (algorithmic_bytes(fmt, M, N, K),
                                                                         algorithmic_bytes(fmt, M, N, K) / hbm))
+    if roof["bound"] == "tensor" and "bf16_tflops_sustained" in peaks:
+        # the same against the GPU's sustained (power-capped) bf16 rate, for
+        # a kernel that runs back to back for the whole timed region
+        sus = peaks["bf16_tflops_sustained"] * (2.0 if fmt == 0 else 4.0)
+        roof["frac_of_sustained"] = achieved / sus
+        roof["peak_sustained"] = sus
+    roof["kernel_clocks"] = clocks_kernel
     roof["kernel"] = ("mx_gemm_kernel (scale conversion fused)" if fused else
                       "mx_gemm_pair_kernel" if "pair=1" in plan else "mx_gemm_kernel")
     roof["algorithmic_bytes"] = algorithmic_bytes(fmt, M, N, K)

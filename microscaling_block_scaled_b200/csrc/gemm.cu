@@ -108,11 +108,15 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
         pl.counter_bytes = 4;
         pl.tail_first = pl.tiles;
         pl.tail_split = 1;
-        // Automatic schedule: when the last wave of whole tiles would leave
-        // pairs idle, split each of its tiles into up to four K ranges over
-        // them; the split tiles' FP32 partials (128 KB per CTA and range)
-        // are summed by the range that finishes last.
-        if (sched == 0) {
+        // Last-wave split (measurement knob MXGEMM_TAIL=1): when the last
+        // wave of whole tiles would leave pairs idle, split each of its tiles
+        // into up to four K ranges over them; the split tiles' FP32 partials
+        // (128 KB per CTA and range) are summed by the range that finishes
+        // last.  Off by default: in chained steps, where the next GEMM's CTAs
+        // start on the pairs the last wave leaves idle, it measured slower
+        // (MXFP4 2048x28672x8192: 4418 TFLOPS whole tiles, 3703 split).
+        const char *tail = getenv("MXGEMM_TAIL");
+        if (sched == 0 && tail && atoi(tail) == 1) {
             const int64_t full = pl.tiles / npairs * npairs, rest = pl.tiles - full;
             int64_t sp = rest > 0 ? npairs / rest : 1;
             sp = sp > 4 ? 4 : sp;
@@ -195,7 +199,7 @@ GemmPlan make_grouped_plan(int fmt, int64_t G, int64_t M_total, int64_t N, int64
     pl.K = K;
     pl.swap = 0;
     pl.pair = 0;
-    pl.bn = 128;
+    pl.bn = N >= 256 ? 256 : 128;         // 128 x 256 tiles halve the row operand's reads per output
     pl.P = M_total;
     pl.Q = N;
     const int64_t chunks = (row_bytes(fmt, K) + 127) / 128;

@@ -492,45 +492,46 @@ struct EpiOps {
     int64_t P, Q, ldc;
 };
 
-// Fused operations on cw values of C held by one thread: v = act(v +
-// bias[n]) + residual[m][n], each step rounded to FP32.  Plain layout: the
-// thread holds row m = p, columns n = q0 + j (valid below Q); swapped: column
-// n = p (valid below P), rows m = q0 + j (valid below Q).  Values outside C
-// are left alone.
+// Fused operations on cw (<= 32) values of C held by one thread: v =
+// act(v + bias[n]) + residual[m][n], each step rounded to FP32.  Plain
+// layout: the thread holds row m = p, columns n = q0 + j (valid below Q);
+// swapped: column n = p (valid below P), rows m = q0 + j (valid below Q).
+// Values outside C are left alone.  All bias and residual loads are issued
+// before any arithmetic, so the thread waits for memory once, not once per
+// value.
 static __device__ __noinline__ void apply_epilogue_ops(float *v, int cw, const EpiOps e, int64_t p, int64_t plim,
-                                                int64_t q0)
+                                                       int64_t q0)
 {
+    float b[32], r[32];
+    int64_t nv;
     if (!e.swap) {
         if (p >= plim)
             return;
-        const uint16_t *res = e.residual ? e.residual + p * e.ldc : nullptr;
-        for (int j = 0; j < cw; ++j) {
-            const int64_t n = q0 + j;
-            if (n >= e.Q)
-                break;
-            float x = e.bias ? __fadd_rn(v[j], bf16_bits_to_float(e.bias[n])) : v[j];
-            x = activate(x, e.act);
-            v[j] = res ? __fadd_rn(x, bf16_bits_to_float(res[n])) : x;
+        nv = e.Q - q0 < cw ? e.Q - q0 : cw;
+        const uint16_t *res = e.residual ? e.residual + p * e.ldc + q0 : nullptr;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            b[j] = (e.bias && j < nv) ? bf16_bits_to_float(e.bias[q0 + j]) : 0.0f;
+            r[j] = (res && j < nv) ? bf16_bits_to_float(res[j]) : 0.0f;
         }
     } else {
         if (p >= e.P)
             return;
-        const float b = e.bias ? bf16_bits_to_float(e.bias[p]) : 0.0f;
-        for (int j = 0; j < cw; ++j) {
-            const int64_t m = q0 + j;
-            if (m >= e.Q)
-                break;
-            float x = e.bias ? __fadd_rn(v[j], b) : v[j];
-            x = activate(x, e.act);
-            v[j] = e.residual ? __fadd_rn(x, bf16_bits_to_float(e.residual[m * e.ldc + p])) : x;
+        nv = e.Q - q0 < cw ? e.Q - q0 : cw;
+        const float bp = e.bias ? bf16_bits_to_float(e.bias[p]) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            b[j] = bp;
+            r[j] = (e.residual && j < nv) ? bf16_bits_to_float(e.residual[(q0 + j) * e.ldc + p]) : 0.0f;
         }
+    }
+    for (int j = 0; j < nv; ++j) {
+        float x = e.bias ? __fadd_rn(v[j], b[j]) : v[j];
+        x = activate(x, e.act);
+        v[j] = e.residual ? __fadd_rn(x, r[j]) : x;
     }
 }
 
-// Quantised output, plain layout: the 32 values v of row m = p, columns
-// n = q0 .. q0 + 31 of C (one run of the next layer's K) become one E8M0
-// scale and 32 MX codes by the rule of the input quantiser, applied to the
-// values rounded to BF16.
 struct QOut {
     uint8_t *Cq, *Cs;
     int64_t ldc;           // N
@@ -572,23 +573,28 @@ static __device__ __noinline__ void quantise_store_plain(const float *vin, const
 
 // Quantised output, swapped layout: the 32 lanes of the calling warp hold
 // C[m][n] for 32 consecutive n (n = p of each lane, the first a multiple of
-// 32); together they form one run.  All 32 lanes must call.
-static __device__ __noinline__ void quantise_store_swapped(float vin, const QOut kp, int64_t p, int64_t m, int lane)
+// 32) and rows m = m0 .. m0 + nm - 1 (values vin[j]); for each row the 32
+// lanes form one run.  All 32 lanes must call with the same m0 and nm.
+static __device__ __noinline__ void quantise_store_swapped(const float *vin, int nm, const QOut kp, int64_t p,
+                                                           int64_t m0, int lane)
 {
-    const float v = __bfloat162float(__float2bfloat16_rn(vin));
-    const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(v) & 0x7FFFFFFFu);
-    float inv;
-    const uint32_t sb = kp.qfmt == kFmtMXFP8 ? mx_block_scale<8>(amax, &inv) : mx_block_scale<2>(amax, &inv);
-    const float q = sb == 0xFFu ? 0.0f : __fmul_rn(v, inv);
-    if (kp.qfmt == kFmtMXFP8) {
-        kp.Cq[m * kp.ldc + p] = static_cast<uint8_t>(cvt_e4m3(q));
-    } else {
-        const float hi = __shfl_down_sync(0xffffffffu, q, 1);
-        if ((lane & 1) == 0)
-            kp.Cq[m * (kp.ldc / 2) + p / 2] = static_cast<uint8_t>(cvt_e2m1x2(hi, q));
+    for (int j = 0; j < nm; ++j) {
+        const int64_t m = m0 + j;
+        const float v = __bfloat162float(__float2bfloat16_rn(vin[j]));
+        const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(v) & 0x7FFFFFFFu);
+        float inv;
+        const uint32_t sb = kp.qfmt == kFmtMXFP8 ? mx_block_scale<8>(amax, &inv) : mx_block_scale<2>(amax, &inv);
+        const float q = sb == 0xFFu ? 0.0f : __fmul_rn(v, inv);
+        if (kp.qfmt == kFmtMXFP8) {
+            kp.Cq[m * kp.ldc + p] = static_cast<uint8_t>(cvt_e4m3(q));
+        } else {
+            const float hi = __shfl_down_sync(0xffffffffu, q, 1);
+            if ((lane & 1) == 0)
+                kp.Cq[m * (kp.ldc / 2) + p / 2] = static_cast<uint8_t>(cvt_e2m1x2(hi, q));
+        }
+        if (lane == 0)
+            kp.Cs[m * (kp.ldc / 32) + p / 32] = static_cast<uint8_t>(sb);
     }
-    if (lane == 0)
-        kp.Cs[m * (kp.ldc / 32) + p / 32] = static_cast<uint8_t>(sb);
 }
 
 template <int FMT, int BN, int KC>
@@ -1030,12 +1036,13 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                         t[j] = v[j];
                     quantise_store_plain(t, qo, p, q0);
                 }
-            } else if (p - lane < kp.P) {       // the warp's first n: uniform over the warp
-                const int64_t nq = kp.Q - q0 < CW ? kp.Q - q0 : CW;
+            } else if (p - lane < kp.P && q0 < kp.Q) {   // the warp's first n: uniform over the warp
+                const int nq = static_cast<int>(kp.Q - q0 < CW ? kp.Q - q0 : CW);
+                float t[CW];
 #pragma unroll
                 for (int j = 0; j < CW; ++j)
-                    if (j < nq)
-                        quantise_store_swapped(v[j], qo, p, q0 + j, lane);
+                    t[j] = v[j];
+                quantise_store_swapped(t, nq, qo, p, q0, lane);
             }
         };
 

@@ -115,8 +115,8 @@ def test_gemm_k_chunks_per_stage(fmt, kc, M, N, K):
 @pytest.mark.parametrize("M,N,K", [(1024, 5120, 1024), (1000, 5000, 2048), (2048, 4864, 1024)])
 def test_gemm_cta_pair_last_wave_split(fmt, M, N, K):
     """CTA-pair plans whose last wave of whole tiles would leave pairs idle
-    split that wave's tiles into K ranges; the FP32 partials are summed by
-    the range that finishes last."""
+    split that wave's tiles into K ranges (under the MXGEMM_TAIL knob); the
+    FP32 partials are summed by the range that finishes last."""
     _, plan = rows_case(fmt, M, N, K, seed=M + K)
     assert "pair=1" in plan and "sched=dptail" in plan, plan
     # the same shape again: the tile counters were left at zero
@@ -163,6 +163,16 @@ PATHS = {
 
 def _shape(path, default):
     return PATHS[path][0] or default
+
+
+@pytest.fixture(autouse=True)
+def _last_wave_split_knob(request, monkeypatch):
+    # the last-wave split of CTA-pair plans is a measurement knob: on for the
+    # cases that exercise it, unset for all others
+    if "tail" in request.node.name or "last_wave" in request.node.name:
+        monkeypatch.setenv("MXGEMM_TAIL", "1")
+    else:
+        monkeypatch.delenv("MXGEMM_TAIL", raising=False)
 
 
 def _codes_case(fmt, A, SA, B, SB, K, path="auto"):

@@ -26,9 +26,11 @@ def _library():
 
 @pytest.fixture(autouse=True)
 def _default_planner(monkeypatch):
-    # the planner's two measurement knobs stay unset
+    # the planner's measurement knobs stay unset
     monkeypatch.delenv("MXGEMM_BN", raising=False)
     monkeypatch.delenv("MXGEMM_PAIR", raising=False)
+    monkeypatch.delenv("MXGEMM_BAND", raising=False)
+    monkeypatch.delenv("MXGEMM_TAIL", raising=False)
 
 
 def plan(fmt, M, N, K, sms=B200_SMS):
@@ -75,6 +77,17 @@ def test_cta_pairs_for_large_M(M, N, pair):
         assert p["grid"] == 2 * min(p["tiles"], B200_SMS // 2)
 
 
+@pytest.fixture
+def _tail_knob(monkeypatch):
+    monkeypatch.setenv("MXGEMM_TAIL", "1")
+
+
+def test_pair_plans_keep_whole_tiles_by_default():
+    p = plan(F8, 4096, 4096, 8192)
+    assert p["sched"] == "dp" and p["workers"] == p["tiles"] and "tail_split" not in p
+
+
+@pytest.mark.usefixtures("_tail_knob")
 @pytest.mark.parametrize("M,N,full,split", [
     (4096, 4096, 222, 2),      # 256 tiles on 74 pairs: 3 whole waves, 34 tiles split in two
     (2048, 28672, 888, 4),     # 896 tiles: 12 waves, 8 tiles split in four (at most four)

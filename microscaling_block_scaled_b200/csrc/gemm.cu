@@ -63,11 +63,10 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
     const int64_t chunks = (row_bytes(fmt, K) + 127) / 128;
     const bool whole = row_bytes(fmt, K) % 128 == 0;
     pl.kc = (whole && chunks >= 2) ? 2 : 1;
-    // 64-column MXFP8 decode tiles: four chunks per stage measured faster
-    // (64x4096x4096: 15.1 us against 15.4 us with two; MXFP4 is faster with
-    // two, 10.3 us against 11.6 us)
-    if (whole && pl.swap && pl.bn == 64 && chunks >= 4 && fmt == kFmtMXFP8)
-        pl.kc = 4;
+    // (four chunks per stage, mxgemm_set_kchunks(4), fit only two ring
+    // stages on 64-column decode tiles and measured slower in chained steps:
+    // MXFP8 64x4096x4096 15.2 us against 13.0 us with two chunks, MXFP4
+    // 11.5 us against 10.3 us)
     if (force_kc == 1 || (force_kc == 2 && whole))
         pl.kc = force_kc;
     if (force_kc == 4 && whole && pl.bn <= 64)
@@ -143,11 +142,15 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
     int s = sched;
     int auto_splits = 1;
     if (s == 0) {
-        // auto: whole tiles unless the tiles fill at most half the GPU and
-        // each tile has enough K steps to amortise a two-way split's fixup
-        // (measured on B200 for the decode shapes: the split's partial
-        // write, atomic and reduction cost ~2 us per tile).
-        if (pl.tiles * 2 <= sms && pl.kt >= 16) {
+        // auto: whole tiles unless the tiles fill at most a quarter of the
+        // GPU and each tile has enough K steps to amortise a two-way split's
+        // fixup (the partial write, atomic and reduction cost ~2 us per
+        // tile).  Measured in chained steps, where the next GEMM's CTAs
+        // start on the SMs a GEMM leaves idle: a split pays on the dense
+        // BF16 64x4096x4096 (32 tiles, 32 K steps: 18.0 against 18.9 us) and
+        // not on the MX decode shapes (MXFP8 64x4096x4096, 16 K steps: 15.3
+        // against 13.0 us whole).
+        if (pl.tiles * 4 <= sms && pl.kt >= 32) {
             s = 2;
             auto_splits = 2;
         } else {

@@ -467,23 +467,19 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b)
 // e^-x) for x >= 0 and x e^x / (1 + e^x) below, so no intermediate
 // overflows), GELU x * Phi(x) with Phi(x) = erfc(-x / sqrt 2) / 2 (no
 // cancellation in the negative tail).  NaN passes through all three.
-static __device__ __noinline__ float activate(float x, int act)
+__device__ __forceinline__ float act_relu(float x) { return x < 0.0f ? 0.0f : x; }
+
+__device__ __forceinline__ float act_silu(float x)
 {
-    switch (act) {
-    case 1:
-        return x < 0.0f ? 0.0f : x;
-    case 2:
-        if (x >= 0.0f)
-            return __fdiv_rn(x, __fadd_rn(1.0f, expf(-x)));
-        else {
-            const float e = expf(x);
-            return __fdiv_rn(__fmul_rn(x, e), __fadd_rn(1.0f, e));
-        }
-    case 3:
-        return __fmul_rn(__fmul_rn(0.5f, x), erfcf(__fmul_rn(x, -0.70710678118654752f)));
-    default:
-        return x;
-    }
+    if (x >= 0.0f)
+        return __fdiv_rn(x, __fadd_rn(1.0f, expf(-x)));
+    const float e = expf(x);
+    return __fdiv_rn(__fmul_rn(x, e), __fadd_rn(1.0f, e));
+}
+
+__device__ __forceinline__ float act_gelu(float x)
+{
+    return __fmul_rn(__fmul_rn(0.5f, x), erfcf(__fmul_rn(x, -0.70710678118654752f)));
 }
 
 struct EpiOps {
@@ -492,17 +488,34 @@ struct EpiOps {
     int64_t P, Q, ldc;
 };
 
+// v[j] = act(v[j] + b[j]) + r[j] for the first nv of 32 values, unrolled so
+// the values' independent arithmetic overlaps (one warp per sub-partition
+// runs the epilogue: nothing else hides a long dependency chain).
+template <int ACT>
+__device__ __forceinline__ void ops_run(float (&v)[32], const float (&b)[32], const float (&r)[32], int64_t nv,
+                                        bool has_bias, bool has_res)
+{
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        if (j < nv) {
+            float x = has_bias ? __fadd_rn(v[j], b[j]) : v[j];
+            x = ACT == 1 ? act_relu(x) : (ACT == 2 ? act_silu(x) : (ACT == 3 ? act_gelu(x) : x));
+            v[j] = has_res ? __fadd_rn(x, r[j]) : x;
+        }
+    }
+}
+
 // Fused operations on cw (<= 32) values of C held by one thread: v =
 // act(v + bias[n]) + residual[m][n], each step rounded to FP32.  Plain
 // layout: the thread holds row m = p, columns n = q0 + j (valid below Q);
 // swapped: column n = p (valid below P), rows m = q0 + j (valid below Q).
 // Values outside C are left alone.  All bias and residual loads are issued
-// before any arithmetic, so the thread waits for memory once, not once per
-// value.
-static __device__ __noinline__ void apply_epilogue_ops(float *v, int cw, const EpiOps e, int64_t p, int64_t plim,
+// before any arithmetic.  Out of line (one copy per translation unit, not
+// per kernel instance); the arithmetic inside is unrolled.
+static __device__ __noinline__ void apply_epilogue_ops(float *vio, int cw, const EpiOps e, int64_t p, int64_t plim,
                                                        int64_t q0)
 {
-    float b[32], r[32];
+    float v[32], b[32], r[32];
     int64_t nv;
     if (!e.swap) {
         if (p >= plim)
@@ -525,11 +538,20 @@ static __device__ __noinline__ void apply_epilogue_ops(float *v, int cw, const E
             r[j] = (e.residual && j < nv) ? bf16_bits_to_float(e.residual[(q0 + j) * e.ldc + p]) : 0.0f;
         }
     }
-    for (int j = 0; j < nv; ++j) {
-        float x = e.bias ? __fadd_rn(v[j], b[j]) : v[j];
-        x = activate(x, e.act);
-        v[j] = e.residual ? __fadd_rn(x, r[j]) : x;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+        v[j] = j < nv ? vio[j] : 0.0f;
+    const bool hb = e.bias != nullptr, hr = e.residual != nullptr;
+    switch (e.act) {
+    case 1: ops_run<1>(v, b, r, nv, hb, hr); break;
+    case 2: ops_run<2>(v, b, r, nv, hb, hr); break;
+    case 3: ops_run<3>(v, b, r, nv, hb, hr); break;
+    default: ops_run<0>(v, b, r, nv, hb, hr); break;
     }
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+        if (j < nv)
+            vio[j] = v[j];
 }
 
 struct QOut {
@@ -573,27 +595,38 @@ static __device__ __noinline__ void quantise_store_plain(const float *vin, const
 
 // Quantised output, swapped layout: the 32 lanes of the calling warp hold
 // C[m][n] for 32 consecutive n (n = p of each lane, the first a multiple of
-// 32) and rows m = m0 .. m0 + nm - 1 (values vin[j]); for each row the 32
-// lanes form one run.  All 32 lanes must call with the same m0 and nm.
+// 32) and rows m = m0 .. m0 + nm - 1 (values vin[j], nm <= 32); for each row
+// the 32 lanes form one run.  All 32 lanes must call with the same m0 and
+// nm.  Unrolled over the rows so their reductions and conversions overlap.
 static __device__ __noinline__ void quantise_store_swapped(const float *vin, int nm, const QOut kp, int64_t p,
                                                            int64_t m0, int lane)
 {
-    for (int j = 0; j < nm; ++j) {
-        const int64_t m = m0 + j;
-        const float v = __bfloat162float(__float2bfloat16_rn(vin[j]));
-        const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(v) & 0x7FFFFFFFu);
-        float inv;
-        const uint32_t sb = kp.qfmt == kFmtMXFP8 ? mx_block_scale<8>(amax, &inv) : mx_block_scale<2>(amax, &inv);
-        const float q = sb == 0xFFu ? 0.0f : __fmul_rn(v, inv);
-        if (kp.qfmt == kFmtMXFP8) {
-            kp.Cq[m * kp.ldc + p] = static_cast<uint8_t>(cvt_e4m3(q));
-        } else {
-            const float hi = __shfl_down_sync(0xffffffffu, q, 1);
-            if ((lane & 1) == 0)
-                kp.Cq[m * (kp.ldc / 2) + p / 2] = static_cast<uint8_t>(cvt_e2m1x2(hi, q));
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+        v[j] = j < nm ? __bfloat162float(__float2bfloat16_rn(vin[j])) : 0.0f;
+    uint32_t amax[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+        amax[j] = __reduce_max_sync(0xffffffffu, __float_as_uint(v[j]) & 0x7FFFFFFFu);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        if (j < nm) {
+            const int64_t m = m0 + j;
+            float inv;
+            const uint32_t sb =
+                kp.qfmt == kFmtMXFP8 ? mx_block_scale<8>(amax[j], &inv) : mx_block_scale<2>(amax[j], &inv);
+            const float q = sb == 0xFFu ? 0.0f : __fmul_rn(v[j], inv);
+            if (kp.qfmt == kFmtMXFP8) {
+                kp.Cq[m * kp.ldc + p] = static_cast<uint8_t>(cvt_e4m3(q));
+            } else {
+                const float hi = __shfl_down_sync(0xffffffffu, q, 1);
+                if ((lane & 1) == 0)
+                    kp.Cq[m * (kp.ldc / 2) + p / 2] = static_cast<uint8_t>(cvt_e2m1x2(hi, q));
+            }
+            if (lane == 0)
+                kp.Cs[m * (kp.ldc / 32) + p / 32] = static_cast<uint8_t>(sb);
         }
-        if (lane == 0)
-            kp.Cs[m * (kp.ldc / 32) + p / 32] = static_cast<uint8_t>(sb);
     }
 }
 

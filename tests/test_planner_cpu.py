@@ -117,8 +117,8 @@ def test_pair_grid_on_a_small_device():
     (F8, 128, 128, 1),      # one 128-byte chunk
     (F8, 128, 256, 2),
     (F4, 128, 512, 2),
-    (F8, 64, 512, 4),       # 64-column MXFP8 decode tiles take four chunks when rows have them
-    (F4, 64, 4096, 2),      # ... MXFP4 ones two
+    (F8, 64, 512, 2),       # 64-column decode tiles: two chunks (four fit only two stages)
+    (F4, 64, 4096, 2),
     (F8, 64, 384, 2),       # ... and two with fewer than four
     (F4, 32, 4096, 2),
 ])
@@ -126,17 +126,20 @@ def test_k_chunks_per_stage(fmt, M, K, kc):
     assert plan(fmt, M, 1024, K)["kc"] == kc
 
 
-def test_split_k_when_tiles_fill_at_most_half_the_gpu():
+def test_split_k_when_tiles_fill_at_most_a_quarter_of_the_gpu():
     # 2 tiles of 128 x 32, 32 K steps: two-way split, FP32 partials of 128 x BN
     p = plan(F8, 32, 256, 8192)
     assert p["sched"] == "splitk" and p["tiles"] == 2 and p["workers"] == 4 and p["grid"] == 4
     assert p["partial_bytes"] == 2 * p["workers"] * 128 * p["BN"] * 4
     # too few K steps to pay for the fixup: whole tiles
-    q = plan(F8, 32, 256, 1024)
+    q = plan(F8, 32, 256, 4096)
     assert q["sched"] == "dp" and q["workers"] == q["tiles"] and q["partial_bytes"] == 0
     # enough tiles: whole tiles
     r = plan(F8, 32, 4096 * 8, 8192)
     assert r["sched"] == "dp"
+    # the dense BF16 decode shape: 32 tiles, 32 K steps: split in two
+    b = plan(mxgemm.FMT_BF16, 64, 4096, 4096)
+    assert b["sched"] == "splitk" and b["workers"] == 64
 
 
 def test_fused_scales_need_a_deep_one_cta_ring():
@@ -144,8 +147,9 @@ def test_fused_scales_need_a_deep_one_cta_ring():
                          (F8, 64, 4096, 4096), (F4, 64, 4096, 4096), (F8, 4096, 4096, 4096)]:
         p = plan(fmt, M, N, K)
         assert (p["scales"] == "fused") == (p["pair"] == 0 and p["stages"] >= 4), p
-    # 64-column decode tiles with four chunks per stage fit two stages: repack first
-    assert plan(F8, 64, 4096, 4096)["stages"] == 2 and plan(F8, 64, 4096, 4096)["scales"] == "repack"
+    # the 64x4096x4096 decode shape: two chunks per stage, four stages, one launch, whole tiles
+    p = plan(F8, 64, 4096, 4096)
+    assert p["kc"] == 2 and p["stages"] == 4 and p["scales"] == "fused" and p["sched"] == "dp"
 
 
 def test_plan_invariants_over_random_shapes():

@@ -37,8 +37,13 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MX scaled-GEMM TFLOPS (MXFP8/MXFP4, NT) and % of roofline on 1 B200"
 DEFAULT_WORKLOAD = "mxfp8_8192x8192x8192"
-KERNEL_SOURCES = ["microscaling_block_scaled_b200/csrc/gemm_kernel.cuh", "microscaling_block_scaled_b200/csrc/sm100_ptx.cuh",
-                  "microscaling_block_scaled_b200/csrc/mx_convert.cuh"]
+_CSRC = "microscaling_block_scaled_b200/csrc/"
+# the sources each GEMM kernel is compiled from (a recorded DRAM traffic
+# figure is valid only for the source it was captured on)
+KERNEL_SOURCES = {
+    "one_cta": [_CSRC + f for f in ("gemm_kernel.cuh", "gemm_common.cuh", "sm100_ptx.cuh", "mx_convert.cuh")],
+    "pair": [_CSRC + f for f in ("gemm_pair_kernel.cuh", "gemm_common.cuh", "sm100_ptx.cuh", "mx_convert.cuh")],
+}
 
 
 def parse():
@@ -131,24 +136,25 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def kernel_hash():
+def kernel_hash(kind):
+    """Hash of the sources of one GEMM kernel ("one_cta" or "pair")."""
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload_name):
+def recorded_traffic(workload_name, kind):
     """DRAM bytes per GEMM launch from the committed ncu summary, if it was
-    taken on the current kernel source."""
+    taken on the current source of that kernel."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(workload_name)
-    if not e or e.get("kernel_hash") != kernel_hash():
+    if not e or e.get("kernel_hash") != kernel_hash(kind):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -457,8 +463,8 @@ def run_extra(args, w):
     else:
         ach = fl / (us * 1e-6) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": tc_peak, "unit": "TFLOP/s", "frac": ach / tc_peak}
-    roof.update({"traffic": None, "peak_source": peak_src, "kernel": "mx_gemm_kernel (one-CTA)",
-                 "algorithmic_bytes": abytes, "flops": fl})
+    roof.update({"traffic": recorded_traffic(args.workload, "one_cta"), "peak_source": peak_src,
+                 "kernel": "mx_gemm_kernel (one-CTA)", "algorithmic_bytes": abytes, "flops": fl})
     # end to end: inputs H2D from pinned memory, the op, output D2H, every step
     hx = [t.cpu().pin_memory() for t in sets[0][0] + sets[0][1]]
     ho = [t.cpu().pin_memory() for t in sets[0][2]]
@@ -652,7 +658,7 @@ def run_ours(args):
         achieved = flops(M, N, K) / (kernel_us * 1e-6) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": achieved / tc_peak}
-    tr = recorded_traffic(args.workload)
+    tr = recorded_traffic(args.workload, "pair" if "pair=1" in plan else "one_cta")
     roof["traffic"] = tr
     roof["peak_source"] = "%s (%s)" % (peak_src, "hbm_gbs" if roof["bound"] == "hbm" else
                                        "bf16_tflops x %d (nominal MX/bf16 ratio)" % (2 if fmt == 0 else 4))

@@ -22,7 +22,8 @@ BUILD = os.path.join(ROOT, "_build")
 
 SOURCES = ["api.cu", "gemm.cu", "gemm_mxfp8.cu", "gemm_mxfp4.cu", "gemm_bf16.cu", "gemm_pair.cu", "quant.cu",
            "repack.cu", "noalloc.cu"]
-HEADERS = ["mx_internal.h", "sm100_ptx.cuh", "gemm_kernel.cuh", "mx_convert.cuh"]
+HEADERS = ["mx_internal.h", "sm100_ptx.cuh", "gemm_common.cuh", "gemm_kernel.cuh", "gemm_pair_kernel.cuh",
+           "mx_convert.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I" + os.path.join(ROOT, "include")]

@@ -1,6 +1,6 @@
 // gemm_pair.cu -- instantiates the CTA-pair (cta_group::2) GEMM kernel for
-// MXFP8 and MXFP4 operands (the kernel itself is in gemm_kernel.cuh).
-#include "gemm_kernel.cuh"
+// MXFP8 and MXFP4 operands (the kernel itself is in gemm_pair_kernel.cuh).
+#include "gemm_pair_kernel.cuh"
 
 namespace mxg {
 

@@ -53,18 +53,22 @@ def test_measured_peaks_and_fallback(tmp_path, monkeypatch):
 
 def test_recorded_traffic_only_for_the_captured_source(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.recorded_traffic("mxfp4_32x14336x4096") is None          # no file
+    assert bench.recorded_traffic("mxfp4_32x14336x4096", "one_cta") is None        # no file
     (tmp_path / "profiles").mkdir()
     (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(
         {"mxfp4_32x14336x4096": {"kernel_hash": "aaaa", "dram_bytes_per_launch": 123}}))
-    monkeypatch.setattr(bench, "kernel_hash", lambda: "aaaa")
-    assert bench.recorded_traffic("mxfp4_32x14336x4096") == 123
-    assert bench.recorded_traffic("mxfp8_32x256x512") is None               # not captured
-    monkeypatch.setattr(bench, "kernel_hash", lambda: "bbbb")
-    assert bench.recorded_traffic("mxfp4_32x14336x4096") is None            # kernel changed since
+    monkeypatch.setattr(bench, "kernel_hash", lambda kind: "aaaa" if kind == "one_cta" else "cccc")
+    assert bench.recorded_traffic("mxfp4_32x14336x4096", "one_cta") == 123
+    assert bench.recorded_traffic("mxfp4_32x14336x4096", "pair") is None            # another kernel
+    assert bench.recorded_traffic("mxfp8_32x256x512", "one_cta") is None           # not captured
+    monkeypatch.setattr(bench, "kernel_hash", lambda kind: "bbbb")
+    assert bench.recorded_traffic("mxfp4_32x14336x4096", "one_cta") is None        # kernel changed since
 
 
-def test_kernel_hash_covers_the_kernel_sources():
-    h = bench.kernel_hash()
-    assert len(h) == 16 and int(h, 16) >= 0
-    assert any(p.endswith("gemm_kernel.cuh") for p in bench.KERNEL_SOURCES)
+def test_kernel_hash_covers_each_kernels_sources():
+    for kind, main in (("one_cta", "gemm_kernel.cuh"), ("pair", "gemm_pair_kernel.cuh")):
+        h = bench.kernel_hash(kind)
+        assert len(h) == 16 and int(h, 16) >= 0
+        assert any(p.endswith(main) for p in bench.KERNEL_SOURCES[kind])
+        assert any(p.endswith("gemm_common.cuh") for p in bench.KERNEL_SOURCES[kind])
+    assert bench.kernel_hash("one_cta") != bench.kernel_hash("pair")

@@ -38,11 +38,14 @@ sys.path.insert(0, ROOT)
 METRIC = "MX scaled-GEMM TFLOPS (MXFP8/MXFP4, NT) and % of roofline on 1 B200"
 DEFAULT_WORKLOAD = "mxfp8_8192x8192x8192"
 _CSRC = "microscaling_block_scaled_b200/csrc/"
-# the sources each GEMM kernel is compiled from (a recorded DRAM traffic
-# figure is valid only for the source it was captured on)
+# the sources each GEMM kernel is compiled from, and the planner that picks
+# its tiles and their order (a recorded DRAM traffic figure is valid only
+# for the source it was captured on)
 KERNEL_SOURCES = {
-    "one_cta": [_CSRC + f for f in ("gemm_kernel.cuh", "gemm_common.cuh", "sm100_ptx.cuh", "mx_convert.cuh")],
-    "pair": [_CSRC + f for f in ("gemm_pair_kernel.cuh", "gemm_common.cuh", "sm100_ptx.cuh", "mx_convert.cuh")],
+    "one_cta": [_CSRC + f for f in ("gemm_kernel.cuh", "gemm_common.cuh", "sm100_ptx.cuh", "mx_convert.cuh",
+                                    "gemm.cu")],
+    "pair": [_CSRC + f for f in ("gemm_pair_kernel.cuh", "gemm_common.cuh", "sm100_ptx.cuh", "mx_convert.cuh",
+                                 "gemm.cu")],
 }
 
 

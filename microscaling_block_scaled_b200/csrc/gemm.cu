@@ -91,8 +91,13 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
         pl.kt = (chunks + pl.kc - 1) / pl.kc;
         pl.tiles = pl.tilesP * pl.tilesQ;
         pl.iters = pl.tiles * pl.kt;
-        // tile order: bands of tile rows (measurement knob MXGEMM_BAND)
-        pl.band = pl.tilesP;
+        // Tile order: bands of 8 tile rows (2048 rows of A).  In plain
+        // column-major order the pairs at work at one time span all tile
+        // rows, so every wave re-reads A from DRAM: MXFP8 8192x8192x8192
+        // read 946 MB per launch against 273 MB of A, B, scales and C.  In a
+        // band of 8 rows, A's rows stay in L2 while the band's columns pass.
+        // Measurement knob MXGEMM_BAND.
+        pl.band = pl.tilesP < 8 ? pl.tilesP : 8;
         if (const char *e = getenv("MXGEMM_BAND"))
             if (atoi(e) > 0)
                 pl.band = atoi(e) < pl.tilesP ? atoi(e) : pl.tilesP;

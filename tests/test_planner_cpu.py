@@ -73,6 +73,7 @@ def test_cta_pairs_for_large_M(M, N, pair):
     assert p["pair"] == pair
     if pair:
         assert p["BN"] == 256 and p["scales"] == "repack" and p["sched"] in ("dp", "dptail")
+        assert p["band"] == min(8, cdiv(M, 256))      # tile order: bands of at most 8 tile rows
         assert p["tiles"] == cdiv(M, 256) * cdiv(N, 256)
         assert p["grid"] == 2 * min(p["tiles"], B200_SMS // 2)
 

@@ -60,7 +60,53 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     ap.add_argument("--reps", type=int, default=20, help="extra replays of the step graph for the spread")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--schedule", default="auto",
+                    help="planner override: auto, dp, splitk:S (S K ranges per tile) or streamk:W (W workers)")
+    ap.add_argument("--kchunks", type=int, default=0, choices=[0, 1, 2, 4],
+                    help="128-byte K chunks per ring stage (0: the planner's choice)")
     return ap.parse_args()
+
+
+def parse_schedule(text):
+    """(schedule, splits, workers) for mxgemm_set_schedule from --schedule."""
+    from microscaling_block_scaled_b200 import mxgemm
+    kind, _, arg = text.partition(":")
+    if kind == "auto" and not arg:
+        return mxgemm.SCHED_AUTO, 1, 0
+    if kind == "dp" and not arg:
+        return mxgemm.SCHED_DP, 1, 0
+    if kind == "splitk" and arg.isdigit() and int(arg) >= 1:
+        return mxgemm.SCHED_SPLITK, int(arg), 0
+    if kind == "streamk" and arg.isdigit() and int(arg) >= 1:
+        return mxgemm.SCHED_STREAMK, 1, int(arg)
+    raise SystemExit("--schedule: auto, dp, splitk:S or streamk:W, not %r" % text)
+
+
+def override_label(args):
+    """'' for the planner's own choice, else the override as a suffix."""
+    parts = []
+    if args.schedule != "auto":
+        parts.append(args.schedule.replace(":", ""))
+    if args.kchunks:
+        parts.append("kc%d" % args.kchunks)
+    return "_".join(parts)
+
+
+def traffic_key(args):
+    """Key of the workload's recorded DRAM traffic: plans chosen by an
+    override are recorded under '<workload>@<override>'."""
+    label = override_label(args)
+    return args.workload + ("@" + label if label else "")
+
+
+def override_config(args):
+    """Config keys naming a planner override (none without one)."""
+    return {"planner_override": override_label(args)} if override_label(args) else {}
+
+
+def apply_overrides(h, args):
+    h.set_schedule(*parse_schedule(args.schedule))
+    h.set_kchunks(args.kchunks)
 
 
 def workload(name):
@@ -409,6 +455,7 @@ def run_extra(args, w):
     sets = [([t.clone() for t in ins], [t.clone() for t in extra], outputs()) for _ in range(nsets)]
     h = mxgemm.Handle()
     h.set_prefetch_b(True)
+    apply_overrides(h, args)
 
     def call(i_set, stream):
         x, e, o = sets[i_set % nsets]
@@ -466,7 +513,7 @@ def run_extra(args, w):
     else:
         ach = fl / (us * 1e-6) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": tc_peak, "unit": "TFLOP/s", "frac": ach / tc_peak}
-    roof.update({"traffic": recorded_traffic(args.workload, "one_cta"), "peak_source": peak_src,
+    roof.update({"traffic": recorded_traffic(traffic_key(args), "one_cta"), "peak_source": peak_src,
                  "kernel": "mx_gemm_kernel (one-CTA)", "algorithmic_bytes": abytes, "flops": fl})
     # end to end: inputs H2D from pinned memory, the op, output D2H, every step
     hx = [t.cpu().pin_memory() for t in sets[0][0] + sets[0][1]]
@@ -496,7 +543,7 @@ def run_extra(args, w):
             "metric": METRIC, "value": job_tflops(fl, world, args.steps, ms), "unit": "TFLOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w["fmt"], "data": "synthetic",
-            "config": dict(base_config(args.workload), **{
+            "config": dict(base_config(args.workload), **override_config(args), **{
                 "l2": "inputs rotate over %d copies (%.1f MB each)" % (nsets, abytes / 1e6),
                 "timing": "CUDA graph of K steps, CUDA events on the launch stream", "step_us": us,
                 "plan": (mxgemm.mxgemm_describe_grouped_plan(sms, fmt, len(w["groups"]), M, N, K) if op == "grouped"
@@ -547,6 +594,7 @@ def run_ours(args):
     # B (the weights) is never written by the step before: consecutive steps
     # may overlap B's stream with the previous GEMM's tail
     h.set_prefetch_b(True)
+    apply_overrides(h, args)
     plan = h.describe(fmt, M, N, K)
 
     def step(i, stream=None):
@@ -661,7 +709,7 @@ def run_ours(args):
         achieved = flops(M, N, K) / (kernel_us * 1e-6) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": achieved / tc_peak}
-    tr = recorded_traffic(args.workload, "pair" if "pair=1" in plan else "one_cta")
+    tr = recorded_traffic(traffic_key(args), "pair" if "pair=1" in plan else "one_cta")
     roof["traffic"] = tr
     roof["peak_source"] = "%s (%s)" % (peak_src, "hbm_gbs" if roof["bound"] == "hbm" else
                                        "bf16_tflops x %d (nominal MX/bf16 ratio)" % (2 if fmt == 0 else 4))
@@ -720,7 +768,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": fmt_name, "data": "synthetic",
-            "config": dict(base_config(args.workload), **{
+            "config": dict(base_config(args.workload), **override_config(args), **{
                        "parallelism": "replicas" if world > 1 else "single",
                        "l2": "inputs rotate over %d copies (%.1f MB each, %.0f MB > 2x L2 %.0f MB)" % (
                            nsets, set_bytes / 1e6, nsets * set_bytes / 1e6, l2 / 1e6),

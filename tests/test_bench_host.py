@@ -72,3 +72,25 @@ def test_kernel_hash_covers_each_kernels_sources():
         assert any(p.endswith(main) for p in bench.KERNEL_SOURCES[kind])
         assert any(p.endswith("gemm_common.cuh") for p in bench.KERNEL_SOURCES[kind])
     assert bench.kernel_hash("one_cta") != bench.kernel_hash("pair")
+
+
+def test_schedule_overrides_parse_and_key_the_traffic():
+    from microscaling_block_scaled_b200 import mxgemm
+    assert bench.parse_schedule("auto") == (mxgemm.SCHED_AUTO, 1, 0)
+    assert bench.parse_schedule("dp") == (mxgemm.SCHED_DP, 1, 0)
+    assert bench.parse_schedule("splitk:3") == (mxgemm.SCHED_SPLITK, 3, 0)
+    assert bench.parse_schedule("streamk:148") == (mxgemm.SCHED_STREAMK, 1, 148)
+    for bad in ("splitk", "splitk:0", "streamk:x", "dp:2", "fast"):
+        with pytest.raises(SystemExit):
+            bench.parse_schedule(bad)
+
+    class A:
+        workload = "mxfp4_32x14336x4096"
+        schedule = "auto"
+        kchunks = 0
+
+    a = A()
+    assert bench.traffic_key(a) == "mxfp4_32x14336x4096" and bench.override_config(a) == {}
+    a.schedule, a.kchunks = "splitk:2", 1
+    assert bench.traffic_key(a) == "mxfp4_32x14336x4096@splitk2_kc1"
+    assert bench.override_config(a) == {"planner_override": "splitk2_kc1"}

@@ -17,10 +17,9 @@ namespace mxg {
 
 namespace {
 
-int stages_for(int fmt, int bn, int kc, int res = 1)
+int stages_for(int fmt, int bn, int kc)
 {
-    return fmt == kFmtMXFP8 ? stages_mxfp8(bn, kc, res)
-                            : (fmt == kFmtMXFP4 ? stages_mxfp4(bn, kc, res) : stages_bf16(bn, kc, res));
+    return fmt == kFmtMXFP8 ? stages_mxfp8(bn, kc) : (fmt == kFmtMXFP4 ? stages_mxfp4(bn, kc) : stages_bf16(bn, kc));
 }
 
 }  // namespace
@@ -138,17 +137,13 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
         pl.valid = pl.iters < (int64_t(1) << 31);
         return pl;
     }
-    // Two CTAs per SM on decode tiles (measurement knob MXGEMM_RES=2): half
-    // the ring and 256 TMEM columns each, so the next GEMM's CTAs can start
-    // beside the running ones.
-    if (pl.swap && pl.kc <= 2)
-        if (const char *e = getenv("MXGEMM_RES"))
-            if (atoi(e) == 2) {
-                pl.res = 2;
-                if (pl.bn == 64)
-                    pl.kc = 1;             // a 64-column stage of two chunks leaves room for one
-            }
-    pl.stages = stages_for(fmt, pl.bn, pl.kc, pl.res);
+    pl.stages = stages_for(fmt, pl.bn, pl.kc);
+    // Decode tiles stream the weights once: prefetch each CTA's rows into L2
+    // when it starts (measurement knob MXGEMM_L2PF=0 turns it off).
+    pl.l2pf = pl.swap;
+    if (const char *e = getenv("MXGEMM_L2PF"))
+        if (atoi(e) == 0)
+            pl.l2pf = 0;
     pl.tilesP = (pl.P + 127) / 128;
     pl.tilesQ = (pl.Q + pl.bn - 1) / pl.bn;
     pl.kt = (chunks + pl.kc - 1) / pl.kc;

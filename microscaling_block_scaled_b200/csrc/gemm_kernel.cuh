@@ -66,11 +66,7 @@ namespace mxg {
 
 // ------------------------------------------------------------ configuration
 
-// RES: CTAs of this kernel meant to fit on one SM at the same time.  RES = 2
-// halves the ring and the tensor memory so that a CTA of the next GEMM on
-// the stream can start beside a running one (decode tiles, measurement knob
-// MXGEMM_RES).
-template <int FMT, int BN, int KC, int RES = 1>
+template <int FMT, int BN, int KC>
 struct Cfg {
     static constexpr int kBM = 128;
     static constexpr bool kScaled = FMT != kFmtBF16;          // MX operands carry E8M0 block scales
@@ -94,9 +90,7 @@ struct Cfg {
     static constexpr bool kStaged = BN > 32;
     static constexpr int kChunkOutBytes = 128 * kCW * 2;      // one BF16 output chunk
     static constexpr int kOutBytes = kStaged ? kChunkOutBytes : 0;
-    static constexpr int kSmemCap = RES == 1 ? 227 * 1024 : 113 * 1024;   // per CTA
-    static constexpr int kSmemBudget = kSmemCap - 2048 - 2 * kOutBytes;
-    static constexpr int kTmemCols = RES == 1 ? 512 : 256;
+    static constexpr int kSmemBudget = 227 * 1024 - 2048 - 2 * kOutBytes;
     static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
     static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
     static constexpr int kSFACols = kAtoms * 4;
@@ -115,16 +109,16 @@ struct Cfg {
     static constexpr int kMmaPerUnit = kScaled ? kMmaPerAtom : 4;  // BF16: K = 16 (32 bytes) per MMA
     static constexpr int pick_nmma()
     {
-        // two CTAs per SM share its registers: at most two MMA warps there
-        for (int nm = RES == 1 ? 4 : 2; nm > 1; nm /= 2)
-            if (kUnits % nm == 0 && (BN <= 64 ? nm * BN : 2 * nm * BN) + kSFCols <= kTmemCols)
+        for (int nm = 4; nm > 1; nm /= 2)
+            if (kUnits % nm == 0 && (BN <= 64 ? nm * BN : 2 * nm * BN) + kSFCols <= 512)
                 return nm;
         return 1;
     }
     static constexpr int kNMma = pick_nmma();
     static constexpr int kUnitsPerMma = kUnits / kNMma;
-    static constexpr int kNumAcc = (2 * kNMma * BN + kSFCols <= kTmemCols) ? 2 : 1;
+    static constexpr int kNumAcc = (2 * kNMma * BN + kSFCols <= 512) ? 2 : 1;
     static constexpr int kAccCols = kNumAcc * kNMma * BN;
+    static constexpr int kTmemCols = 512;
     // warps: 0 row-operand TMA, 1 MMA, 2..5 epilogue, 6 column-operand TMA,
     // 7 row-scale TMA, 8 column-scale TMA, 9.. further MMA warps
     static constexpr int kWarps = 9 + kNMma - 1;
@@ -148,8 +142,7 @@ struct Cfg {
     static_assert(kAccCols + kSFCols <= kTmemCols, "TMEM budget");
     static_assert(kBChunk % 1024 == 0, "tiles must keep 1024-byte alignment");
     static_assert(kStaged || 2 * kChunkOutBytes <= kABytes, "ring stage 0 holds two output chunks");
-    static_assert(kSmemBytes <= kSmemCap, "shared memory budget");
-    static_assert(RES == 1 || RES == 2, "one or two resident CTAs per SM");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
 // Instruction descriptor of the block-scaled MMA (PTX ISA, instruction
@@ -563,13 +556,13 @@ static __device__ __noinline__ void quantise_store_swapped(const float *vin, int
     }
 }
 
-template <int FMT, int BN, int KC, int RES = 1>
-__global__ void __launch_bounds__(Cfg<FMT, BN, KC, RES>::kThreads, RES)
+template <int FMT, int BN, int KC>
+__global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmSP, const __grid_constant__ CUtensorMap tmSQ,
                    const __grid_constant__ CUtensorMap tmC, const KParams kp_in)
 {
-    using C_ = Cfg<FMT, BN, KC, RES>;
+    using C_ = Cfg<FMT, BN, KC>;
     constexpr int S = C_::kStages;
     constexpr int CW = C_::kCW;
     constexpr int NM = C_::kNMma;
@@ -948,6 +941,25 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC, RES>::kThreads, RES)
         __syncwarp();
     } else if (warp >= 2 && warp <= 5) {
         // ---------------------------------------------------------- epilogue
+        // Before its first accumulator an epilogue warp is idle: warp 5
+        // prefetches the row operand of the CTA's first two whole-K tiles
+        // (and their scales) into L2, ahead of the ring -- before the
+        // dependency wait when the operand is promised early.
+        if (warp == 5 && kp.l2_prefetch && sc.dp) {
+            if (!(kp.early & 1))
+                grid_dependency_wait();
+            if (lane == 0) {
+                uint32_t n = 0;
+                for (uint32_t t = blockIdx.x; t < W && n < 2; t += gridDim.x, ++n) {
+                    const TileCoord tc = plain_coord(kp, t, BN);
+                    const int64_t r1 = tc.prow + 128 < tc.plim ? tc.prow + 128 : tc.plim;
+                    prefetch_l2_range(kp.opP + tc.prow * kp.ldP, (r1 - tc.prow) * kp.ldP);
+                    if (kp.fused_sf)
+                        prefetch_l2_range(kp.rawP + tc.prow * kp.ldS, (r1 - tc.prow) * kp.ldS);
+                }
+            }
+            __syncwarp();
+        }
         grid_dependency_wait();
         const int quad = warp & 3;             // TMEM lanes 32*quad .. +31
         const int row = quad * 32 + lane;      // accumulator row = MMA row in tile
@@ -1215,18 +1227,18 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC, RES>::kThreads, RES)
 
 namespace {
 
-template <int FMT, int BN, int KC, int RES = 1>
+template <int FMT, int BN, int KC>
 cudaError_t set_attrs()
 {
-    return cudaFuncSetAttribute(mx_gemm_kernel<FMT, BN, KC, RES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Cfg<FMT, BN, KC, RES>::kSmemBytes);
+    return cudaFuncSetAttribute(mx_gemm_kernel<FMT, BN, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Cfg<FMT, BN, KC>::kSmemBytes);
 }
 
-template <int FMT, int BN, int KC, int RES = 1>
+template <int FMT, int BN, int KC>
 cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
                      cudaStream_t st)
 {
-    using C_ = Cfg<FMT, BN, KC, RES>;
+    using C_ = Cfg<FMT, BN, KC>;
     const int64_t rbytes = row_bytes(FMT, pl.K);
     const bool grouped = pl.groups > 0;
     const void *Pptr = pl.swap ? b.B : b.A;
@@ -1308,6 +1320,9 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     kp.band = 0;
     kp.tail_first = 0;
     kp.tail_split = 1;
+    kp.l2_prefetch = (pl.l2pf && !grouped) ? 1 : 0;
+    kp.opP = static_cast<const uint8_t *>(Pptr);
+    kp.ldP = rbytes;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
     cfg.blockDim = dim3(C_::kThreads);
@@ -1318,24 +1333,13 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, mx_gemm_kernel<FMT, BN, KC, RES>, tmP, tmQ, tmSP, tmSQ, tmC, kp);
+    return cudaLaunchKernelEx(&cfg, mx_gemm_kernel<FMT, BN, KC>, tmP, tmQ, tmSP, tmSQ, tmC, kp);
 }
 
 template <int FMT, int KC>
 cudaError_t dispatch_bn(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
                         cudaStream_t st)
 {
-    if (pl.res == 2) {                     // decode tiles, two CTAs per SM
-        switch (pl.bn) {
-        case 16: return launch_t<FMT, 16, KC, 2>(pl, b, limit_ns, inject, pdl, st);
-        case 32: return launch_t<FMT, 32, KC, 2>(pl, b, limit_ns, inject, pdl, st);
-        case 64:                           // 64-column tiles fit two stages only with one chunk each
-            if constexpr (KC == 1)
-                return launch_t<FMT, 64, KC, 2>(pl, b, limit_ns, inject, pdl, st);
-            return cudaErrorInvalidValue;
-        default: return cudaErrorInvalidValue;
-        }
-    }
     switch (pl.bn) {
     case 16: return launch_t<FMT, 16, KC>(pl, b, limit_ns, inject, pdl, st);
     case 32: return launch_t<FMT, 32, KC>(pl, b, limit_ns, inject, pdl, st);

@@ -26,17 +26,8 @@ int stages_kc(int bn)
 
 }  // namespace
 
-int stages_mxfp8(int bn, int kc, int res)
+int stages_mxfp8(int bn, int kc)
 {
-    if (res == 2) {                        // decode tiles, two CTAs per SM: 1 or 2 chunks, BN <= 64
-        const bool k1 = kc == 1;
-        switch (bn) {
-        case 16: return k1 ? Cfg<kFmtMXFP8, 16, 1, 2>::kStages : Cfg<kFmtMXFP8, 16, 2, 2>::kStages;
-        case 32: return k1 ? Cfg<kFmtMXFP8, 32, 1, 2>::kStages : Cfg<kFmtMXFP8, 32, 2, 2>::kStages;
-        case 64: return k1 ? Cfg<kFmtMXFP8, 64, 1, 2>::kStages : 0;
-        default: return 0;
-        }
-    }
     return kc == 4 ? stages_kc<4>(bn) : (kc == 1 ? stages_kc<1>(bn) : stages_kc<2>(bn));
 }
 
@@ -56,8 +47,7 @@ cudaError_t prepare_mxfp8()
         set_attrs<kFmtMXFP8, 16, 1>, set_attrs<kFmtMXFP8, 32, 1>, set_attrs<kFmtMXFP8, 64, 1>, set_attrs<kFmtMXFP8, 128, 1>,
         set_attrs<kFmtMXFP8, 256, 1>, set_attrs<kFmtMXFP8, 16, 2>, set_attrs<kFmtMXFP8, 32, 2>, set_attrs<kFmtMXFP8, 64, 2>,
         set_attrs<kFmtMXFP8, 128, 2>, set_attrs<kFmtMXFP8, 256, 2>, set_attrs<kFmtMXFP8, 16, 4>, set_attrs<kFmtMXFP8, 32, 4>,
-        set_attrs<kFmtMXFP8, 64, 4>, set_attrs<kFmtMXFP8, 16, 1, 2>, set_attrs<kFmtMXFP8, 32, 1, 2>,
-        set_attrs<kFmtMXFP8, 64, 1, 2>, set_attrs<kFmtMXFP8, 16, 2, 2>, set_attrs<kFmtMXFP8, 32, 2, 2>};
+        set_attrs<kFmtMXFP8, 64, 4>};
     for (auto f : fns)
         if (e == cudaSuccess)
             e = f();

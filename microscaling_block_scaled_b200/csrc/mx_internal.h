@@ -68,7 +68,7 @@ struct GemmPlan {
     int64_t counter_bytes = 0;
     int64_t groups = 0;         // > 0: grouped plan (make_grouped_plan)
     int64_t band = 0;           // CTA-pair plans: tile rows per band of the tile order (0: all)
-    int res = 1;                // one-CTA plans: CTAs of the kernel that fit on one SM (1 or 2)
+    int l2pf = 0;               // one-CTA decode plans: whole-tile L2 prefetch of the row operand
     // CTA-pair plans: the tiles from tail_first on (the last, partial wave)
     // are each split into tail_split K ranges (1: whole tiles only)
     int64_t tail_first = 0, tail_split = 1;
@@ -131,9 +131,9 @@ cudaError_t prepare_gemm_kernels();
 // (gemm_mxfp8.cu, gemm_mxfp4.cu, gemm_bf16.cu: one-CTA kernel;
 // gemm_pair.cu: CTA-pair kernel): ring depth of a configuration, launch,
 // and shared-memory attribute setup.
-int stages_mxfp8(int bn, int kc, int res = 1);
-int stages_mxfp4(int bn, int kc, int res = 1);
-int stages_bf16(int bn, int kc, int res = 1);
+int stages_mxfp8(int bn, int kc);
+int stages_mxfp4(int bn, int kc);
+int stages_bf16(int bn, int kc);
 int stages_pair(int fmt, int kc);
 cudaError_t launch_gemm_mxfp8(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns, int inject, int pdl,
                               cudaStream_t st);

@@ -124,23 +124,6 @@ def test_gemm_cta_pair_last_wave_split(fmt, M, N, K):
 
 
 @pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
-@pytest.mark.parametrize("M,N,K", [(32, 1024, 2048), (9, 640, 1536), (64, 768, 1024), (48, 300, 512)])
-@pytest.mark.parametrize("sched", [None, (mxgemm.SCHED_SPLITK, 3, 0)], ids=["auto", "splitk3"])
-def test_gemm_decode_two_per_sm(fmt, M, N, K, sched):
-    """Decode tiles in the two-CTAs-per-SM configuration (half the ring and
-    256 TMEM columns per CTA, at most two MMA warps; measurement knob)."""
-    h = handle()
-    if sched is not None:
-        h.set_schedule(*sched)
-    try:
-        plan = h.describe(fmt, M, N, K)
-    finally:
-        h.set_schedule(mxgemm.SCHED_AUTO)
-    assert "res=2" in plan and "swap=1" in plan, plan
-    full_case(fmt, M, N, K, seed=M + N, schedule=sched)
-
-
-@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
 @pytest.mark.parametrize("kc", [0, 1, 2])
 @pytest.mark.parametrize("M,N,K", [(512, 8192, 256), (640, 8448, 384), (1000, 4104, 512)])
 def test_gemm_cta_pair_tiles(fmt, kc, M, N, K):
@@ -183,18 +166,13 @@ def _shape(path, default):
 
 
 @pytest.fixture(autouse=True)
-def _measurement_knobs(request, monkeypatch):
-    # the last-wave split of CTA-pair plans and two CTAs per SM on decode
-    # tiles are measurement knobs: on for the cases that exercise them,
-    # unset for all others
+def _last_wave_split_knob(request, monkeypatch):
+    # the last-wave split of CTA-pair plans is a measurement knob: on for the
+    # cases that exercise it, unset for all others
     if "tail" in request.node.name or "last_wave" in request.node.name:
         monkeypatch.setenv("MXGEMM_TAIL", "1")
     else:
         monkeypatch.delenv("MXGEMM_TAIL", raising=False)
-    if "two_per_sm" in request.node.name:
-        monkeypatch.setenv("MXGEMM_RES", "2")
-    else:
-        monkeypatch.delenv("MXGEMM_RES", raising=False)
 
 
 def _codes_case(fmt, A, SA, B, SB, K, path="auto"):

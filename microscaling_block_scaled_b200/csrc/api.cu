@@ -259,8 +259,6 @@ void format_plan(const mxg::GemmPlan &pl, char *buf, size_t cap)
         snprintf(buf + n, cap - n, " groups=%lld", static_cast<long long>(pl.groups));
     if (pl.pair && n > 0 && static_cast<size_t>(n) < cap)
         n += snprintf(buf + n, cap - n, " band=%lld", static_cast<long long>(pl.band));
-    if (pl.l2pf && !pl.pair && n > 0 && static_cast<size_t>(n) < cap)
-        n += snprintf(buf + n, cap - n, " l2pf=1");
     if (pl.pair && pl.tail_split > 1 && n > 0 && static_cast<size_t>(n) < cap)
         snprintf(buf + n, cap - n, " tail_first=%lld tail_split=%lld", static_cast<long long>(pl.tail_first),
                  static_cast<long long>(pl.tail_split));

@@ -138,12 +138,6 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
         return pl;
     }
     pl.stages = stages_for(fmt, pl.bn, pl.kc);
-    // Decode tiles stream the weights once: prefetch each CTA's rows into L2
-    // when it starts (measurement knob MXGEMM_L2PF=0 turns it off).
-    pl.l2pf = pl.swap;
-    if (const char *e = getenv("MXGEMM_L2PF"))
-        if (atoi(e) == 0)
-            pl.l2pf = 0;
     pl.tilesP = (pl.P + 127) / 128;
     pl.tilesQ = (pl.Q + pl.bn - 1) / pl.bn;
     pl.kt = (chunks + pl.kc - 1) / pl.kc;

@@ -62,12 +62,6 @@ struct KParams {
     // CTA-pair plans: tiles from tail_first on (the last, partial wave) are
     // split into tail_split K ranges, each its own work unit (1: no split)
     uint32_t tail_first, tail_split;
-    // Decode tiles: the row operand (the weights, read once) and its
-    // row-major scales are prefetched into L2 a whole tile at a time when the
-    // CTA starts, so the DRAM stream does not wait for ring stages to free.
-    int l2_prefetch;
-    const uint8_t *opP;    // row operand, rows of ldP bytes
-    int64_t ldP;
 };
 
 // Error site codes written to the device error word.

@@ -941,25 +941,6 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         __syncwarp();
     } else if (warp >= 2 && warp <= 5) {
         // ---------------------------------------------------------- epilogue
-        // Before its first accumulator an epilogue warp is idle: warp 5
-        // prefetches the row operand of the CTA's first two whole-K tiles
-        // (and their scales) into L2, ahead of the ring -- before the
-        // dependency wait when the operand is promised early.
-        if (warp == 5 && kp.l2_prefetch && sc.dp) {
-            if (!(kp.early & 1))
-                grid_dependency_wait();
-            if (lane == 0) {
-                uint32_t n = 0;
-                for (uint32_t t = blockIdx.x; t < W && n < 2; t += gridDim.x, ++n) {
-                    const TileCoord tc = plain_coord(kp, t, BN);
-                    const int64_t r1 = tc.prow + 128 < tc.plim ? tc.prow + 128 : tc.plim;
-                    prefetch_l2_range(kp.opP + tc.prow * kp.ldP, (r1 - tc.prow) * kp.ldP);
-                    if (kp.fused_sf)
-                        prefetch_l2_range(kp.rawP + tc.prow * kp.ldS, (r1 - tc.prow) * kp.ldS);
-                }
-            }
-            __syncwarp();
-        }
         grid_dependency_wait();
         const int quad = warp & 3;             // TMEM lanes 32*quad .. +31
         const int row = quad * 32 + lane;      // accumulator row = MMA row in tile
@@ -1320,9 +1301,6 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     kp.band = 0;
     kp.tail_first = 0;
     kp.tail_split = 1;
-    kp.l2_prefetch = (pl.l2pf && !grouped) ? 1 : 0;
-    kp.opP = static_cast<const uint8_t *>(Pptr);
-    kp.ldP = rbytes;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
     cfg.blockDim = dim3(C_::kThreads);

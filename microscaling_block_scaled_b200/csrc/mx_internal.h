@@ -68,7 +68,6 @@ struct GemmPlan {
     int64_t counter_bytes = 0;
     int64_t groups = 0;         // > 0: grouped plan (make_grouped_plan)
     int64_t band = 0;           // CTA-pair plans: tile rows per band of the tile order (0: all)
-    int l2pf = 0;               // one-CTA decode plans: whole-tile L2 prefetch of the row operand
     // CTA-pair plans: the tiles from tail_first on (the last, partial wave)
     // are each split into tail_split K ranges (1: whole tiles only)
     int64_t tail_first = 0, tail_split = 1;

@@ -245,27 +245,6 @@ __device__ __forceinline__ void grid_launch_dependents()
 }
 
 // L2 cache policies for the loads (createpolicy results).
-// L2 prefetch of a contiguous global range (PTX ISA, cp.async.bulk.prefetch):
-// the bytes are fetched into L2 without occupying shared memory or
-// registers.  Address and size must be multiples of 16 bytes.
-__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
-                 : "memory");
-}
-
-// Prefetch [p, p + bytes) into L2, shrunk inward to 16-byte boundaries (so
-// nothing outside the range is touched), in pieces of at most 64 KB.
-__device__ __forceinline__ void prefetch_l2_range(const void *p, int64_t bytes)
-{
-    const uint64_t b = (reinterpret_cast<uint64_t>(p) + 15) & ~uint64_t(15);
-    const uint64_t e = (reinterpret_cast<uint64_t>(p) + static_cast<uint64_t>(bytes)) & ~uint64_t(15);
-    for (uint64_t a = b; a < e; a += 65536) {
-        const uint64_t n = e - a < 65536 ? e - a : 65536;
-        bulk_prefetch_l2(reinterpret_cast<const void *>(a), static_cast<uint32_t>(n));
-    }
-}
-
 __device__ __forceinline__ uint64_t policy_evict_first()
 {
     uint64_t p;

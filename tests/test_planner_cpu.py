@@ -31,7 +31,6 @@ def _default_planner(monkeypatch):
     monkeypatch.delenv("MXGEMM_PAIR", raising=False)
     monkeypatch.delenv("MXGEMM_BAND", raising=False)
     monkeypatch.delenv("MXGEMM_TAIL", raising=False)
-    monkeypatch.delenv("MXGEMM_L2PF", raising=False)
 
 
 def plan(fmt, M, N, K, sms=B200_SMS):
@@ -50,15 +49,7 @@ def cdiv(a, b):
 def test_decode_shape_plan():
     p = plan(F4, 32, 14336, 4096)
     assert p == {"fmt": 1, "swap": 1, "pair": 0, "BN": 32, "kc": 2, "stages": 5, "tiles": 112, "kt": 8,
-                 "workers": 112, "grid": 112, "sched": "dp", "partial_bytes": 0, "scales": "fused", "l2pf": 1}
-
-
-def test_l2_prefetch_on_decode_tiles_only(monkeypatch):
-    assert plan(F8, 64, 4096, 4096).get("l2pf") == 1
-    assert plan(F8, 65, 4096, 4096).get("l2pf") is None          # row tiles re-read both operands
-    assert plan(F8, 8192, 8192, 8192).get("l2pf") is None        # CTA pairs
-    monkeypatch.setenv("MXGEMM_L2PF", "0")
-    assert plan(F8, 64, 4096, 4096).get("l2pf") is None
+                 "workers": 112, "grid": 112, "sched": "dp", "partial_bytes": 0, "scales": "fused"}
 
 
 @pytest.mark.parametrize("M,swap,bn", [(1, 1, 16), (16, 1, 16), (17, 1, 32), (32, 1, 32), (33, 1, 64),

@@ -87,7 +87,9 @@ enum {
     MXGEMM_SCHED_AUTO = 0,     /* pick per shape (default) */
     MXGEMM_SCHED_DP = 1,       /* one whole output tile per work unit */
     MXGEMM_SCHED_SPLITK = 2,   /* each tile split into `splits` equal K ranges */
-    MXGEMM_SCHED_STREAMK = 3   /* K iterations of all tiles split evenly over the SMs */
+    MXGEMM_SCHED_STREAMK = 3,  /* K iterations of all tiles split evenly over the SMs */
+    MXGEMM_SCHED_KSPLIT = 4    /* decode tiles: each tile's K range split over a cluster of
+                                  `splits` (2-4) CTAs, summed in distributed shared memory */
 };
 
 /* Create a handle bound to the current CUDA device.  The device must be an
@@ -270,8 +272,10 @@ MXGEMM_API int mxgemm_quantize_bf16(int fmt, int64_t R, int64_t K, const void *X
                          void *Q, uint8_t *scales, void *stream);
 
 /* Force a schedule for later mxgemm_run / mxgemm_gemm calls on this handle.
- * splits is used by MXGEMM_SCHED_SPLITK (>= 1); workers by
- * MXGEMM_SCHED_STREAMK (0 = number of SMs). */
+ * splits is used by MXGEMM_SCHED_SPLITK (>= 1) and MXGEMM_SCHED_KSPLIT
+ * (clamped to 2-4; shapes that are not decode tiles, or whose clusters would
+ * not all fit on the GPU at once, take MXGEMM_SCHED_SPLITK instead); workers
+ * by MXGEMM_SCHED_STREAMK (0 = number of SMs). */
 MXGEMM_API int mxgemm_set_schedule(mxgemm_handle h, int schedule, int splits, int workers);
 
 /* Force the number of 128-byte K chunks each pipeline stage of later GEMMs
@@ -286,10 +290,11 @@ MXGEMM_API int mxgemm_set_kchunks(mxgemm_handle h, int kc);
  * grid=112 sched=dp partial_bytes=0 scales=fused".  "scales" says how
  * mxgemm_run treats the scales for this shape: "fused" (the GEMM converts
  * the row-major scales itself, one launch) or "repack" (scale repack, then
- * the GEMM).  sched is dp (whole tiles), splitk, streamk, or for CTA-pair
- * plans dptail: whole tiles, except that the tiles of the last, partial wave
- * (from tail_first on, fields appended) are split into tail_split K ranges
- * over the pairs that wave would leave idle. */
+ * the GEMM).  sched is dp (whole tiles), splitk, streamk, ksplit (the K
+ * range of each tile split over a cluster of `ksplit` CTAs, field appended),
+ * or for CTA-pair plans dptail: whole tiles, except that the tiles of the
+ * last, partial wave (from tail_first on, fields appended) are split into
+ * tail_split K ranges over the pairs that wave would leave idle. */
 MXGEMM_API int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
                          char *buf, size_t cap);
 
@@ -307,7 +312,8 @@ MXGEMM_API int mxgemm_describe_plan_for(int num_sms, int fmt, int64_t M, int64_t
  * up, else a nonzero site code (1 producer waiting for a free stage, 2 MMA
  * waiting for a loaded stage, 3 MMA waiting for a free accumulator,
  * 4 epilogue waiting for a finished accumulator, 5 end-of-kernel drain,
- * 6 kernel launched with a block size it was not built for); the return
+ * 6 kernel launched with a block size it was not built for, 7 cluster K
+ * split waiting for a partial tile or for the go-ahead to write one); the return
  * value is MXGEMM_ERR_TIMEOUT in that case, else MXGEMM_OK. */
 MXGEMM_API int mxgemm_check_device_error(mxgemm_handle h, int *code);
 

@@ -246,19 +246,21 @@ bool optional_aligned16(const void *p) { return p == nullptr || aligned16(p); }
 
 void format_plan(const mxg::GemmPlan &pl, char *buf, size_t cap)
 {
-    static const char *names[] = {"auto", "dp", "splitk", "streamk", "dptail"};
+    static const char *names[] = {"auto", "dp", "splitk", "streamk", "ksplit", "dptail"};
     const char *scales = pl.fmt == mxg::kFmtBF16 ? "none" : ((fuse_scales(pl) || pl.groups > 0) ? "fused" : "repack");
     int n = snprintf(buf, cap,
                      "fmt=%d swap=%d pair=%d BN=%d kc=%d stages=%d tiles=%lld kt=%lld workers=%lld grid=%d sched=%s "
                      "partial_bytes=%lld scales=%s",
                      pl.fmt, pl.swap, pl.pair, pl.bn, pl.kc, pl.stages, static_cast<long long>(pl.tiles),
                      static_cast<long long>(pl.kt), static_cast<long long>(pl.workers), pl.grid,
-                     names[pl.sched >= 0 && pl.sched <= 4 ? pl.sched : 0],
+                     names[pl.sched >= 0 && pl.sched <= 5 ? pl.sched : 0],
                      static_cast<long long>(pl.partial_bytes), scales);
     if (pl.groups > 0 && n > 0 && static_cast<size_t>(n) < cap)
         snprintf(buf + n, cap - n, " groups=%lld", static_cast<long long>(pl.groups));
     if (pl.pair && n > 0 && static_cast<size_t>(n) < cap)
         n += snprintf(buf + n, cap - n, " band=%lld", static_cast<long long>(pl.band));
+    if (pl.ksplit > 1 && n > 0 && static_cast<size_t>(n) < cap)
+        n += snprintf(buf + n, cap - n, " ksplit=%lld", static_cast<long long>(pl.ksplit));
     if (pl.pair && pl.tail_split > 1 && n > 0 && static_cast<size_t>(n) < cap)
         snprintf(buf + n, cap - n, " tail_first=%lld tail_split=%lld", static_cast<long long>(pl.tail_first),
                  static_cast<long long>(pl.tail_split));
@@ -631,7 +633,7 @@ int mxgemm_quantize(int fmt, int64_t R, int64_t K, const float *X, void *Q, uint
 
 int mxgemm_set_schedule(mxgemm_handle h, int schedule, int splits, int workers)
 {
-    if (!h || schedule < MXGEMM_SCHED_AUTO || schedule > MXGEMM_SCHED_STREAMK || splits < 1 || workers < 0)
+    if (!h || schedule < MXGEMM_SCHED_AUTO || schedule > MXGEMM_SCHED_KSPLIT || splits < 1 || workers < 0)
         return MXGEMM_ERR_INVALID_ARG;
     h->sched = schedule;
     h->splits = splits;

@@ -129,7 +129,7 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
                 pl.tail_first = full;
                 pl.tail_split = sp;
                 pl.workers = full + rest * sp;
-                pl.sched = 4;
+                pl.sched = 5;
                 pl.partial_bytes = rest * sp * 2 * 128 * 256 * 4;
                 pl.counter_bytes = rest * 2 * 4;
             }
@@ -146,20 +146,41 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
     const int64_t sms = num_sms > 0 ? num_sms : 1;
     int s = sched;
     int auto_splits = 1;
+    int64_t ks = 1;                    // CTAs of a cluster sharing one tile's K range
     if (s == 0) {
-        // auto: whole tiles unless the tiles fill at most a quarter of the
-        // GPU and each tile has enough K steps to amortise a two-way split's
-        // fixup (the partial write, atomic and reduction cost ~2 us per
-        // tile).  Measured in chained steps, where the next GEMM's CTAs
-        // start on the SMs a GEMM leaves idle: a split pays on the dense
-        // BF16 64x4096x4096 (32 tiles, 32 K steps: 18.0 against 18.9 us) and
-        // not on the MX decode shapes (MXFP8 64x4096x4096, 16 K steps: 15.3
-        // against 13.0 us whole).
-        if (pl.tiles * 4 <= sms && pl.kt >= 32) {
+        // auto: decode tiles (swapped, at most 64 columns) that fill at most
+        // half the GPU split each tile's K range over a cluster of 4 or 2
+        // CTAs, every CTA with at least two K steps; the partial tiles are
+        // summed through distributed shared memory, so the split costs no
+        // global round trip.  (MXFP8 64x4096x4096 runs 32 tiles: whole tiles
+        // leave 116 SMs idle and take 15 us per chained step, a split with
+        // the partials summed through global memory 15.7 us.)
+        if (pl.swap)
+            for (int64_t c = 4; c >= 2; c /= 2)
+                if (pl.tiles * c <= sms && pl.kt >= 2 * c) {
+                    ks = c;
+                    break;
+                }
+        if (ks > 1) {
+            s = 4;
+        } else if (pl.tiles * 4 <= sms && pl.kt >= 32) {
+            // other shapes with few tiles and many K steps: a two-way split
+            // with the partials summed through global memory (the dense BF16
+            // 64x4096x4096 measured 18.0 against 18.9 us whole)
             s = 2;
             auto_splits = 2;
         } else {
             s = 1;
+        }
+    } else if (s == 4) {
+        // forced cluster split: 2 to 4 CTAs per tile, decode tiles only, all
+        // clusters in one wave; otherwise the global-memory split
+        const int64_t c = splits < 2 ? 2 : (splits > 4 ? 4 : splits);
+        if (pl.swap && pl.tiles * c <= sms && pl.kt >= c) {
+            ks = c;
+        } else {
+            s = 2;
+            splits = static_cast<int>(c);
         }
     }
     if (sched == 0 && s == 2)
@@ -170,6 +191,9 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
     } else if (s == 2) {
         const int64_t sp = splits < 1 ? 1 : (splits > pl.kt ? pl.kt : splits);
         pl.workers = pl.tiles * sp;
+    } else if (s == 4) {
+        pl.workers = pl.tiles * ks;
+        pl.ksplit = ks;
     } else {
         int64_t w = workers > 0 ? workers : sms;
         if (w > pl.iters)
@@ -183,6 +207,11 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
     // the kernel's scheduler arithmetic is 32-bit: iters * workers < 2^32
     // unless whole tiles are scheduled (which needs no products)
     const int64_t lim = (int64_t(1) << 32) - 1;
+    if (pl.ksplit > 1 && pl.iters * pl.workers > lim) {
+        pl.ksplit = 1;                 // too long for one cluster wave's arithmetic: whole tiles
+        pl.sched = 1;
+        pl.workers = pl.tiles;
+    }
     if (pl.workers != pl.tiles && pl.iters * pl.workers > lim) {
         const int64_t w = lim / pl.iters;
         pl.workers = w > pl.tiles ? w : pl.tiles;
@@ -193,7 +222,7 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
     pl.grid = static_cast<int>(pl.workers < sms ? pl.workers : sms);
     pl.kaP = sf_atoms_per_rowblock(fmt, K);
     pl.kaQ = pl.kaP;
-    pl.partial_bytes = (pl.workers == pl.tiles) ? 0 : 2 * pl.workers * 128 * pl.bn * 4;
+    pl.partial_bytes = (pl.workers == pl.tiles || pl.ksplit > 1) ? 0 : 2 * pl.workers * 128 * pl.bn * 4;
     pl.counter_bytes = pl.tiles * 4;
     return pl;
 }

@@ -62,6 +62,10 @@ struct KParams {
     // CTA-pair plans: tiles from tail_first on (the last, partial wave) are
     // split into tail_split K ranges, each its own work unit (1: no split)
     uint32_t tail_first, tail_split;
+    // One-CTA plans: > 1 when each tile's K range is split over a cluster of
+    // ksplit CTAs (blockIdx.x = tile * ksplit + cluster rank) whose partial
+    // accumulators are summed through distributed shared memory by rank 0.
+    int ksplit;
 };
 
 // Error site codes written to the device error word.
@@ -72,6 +76,7 @@ enum : int {
     kErrEpiAccFull = 4,
     kErrDrain = 5,
     kErrLaunch = 6,        // launched with a block size the kernel was not built for
+    kErrReduce = 7,        // cluster K split: a partial sum or the leader's go-ahead never came
 };
 
 __device__ __forceinline__ void record_error(int *err, int code, volatile int *abort_flag)

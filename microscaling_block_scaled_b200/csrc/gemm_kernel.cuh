@@ -132,7 +132,14 @@ struct Cfg {
     static constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
     static constexpr int kOffOut = (kOffSFB + kStages * kSFBBytes + 1023) / 1024 * 1024;
     static constexpr int kOffBar = kOffOut + 2 * kOutBytes;
-    static constexpr int kNumBars = 2 * kStages + 2 * kNumAcc + 1;
+    // Cluster K split: rank 0 of a cluster sums the other ranks' partial
+    // tiles, which they write into its ring once it has drained (FP32, 16-byte
+    // column groups: group q of row r at (q * 128 + r) * 16).  The first 16 KB
+    // stay free for the output staging of narrow tiles.
+    static constexpr int kRedOff = kOffA + 16384;
+    static constexpr int kRedSlot = 128 * BN * 4;
+    static constexpr int kMaxKsplit = BN <= 64 ? 4 : 1;
+    static constexpr int kNumBars = 2 * kStages + 2 * kNumAcc + 3;   // + drain, go-ahead, reduction
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 64 + 1024;   // + alignment slack
 
@@ -143,6 +150,7 @@ struct Cfg {
     static_assert(kBChunk % 1024 == 0, "tiles must keep 1024-byte alignment");
     static_assert(kStaged || 2 * kChunkOutBytes <= kABytes, "ring stage 0 holds two output chunks");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+    static_assert(kRedOff + (kMaxKsplit - 1) * kRedSlot <= kOffOut, "partial tiles of a cluster split fit the ring");
 };
 
 // Instruction descriptor of the block-scaled MMA (PTX ISA, instruction
@@ -582,6 +590,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
     auto accf_bar = [&](int a) { return bar0 + 8u * (2 * S + a); };
     auto acce_bar = [&](int a) { return bar0 + 8u * (2 * S + C_::kNumAcc + a); };
     const uint32_t drain_bar = bar0 + 8u * (2 * S + 2 * C_::kNumAcc);
+    const uint32_t go_bar = drain_bar + 8u;       // cluster K split: rank 0's ring is free
+    const uint32_t red_bar = drain_bar + 16u;     // cluster K split: the other ranks' partials are in
     volatile uint32_t *s_tmem = reinterpret_cast<volatile uint32_t *>(smem + C_::kOffMisc);
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C_::kOffMisc + 4);
     volatile int *s_last = reinterpret_cast<volatile int *>(smem + C_::kOffMisc + 8);
@@ -625,6 +635,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
             mbar_init(acce_bar(a), 4);
         }
         mbar_init(drain_bar, NM);
+        mbar_init(go_bar, 1);
+        mbar_init(red_bar, kp.ksplit > 1 ? (kp.ksplit - 1) * 128 : 1);
         *s_abort = 0;
         *s_last = 0;
         fence_mbar_init();
@@ -638,6 +650,11 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    // A cluster K split signals between CTAs: every barrier must be
+    // initialised before any CTA of the cluster can arrive on it.
+    if (kp.ksplit > 1)
+        cluster_sync_all();
+    bool cl_arrived = false;          // this thread's arrival on the final cluster barrier
 
     const Sched sc{kp.iters, kp.workers, kp.kt, kp.tilesP, kp.dp != 0};
     const uint32_t W = sc.W;
@@ -1118,6 +1135,78 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                         }
                         emit(v, tc, tc.qcol + c);
                     }
+                } else if (kp.ksplit > 1) {
+                    // Cluster K split: one work unit per CTA, the tile's ranks
+                    // in one cluster.  Rank 0 hands its drained ring to the
+                    // others, which write their partial tiles into it and
+                    // arrive on its reduction barrier; rank 0 adds them in
+                    // rank order to its own accumulator and writes the tile.
+                    const uint32_t rank = w - g_first;
+                    // the plan puts exactly one cluster on each tile; anything
+                    // else would address partial slots that do not exist
+                    const bool shape_ok = g_first % static_cast<uint32_t>(kp.ksplit) == 0 &&
+                                          g_last - g_first + 1 == static_cast<uint32_t>(kp.ksplit) &&
+                                          kp.ksplit <= C_::kMaxKsplit;
+                    if (!shape_ok) {
+                        if (etid == 0)
+                            record_error(kp.error, kErrReduce, s_abort);
+                    } else if (rank == 0) {
+                        if (etid == 0)
+                            for (int r = 1; r < kp.ksplit; ++r)
+                                mbar_arrive_remote(go_bar, static_cast<uint32_t>(r));
+                        int got = 1;
+                        if (lane == 0)
+                            got = mbar_wait_cluster_parked(red_bar, 0, s_abort, kp.limit_ns);
+                        got = __shfl_sync(0xffffffffu, got, 0);
+                        if (!got && lane == 0)
+                            record_error(kp.error, kErrReduce, s_abort);
+                        // nothing more arrives here: the cluster may finish
+                        cluster_arrive();
+                        cl_arrived = true;
+                        if (!named_bar_or(1, 128, got ? 0 : 1)) {
+#pragma unroll 1
+                            for (int c = 0; c < BN; c += CW) {
+                                float v[CW];
+                                load_acc(t_acc, c, v);
+                                for (int r = 1; r < kp.ksplit; ++r) {
+                                    const float4 *src = reinterpret_cast<const float4 *>(
+                                        smem + C_::kRedOff + (r - 1) * C_::kRedSlot);
+#pragma unroll
+                                    for (int j = 0; j < CW / 4; ++j) {
+                                        const float4 x = src[(c / 4 + j) * 128 + row];
+                                        v[4 * j + 0] += x.x;
+                                        v[4 * j + 1] += x.y;
+                                        v[4 * j + 2] += x.z;
+                                        v[4 * j + 3] += x.w;
+                                    }
+                                }
+                                if (kp.has_ops)
+                                    apply_ops(v, p, tc.plim, tc.qcol + c);
+                                emit(v, tc, tc.qcol + c);
+                            }
+                        }
+                    } else {
+                        int go = 1;
+                        if (lane == 0)
+                            go = mbar_wait_cluster_parked(go_bar, 0, s_abort, kp.limit_ns);
+                        go = __shfl_sync(0xffffffffu, go, 0);
+                        if (!go && lane == 0)
+                            record_error(kp.error, kErrReduce, s_abort);
+                        if (go) {
+                            const uint32_t dst =
+                                cluster_addr(sbase + C_::kRedOff + (rank - 1) * C_::kRedSlot, 0);
+#pragma unroll 1
+                            for (int c = 0; c < BN; c += CW) {
+                                float v[CW];
+                                load_acc(t_acc, c, v);
+#pragma unroll
+                                for (int j = 0; j < CW / 4; ++j)
+                                    st_cluster_v4(dst + ((c / 4 + j) * 128 + row) * 16, v[4 * j], v[4 * j + 1],
+                                                  v[4 * j + 2], v[4 * j + 3]);
+                            }
+                            mbar_arrive_remote(red_bar, 0);
+                        }
+                    }
                 } else {
                     const int64_t slot = 2 * static_cast<int64_t>(w) + (first ? 0 : 1);
                     float *mine = kp.partials + (slot * 128 + row) * BN;
@@ -1196,11 +1285,19 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
             bulk_wait_group<0>();
     }
 
+    if (kp.ksplit > 1 && !cl_arrived)
+        cluster_arrive();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 1)
         tmem_dealloc(tmem, C_::kTmemCols);
+    // No CTA of a cluster K split leaves while another may still touch its
+    // shared memory: each thread arrived when its part was done (rank 0's
+    // epilogue once every partial was in), so the other ranks leave as soon
+    // as rank 0 has its partials.
+    if (kp.ksplit > 1)
+        cluster_wait();
 }
 
 
@@ -1301,16 +1398,30 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     kp.band = 0;
     kp.tail_first = 0;
     kp.tail_split = 1;
+    kp.ksplit = static_cast<int>(pl.ksplit);
+    if (pl.ksplit > 1 && (pl.ksplit > C_::kMaxKsplit || pl.grid != pl.workers || pl.grid % pl.ksplit != 0))
+        return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
     cfg.blockDim = dim3(C_::kThreads);
     cfg.dynamicSmemBytes = C_::kSmemBytes;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (pl.ksplit > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = static_cast<unsigned>(pl.ksplit);
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, mx_gemm_kernel<FMT, BN, KC>, tmP, tmQ, tmSP, tmSQ, tmC, kp);
 }
 

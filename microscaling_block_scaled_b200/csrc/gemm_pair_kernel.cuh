@@ -608,6 +608,7 @@ cudaError_t launch_pair_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t lim
     kp.band = static_cast<uint32_t>(pl.band > 0 ? pl.band : pl.tilesP);
     kp.tail_first = static_cast<uint32_t>(pl.tail_first);
     kp.tail_split = static_cast<uint32_t>(pl.tail_split > 1 ? pl.tail_split : 1);
+    kp.ksplit = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
     cfg.blockDim = dim3(C_::kThreads);

@@ -67,7 +67,8 @@ struct GemmPlan {
     bool valid = true;          // false: the shape exceeds the kernel's 32-bit scheduler range
     int64_t counter_bytes = 0;
     int64_t groups = 0;         // > 0: grouped plan (make_grouped_plan)
-    int64_t band = 0;           // CTA-pair plans: tile rows per band of the tile order (0: all)
+    int64_t band = 0;           // CTA-pair plans: tile rows per band of the tile order
+    int64_t ksplit = 1;         // one-CTA plans: CTAs of a cluster sharing one tile's K range (0: all)
     // CTA-pair plans: the tiles from tail_first on (the last, partial wave)
     // are each split into tail_split K ranges (1: whole tiles only)
     int64_t tail_first = 0, tail_split = 1;

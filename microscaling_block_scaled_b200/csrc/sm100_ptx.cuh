@@ -538,6 +538,27 @@ __device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t pa
     return ok != 0;
 }
 
+// 16-byte store into the shared memory of a CTA of this cluster (`addr` from
+// cluster_addr).
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d)
+{
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+// The two halves of the cluster barrier, per thread (not warp-aligned): a
+// thread's arrive releases its earlier memory operations to the cluster; the
+// wait returns once every thread of the cluster has arrived.
+__device__ __forceinline__ void cluster_arrive()
+{
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait()
+{
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+
 // Shared::cluster address of the object at this CTA's shared address `addr`
 // in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t cluster_addr(uint32_t addr, uint32_t rank)

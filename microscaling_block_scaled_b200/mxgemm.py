@@ -21,7 +21,7 @@ FMT_NAMES = {"mxfp8": FMT_MXFP8, "mxfp4": FMT_MXFP4, "bf16": FMT_BF16}
 
 ACT_NONE, ACT_RELU, ACT_SILU, ACT_GELU = 0, 1, 2, 3
 
-SCHED_AUTO, SCHED_DP, SCHED_SPLITK, SCHED_STREAMK = 0, 1, 2, 3
+SCHED_AUTO, SCHED_DP, SCHED_SPLITK, SCHED_STREAMK, SCHED_KSPLIT = 0, 1, 2, 3, 4
 
 OK = 0
 ERR_INVALID_ARG = 1

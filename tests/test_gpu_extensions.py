@@ -97,6 +97,8 @@ FUSED_PATHS = {
     "splitk3": ((100, 640, 2048), (mxgemm.SCHED_SPLITK, 3, 0)),
     "streamk37": ((100, 640, 2048), (mxgemm.SCHED_STREAMK, 1, 37)),
     "swap-splitk3": ((48, 512, 2048), (mxgemm.SCHED_SPLITK, 3, 0)),
+    "swap-ksplit4": ((48, 512, 2048), (mxgemm.SCHED_KSPLIT, 4, 0)),
+    "swap-dp": ((48, 512, 2048), (mxgemm.SCHED_DP, 1, 0)),
 }
 
 
@@ -123,7 +125,8 @@ def test_fused_epilogue(fmt, act, path):
         assert ok, (path, act, use_bias, use_res, rep)
     plan = _with_schedule(h, sched, lambda: h.describe(fmt, M, N, K))
     if sched is not None:
-        assert ("sched=splitk" if sched[0] == mxgemm.SCHED_SPLITK else "sched=streamk") in plan
+        assert "sched=" + {mxgemm.SCHED_SPLITK: "splitk", mxgemm.SCHED_STREAMK: "streamk",
+                           mxgemm.SCHED_KSPLIT: "ksplit", mxgemm.SCHED_DP: "dp"}[sched[0]] in plan, plan
 
 
 def test_fused_epilogue_residual_in_place():
@@ -170,6 +173,7 @@ QPATHS = {
     "plain": ((200, 384, 768), None),
     "splitk3": ((100, 640, 2048), (mxgemm.SCHED_SPLITK, 3, 0)),
     "swap-streamk": ((40, 512, 2048), (mxgemm.SCHED_STREAMK, 1, 37)),
+    "swap-ksplit2": ((32, 512, 2048), (mxgemm.SCHED_KSPLIT, 2, 0)),
 }
 
 
@@ -194,7 +198,7 @@ def test_quantised_output_integer_exact(fmt, out_fmt, path):
 
 @pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
 @pytest.mark.parametrize("out_fmt", [F8, F4], ids=["to-mxfp8", "to-mxfp4"])
-@pytest.mark.parametrize("path", ["swap", "plain", "splitk3"])
+@pytest.mark.parametrize("path", ["swap", "plain", "splitk3", "swap-ksplit2"])
 @pytest.mark.parametrize("act", [mxgemm.ACT_NONE, mxgemm.ACT_GELU], ids=["none", "gelu"])
 def test_quantised_output_normal_inputs(fmt, out_fmt, path, act):
     """Normal inputs (with bias and GELU on one variant): wherever the GPU's
@@ -280,7 +284,8 @@ def test_bf16_gemm_full(M, N, K):
 
 
 @pytest.mark.parametrize("sched", [(mxgemm.SCHED_SPLITK, 3, 0), (mxgemm.SCHED_STREAMK, 1, 148),
-                                   (mxgemm.SCHED_STREAMK, 1, 37)], ids=["splitk3", "streamk148", "streamk37"])
+                                   (mxgemm.SCHED_STREAMK, 1, 37), (mxgemm.SCHED_KSPLIT, 4, 0)],
+                         ids=["splitk3", "streamk148", "streamk37", "ksplit4"])
 @pytest.mark.parametrize("M,N,K", [(40, 1024, 2048), (200, 640, 1536)])
 def test_bf16_gemm_forced_schedules(sched, M, N, K):
     rng = np.random.default_rng(7)

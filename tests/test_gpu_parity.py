@@ -89,10 +89,31 @@ def test_config_mxfp8_32x256x512_full():
 @pytest.mark.parametrize("sched", [
     (mxgemm.SCHED_DP, 1, 0), (mxgemm.SCHED_SPLITK, 3, 0), (mxgemm.SCHED_SPLITK, 8, 0),
     (mxgemm.SCHED_STREAMK, 1, 0), (mxgemm.SCHED_STREAMK, 1, 7), (mxgemm.SCHED_STREAMK, 1, 37),
+    (mxgemm.SCHED_KSPLIT, 2, 0), (mxgemm.SCHED_KSPLIT, 3, 0), (mxgemm.SCHED_KSPLIT, 4, 0),
 ])
 @pytest.mark.parametrize("M,N,K", [(64, 1024, 2048), (200, 640, 1536)])
 def test_gemm_forced_schedules(fmt, sched, M, N, K):
     full_case(fmt, M, N, K, seed=9, schedule=sched)
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("M,N,K", [
+    (1, 4096, 4096), (9, 640, 2048), (33, 300, 2048), (64, 4104, 2048), (48, 1000, 8192),
+    (16, 128 * 60, 2048), (64, 4096, 4096), (17, 256, 1152), (17, 256, 2304),
+])
+def test_gemm_cluster_k_split(fmt, M, N, K):
+    """Decode tiles that fill at most half the GPU split each tile's K range
+    over a cluster of CTAs; the other ranks write their FP32 partial tiles
+    into rank 0's drained ring through distributed shared memory and rank 0
+    adds them.  Ragged N, K tails (MXFP4 K = 1152: 4.5 chunks per row) and
+    one tile column of 1 to 64 rows."""
+    h = handle()
+    plan = h.describe(fmt, M, N, K)
+    field = dict(f.split("=") for f in plan.split())
+    kt, tiles = int(field["kt"]), int(field["tiles"])
+    want = 4 if kt >= 8 and 4 * tiles <= 148 else 2
+    assert field["sched"] == "ksplit" and int(field["ksplit"]) == want, plan
+    full_case(fmt, M, N, K, seed=M * 3 + K)
 
 
 @pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
@@ -142,10 +163,12 @@ def test_gemm_cta_pair_tiles(fmt, kc, M, N, K):
 #
 # Every edge case runs through every execution path of the GEMM: the small
 # shape under the automatic plan (one-CTA whole tiles, swapped when M <= 64),
-# a shape that takes the CTA pair (cta_group::2, 256x256 tiles), and forced
+# a shape that takes the CTA pair (cta_group::2, 256x256 tiles), forced
 # split-K and stream-K schedules on one-CTA tiles, where the output is the
-# FP32 sum of per-worker partials (last-arriver fixup).  NaN and +-Inf
-# patterns must come out identical on every path.
+# FP32 sum of per-worker partials (last-arriver fixup), and decode tiles as
+# whole tiles and with their K range split over a cluster (partials summed in
+# distributed shared memory).  NaN and +-Inf patterns must come out identical
+# on every path.
 
 PATHS = {
     # name: (shape override or None, schedule or None)
@@ -158,6 +181,9 @@ PATHS = {
     "streamk37": ((200, 640, 2048), (mxgemm.SCHED_STREAMK, 1, 37)),
     "swap-splitk3": ((40, 1024, 2048), (mxgemm.SCHED_SPLITK, 3, 0)),
     "swap-streamk148": ((40, 1024, 2048), (mxgemm.SCHED_STREAMK, 1, 148)),
+    "swap-dp": ((40, 1024, 2048), (mxgemm.SCHED_DP, 1, 0)),
+    "ksplit2": ((40, 1024, 2048), (mxgemm.SCHED_KSPLIT, 2, 0)),
+    "ksplit4": ((40, 1024, 2048), (mxgemm.SCHED_KSPLIT, 4, 0)),
 }
 
 
@@ -203,6 +229,10 @@ def _codes_case(fmt, A, SA, B, SB, K, path="auto"):
         assert "sched=splitk" in plan and "pair=0" in plan, plan
     elif "streamk" in path:
         assert "sched=streamk" in plan and "pair=0" in plan, plan
+    elif path.startswith("ksplit"):
+        assert "sched=ksplit" in plan and "ksplit=" + path[-1] in plan and "swap=1" in plan, plan
+    elif path == "swap-dp":
+        assert "sched=dp" in plan, plan
     if path.startswith("swap"):
         assert "swap=1" in plan, plan
     ref, _, mag = oracle.gemm(fmt, K, A, SA, B, SB)

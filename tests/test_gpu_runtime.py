@@ -53,13 +53,17 @@ def test_profiling_reports_repack_and_gemm_times():
 
 
 @pytest.mark.parametrize("fmt,M,N,K", [
-    (F4, 32, 1024, 2048),       # swapped decode tile
+    (F4, 32, 1024, 2048),       # swapped decode tiles, K split over clusters of two
+    (F8, 64, 1024, 4096),       # swapped decode tiles, K split over clusters of four
     (F8, 200, 640, 1536),       # 128-column tiles
     (F8, 512, 8192, 256),       # CTA-pair tiles
-], ids=["decode", "mid", "pair"])
+], ids=["decode", "decode-ksplit4", "mid", "pair"])
 def test_stalled_stage_times_out_and_handle_recovers(fmt, M, N, K):
     torch.cuda.set_device(0)
     h = mxgemm.Handle()
+    if M <= 64:
+        # every CTA of every cluster stalls: the reduction waits are never reached
+        assert "sched=ksplit" in h.describe(fmt, M, N, K)
     (qa, sa, qb, sb), (ref, mag) = _operands(fmt, M, N, K, seed=62)
     h.set_wait_limit(20_000_000)        # 20 ms per wait
     h.debug_inject(1)

@@ -127,20 +127,36 @@ def test_k_chunks_per_stage(fmt, M, K, kc):
     assert plan(fmt, M, 1024, K)["kc"] == kc
 
 
-def test_split_k_when_tiles_fill_at_most_a_quarter_of_the_gpu():
-    # 2 tiles of 128 x 32, 32 K steps: two-way split, FP32 partials of 128 x BN
+def test_cluster_split_for_decode_tiles_that_fill_at_most_half_the_gpu():
+    # the 64x4096x4096 decode shapes: 32 tiles, each K range over a cluster of
+    # four CTAs (every CTA >= 2 K steps), no global partials
+    for fmt in (F8, F4, mxgemm.FMT_BF16):
+        p = plan(fmt, 64, 4096, 4096)
+        assert (p["sched"], p["ksplit"], p["tiles"], p["workers"], p["grid"]) == ("ksplit", 4, 32, 128, 128), p
+        assert p["partial_bytes"] == 0
+    # 2 tiles, 32 K steps: four-way
     p = plan(F8, 32, 256, 8192)
+    assert (p["sched"], p["ksplit"], p["workers"]) == ("ksplit", 4, 8)
+    # 37..74 tiles: two-way; 2 K steps per CTA at least
+    p = plan(F8, 16, 128 * 60, 1024)
+    assert (p["sched"], p["ksplit"], p["workers"]) == ("ksplit", 2, 120) and p["kt"] == 4
+    # too few K steps: whole tiles
+    q = plan(F8, 32, 256, 512)
+    assert q["sched"] == "dp" and "ksplit" not in q
+    # more than half the GPU: whole tiles
+    for M, N, K in [(32, 14336, 4096), (16, 14336, 4096), (32, 4096 * 8, 8192)]:
+        r = plan(F8, M, N, K)
+        assert r["sched"] == "dp" and "ksplit" not in r, r
+
+
+def test_global_split_k_for_few_row_tiles_with_many_k_steps():
+    # not a decode tile (M > 64): 2 tiles of 128 x 128, 64 K steps: two-way
+    # split with FP32 partials of 128 x BN in global memory
+    p = plan(F8, 128, 256, 16384)
     assert p["sched"] == "splitk" and p["tiles"] == 2 and p["workers"] == 4 and p["grid"] == 4
     assert p["partial_bytes"] == 2 * p["workers"] * 128 * p["BN"] * 4
-    # too few K steps to pay for the fixup: whole tiles
-    q = plan(F8, 32, 256, 4096)
-    assert q["sched"] == "dp" and q["workers"] == q["tiles"] and q["partial_bytes"] == 0
-    # enough tiles: whole tiles
-    r = plan(F8, 32, 4096 * 8, 8192)
-    assert r["sched"] == "dp"
-    # the dense BF16 decode shape: 32 tiles, 32 K steps: split in two
-    b = plan(mxgemm.FMT_BF16, 64, 4096, 4096)
-    assert b["sched"] == "splitk" and b["workers"] == 64
+    q = plan(F8, 128, 256, 4096)           # 16 K steps: whole tiles
+    assert q["sched"] == "dp" and q["partial_bytes"] == 0
 
 
 def test_fused_scales_need_a_deep_one_cta_ring():
@@ -148,9 +164,9 @@ def test_fused_scales_need_a_deep_one_cta_ring():
                          (F8, 64, 4096, 4096), (F4, 64, 4096, 4096), (F8, 4096, 4096, 4096)]:
         p = plan(fmt, M, N, K)
         assert (p["scales"] == "fused") == (p["pair"] == 0 and p["stages"] >= 4), p
-    # the 64x4096x4096 decode shape: two chunks per stage, four stages, one launch, whole tiles
+    # the 64x4096x4096 decode shape: two chunks per stage, four stages, one launch
     p = plan(F8, 64, 4096, 4096)
-    assert p["kc"] == 2 and p["stages"] == 4 and p["scales"] == "fused" and p["sched"] == "dp"
+    assert p["kc"] == 2 and p["stages"] == 4 and p["scales"] == "fused" and p["sched"] == "ksplit"
 
 
 def test_plan_invariants_over_random_shapes():
@@ -181,6 +197,12 @@ def test_plan_invariants_over_random_shapes():
         assert p["stages"] >= 2
         if p["sched"] == "dp":
             assert p["workers"] == p["tiles"] and p["partial_bytes"] == 0
+        elif p["sched"] == "ksplit":
+            # one wave of clusters, each CTA of a cluster with >= 2 K steps
+            ks = p["ksplit"]
+            assert p["swap"] == 1 and p["BN"] <= 64 and ks in (2, 4)
+            assert p["workers"] == p["grid"] == p["tiles"] * ks <= sms and p["kt"] >= 2 * ks
+            assert p["partial_bytes"] == 0
         else:
             assert p["partial_bytes"] == 2 * p["workers"] * 128 * p["BN"] * 4
             assert p["workers"] <= p["tiles"] * p["kt"]

@@ -636,7 +636,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         }
         mbar_init(drain_bar, NM);
         mbar_init(go_bar, 1);
-        mbar_init(red_bar, kp.ksplit > 1 ? (kp.ksplit - 1) * 128 : 1);
+        mbar_init(red_bar, 1);
         *s_abort = 0;
         *s_last = 0;
         fence_mbar_init();
@@ -1137,10 +1137,12 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                     }
                 } else if (kp.ksplit > 1) {
                     // Cluster K split: one work unit per CTA, the tile's ranks
-                    // in one cluster.  Rank 0 hands its drained ring to the
-                    // others, which write their partial tiles into it and
-                    // arrive on its reduction barrier; rank 0 adds them in
-                    // rank order to its own accumulator and writes the tile.
+                    // in one cluster.  Rank 0 arms its reduction barrier for
+                    // the other ranks' partial tiles and hands them its
+                    // drained ring; they write their partials into it with
+                    // asynchronous stores that count their bytes on that
+                    // barrier; rank 0 adds them in rank order to its own
+                    // accumulator and writes the tile.
                     const uint32_t rank = w - g_first;
                     // the plan puts exactly one cluster on each tile; anything
                     // else would address partial slots that do not exist
@@ -1151,9 +1153,12 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                         if (etid == 0)
                             record_error(kp.error, kErrReduce, s_abort);
                     } else if (rank == 0) {
-                        if (etid == 0)
+                        if (etid == 0) {
+                            mbar_arrive_expect_tx(red_bar,
+                                                  static_cast<uint32_t>((kp.ksplit - 1) * C_::kRedSlot));
                             for (int r = 1; r < kp.ksplit; ++r)
                                 mbar_arrive_remote(go_bar, static_cast<uint32_t>(r));
+                        }
                         int got = 1;
                         if (lane == 0)
                             got = mbar_wait_cluster_parked(red_bar, 0, s_abort, kp.limit_ns);
@@ -1195,16 +1200,16 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                         if (go) {
                             const uint32_t dst =
                                 cluster_addr(sbase + C_::kRedOff + (rank - 1) * C_::kRedSlot, 0);
+                            const uint32_t rbar = cluster_addr(red_bar, 0);
 #pragma unroll 1
                             for (int c = 0; c < BN; c += CW) {
                                 float v[CW];
                                 load_acc(t_acc, c, v);
 #pragma unroll
                                 for (int j = 0; j < CW / 4; ++j)
-                                    st_cluster_v4(dst + ((c / 4 + j) * 128 + row) * 16, v[4 * j], v[4 * j + 1],
-                                                  v[4 * j + 2], v[4 * j + 3]);
+                                    st_async_v4(dst + ((c / 4 + j) * 128 + row) * 16, v[4 * j], v[4 * j + 1],
+                                                v[4 * j + 2], v[4 * j + 3], rbar);
                             }
-                            mbar_arrive_remote(red_bar, 0);
                         }
                     }
                 } else {

@@ -538,11 +538,14 @@ __device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t pa
     return ok != 0;
 }
 
-// 16-byte store into the shared memory of a CTA of this cluster (`addr` from
-// cluster_addr).
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d)
+// Asynchronous 16-byte store into the shared memory of a CTA of this
+// cluster whose completion counts 16 transaction bytes on the mbarrier `bar`
+// of that same CTA (both addresses from cluster_addr; PTX ISA st.async).
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t bar)
 {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     addr),
+                 "f"(a), "f"(b), "f"(c), "f"(d), "r"(bar)
                  : "memory");
 }
 

@@ -970,20 +970,20 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         bool tma_tile = false;                 // this tile's BF16 output may go out by TMA stores
 
         // The tile's accumulator is the sum of the NM MMA warps' accumulators.
+        // Two loads per wait: each load-and-wait round trip costs ~0.2 us.
         auto load_acc = [&](uint32_t t_acc, int c, float (&v)[CW]) {
-            uint32_t r[CW];
-            tmem_ld_cols<CW>(t_acc + c, r);
-            tmem_ld_wait();
+            uint32_t r0[CW], r1[CW];
 #pragma unroll
-            for (int j = 0; j < CW; ++j)
-                v[j] = __uint_as_float(r[j]);
-#pragma unroll
-            for (int m = 1; m < NM; ++m) {
-                tmem_ld_cols<CW>(t_acc + m * BN + c, r);
+            for (int m = 0; m < NM; m += 2) {
+                tmem_ld_cols<CW>(t_acc + m * BN + c, r0);
+                if (m + 1 < NM)
+                    tmem_ld_cols<CW>(t_acc + (m + 1) * BN + c, r1);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < CW; ++j)
-                    v[j] += __uint_as_float(r[j]);
+                for (int j = 0; j < CW; ++j) {
+                    const float x = __uint_as_float(r0[j]) + (m + 1 < NM ? __uint_as_float(r1[j]) : 0.0f);
+                    v[j] = m == 0 ? x : v[j] + x;
+                }
             }
         };
 
@@ -1137,11 +1137,13 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                     }
                 } else if (kp.ksplit > 1) {
                     // Cluster K split: one work unit per CTA, the tile's ranks
-                    // in one cluster.  Rank 0 arms its reduction barrier for
-                    // the other ranks' partial tiles and hands them its
-                    // drained ring; they write their partials into it with
-                    // asynchronous stores that count their bytes on that
-                    // barrier; rank 0 adds them in rank order to its own
+                    // in one cluster.  Every rank's ring is drained once its
+                    // accumulator is complete.  The other ranks stage their
+                    // FP32 partial tiles in their own rings; rank 0 arms its
+                    // reduction barrier for their bytes and tells them its
+                    // ring is free; each then pushes its partial into rank
+                    // 0's ring with one bulk copy that counts its bytes on
+                    // that barrier; rank 0 adds them in rank order to its own
                     // accumulator and writes the tile.
                     const uint32_t rank = w - g_first;
                     // the plan puts exactly one cluster on each tile; anything
@@ -1191,25 +1193,25 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                             }
                         }
                     } else {
-                        int go = 1;
-                        if (lane == 0)
-                            go = mbar_wait_cluster_parked(go_bar, 0, s_abort, kp.limit_ns);
-                        go = __shfl_sync(0xffffffffu, go, 0);
-                        if (!go && lane == 0)
-                            record_error(kp.error, kErrReduce, s_abort);
-                        if (go) {
-                            const uint32_t dst =
-                                cluster_addr(sbase + C_::kRedOff + (rank - 1) * C_::kRedSlot, 0);
-                            const uint32_t rbar = cluster_addr(red_bar, 0);
+                        float4 *mine = reinterpret_cast<float4 *>(smem + C_::kRedOff);
 #pragma unroll 1
-                            for (int c = 0; c < BN; c += CW) {
-                                float v[CW];
-                                load_acc(t_acc, c, v);
+                        for (int c = 0; c < BN; c += CW) {
+                            float v[CW];
+                            load_acc(t_acc, c, v);
 #pragma unroll
-                                for (int j = 0; j < CW / 4; ++j)
-                                    st_async_v4(dst + ((c / 4 + j) * 128 + row) * 16, v[4 * j], v[4 * j + 1],
-                                                v[4 * j + 2], v[4 * j + 3], rbar);
-                            }
+                            for (int j = 0; j < CW / 4; ++j)
+                                mine[(c / 4 + j) * 128 + row] =
+                                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                        }
+                        fence_proxy_async_smem();       // the copy engine reads what the threads wrote
+                        named_bar_sync(1, 128);
+                        if (etid == 0) {
+                            if (mbar_wait_cluster_parked(go_bar, 0, s_abort, kp.limit_ns))
+                                bulk_copy_to_cluster(cluster_addr(sbase + C_::kRedOff + (rank - 1) * C_::kRedSlot, 0),
+                                                     sbase + C_::kRedOff, static_cast<uint32_t>(C_::kRedSlot),
+                                                     cluster_addr(red_bar, 0));
+                            else
+                                record_error(kp.error, kErrReduce, s_abort);
                         }
                     }
                 } else {

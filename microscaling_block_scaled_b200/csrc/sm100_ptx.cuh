@@ -538,14 +538,15 @@ __device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t pa
     return ok != 0;
 }
 
-// Asynchronous 16-byte store into the shared memory of a CTA of this
-// cluster whose completion counts 16 transaction bytes on the mbarrier `bar`
-// of that same CTA (both addresses from cluster_addr; PTX ISA st.async).
-__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t bar)
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory to
+// the shared memory of a CTA of this cluster; its completion counts the
+// bytes on the mbarrier `bar` of the destination CTA (dst and bar from
+// cluster_addr; PTX ISA cp.async.bulk, shared::cta to shared::cluster).
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar)
 {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                     addr),
-                 "f"(a), "f"(b), "f"(c), "f"(d), "r"(bar)
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst),
+                 "r"(src), "r"(bytes), "r"(bar)
                  : "memory");
 }
 

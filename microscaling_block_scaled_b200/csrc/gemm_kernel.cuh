@@ -1161,9 +1161,11 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                             for (int r = 1; r < kp.ksplit; ++r)
                                 mbar_arrive_remote(go_bar, static_cast<uint32_t>(r));
                         }
+                        // the CTA's other roles are done: spin rather than park
+                        // (a parked wait wakes late on a remote completion)
                         int got = 1;
                         if (lane == 0)
-                            got = mbar_wait_cluster_parked(red_bar, 0, s_abort, kp.limit_ns);
+                            got = mbar_wait_cluster_bounded(red_bar, 0, s_abort, kp.limit_ns);
                         got = __shfl_sync(0xffffffffu, got, 0);
                         if (!got && lane == 0)
                             record_error(kp.error, kErrReduce, s_abort);
@@ -1206,7 +1208,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                         fence_proxy_async_smem();       // the copy engine reads what the threads wrote
                         named_bar_sync(1, 128);
                         if (etid == 0) {
-                            if (mbar_wait_cluster_parked(go_bar, 0, s_abort, kp.limit_ns))
+                            if (mbar_wait_cluster_bounded(go_bar, 0, s_abort, kp.limit_ns))
                                 bulk_copy_to_cluster(cluster_addr(sbase + C_::kRedOff + (rank - 1) * C_::kRedSlot, 0),
                                                      sbase + C_::kRedOff, static_cast<uint32_t>(C_::kRedSlot),
                                                      cluster_addr(red_bar, 0));

@@ -89,7 +89,7 @@ enum {
     MXGEMM_SCHED_SPLITK = 2,   /* each tile split into `splits` equal K ranges */
     MXGEMM_SCHED_STREAMK = 3,  /* K iterations of all tiles split evenly over the SMs */
     MXGEMM_SCHED_KSPLIT = 4    /* decode tiles: each tile's K range split over a cluster of
-                                  `splits` (2-4) CTAs, summed in distributed shared memory */
+                                  `splits` (2 or 4) CTAs, summed in distributed shared memory */
 };
 
 /* Create a handle bound to the current CUDA device.  The device must be an
@@ -273,9 +273,9 @@ MXGEMM_API int mxgemm_quantize_bf16(int fmt, int64_t R, int64_t K, const void *X
 
 /* Force a schedule for later mxgemm_run / mxgemm_gemm calls on this handle.
  * splits is used by MXGEMM_SCHED_SPLITK (>= 1) and MXGEMM_SCHED_KSPLIT
- * (clamped to 2-4; shapes that are not decode tiles, or whose clusters would
- * not all fit on the GPU at once, take MXGEMM_SCHED_SPLITK instead); workers
- * by MXGEMM_SCHED_STREAMK (0 = number of SMs). */
+ * (2 or 4; 3 takes 2; shapes that are not decode tiles, or whose clusters
+ * would not all fit on the GPU at once, take MXGEMM_SCHED_SPLITK instead);
+ * workers by MXGEMM_SCHED_STREAMK (0 = number of SMs). */
 MXGEMM_API int mxgemm_set_schedule(mxgemm_handle h, int schedule, int splits, int workers);
 
 /* Force the number of 128-byte K chunks each pipeline stage of later GEMMs

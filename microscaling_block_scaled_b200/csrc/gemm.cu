@@ -173,9 +173,9 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
             s = 1;
         }
     } else if (s == 4) {
-        // forced cluster split: 2 to 4 CTAs per tile, decode tiles only, all
-        // clusters in one wave; otherwise the global-memory split
-        const int64_t c = splits < 2 ? 2 : (splits > 4 ? 4 : splits);
+        // forced cluster split: 2 or 4 CTAs per tile (3 takes 2), decode tiles
+        // only, all clusters in one wave; otherwise the global-memory split
+        const int64_t c = splits >= 4 ? 4 : 2;
         if (pl.swap && pl.tiles * c <= sms && pl.kt >= c) {
             ks = c;
         } else {

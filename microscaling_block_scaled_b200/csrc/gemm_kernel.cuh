@@ -132,13 +132,19 @@ struct Cfg {
     static constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
     static constexpr int kOffOut = (kOffSFB + kStages * kSFBBytes + 1023) / 1024 * 1024;
     static constexpr int kOffBar = kOffOut + 2 * kOutBytes;
-    // Cluster K split: rank 0 of a cluster sums the other ranks' partial
-    // tiles, which they write into its ring once it has drained (FP32, 16-byte
-    // column groups: group q of row r at (q * 128 + r) * 16).  The first 16 KB
-    // stay free for the output staging of narrow tiles.
+    // Cluster K split (decode tiles, BN <= 64): rank r of a cluster of S = 2
+    // or 4 CTAs owns the tile rows of 4/S of the epilogue warps' 32-row TMEM
+    // lane quarters.  The other ranks ship their partials of those rows into
+    // its drained ring (FP32, 16-byte column groups: group g of quarter row i
+    // at (g * 32 + i) * 16): incoming quarters from kRedOff (slot s, quarter
+    // j at (s * 4/S + j) * kQuadBytes), this rank's outgoing quarters from
+    // kRedOut, per-quarter output staging (two chunks each) from kRedStage.
     static constexpr int kRedOff = kOffA + 16384;
-    static constexpr int kRedSlot = 128 * BN * 4;
-    static constexpr int kMaxKsplit = BN <= 64 ? 4 : 1;
+    static constexpr int kQuadBytes = 32 * BN * 4;
+    static constexpr int kRedOut = kRedOff + 3 * kQuadBytes;
+    static constexpr int kRedStage = kRedOut + 4 * kQuadBytes;
+    static constexpr int kQStageBytes = kCW * 32 * 2;
+    static constexpr bool kCanKsplit = BN <= 64;
     static constexpr int kNumBars = 2 * kStages + 2 * kNumAcc + 3;   // + drain, go-ahead, reduction
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 64 + 1024;   // + alignment slack
@@ -150,7 +156,7 @@ struct Cfg {
     static_assert(kBChunk % 1024 == 0, "tiles must keep 1024-byte alignment");
     static_assert(kStaged || 2 * kChunkOutBytes <= kABytes, "ring stage 0 holds two output chunks");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-    static_assert(kRedOff + (kMaxKsplit - 1) * kRedSlot <= kOffOut, "partial tiles of a cluster split fit the ring");
+    static_assert(!kCanKsplit || kRedStage + 8 * kQStageBytes <= kOffOut, "cluster split buffers fit the ring");
 };
 
 // Instruction descriptor of the block-scaled MMA (PTX ISA, instruction
@@ -590,7 +596,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
     auto accf_bar = [&](int a) { return bar0 + 8u * (2 * S + a); };
     auto acce_bar = [&](int a) { return bar0 + 8u * (2 * S + C_::kNumAcc + a); };
     const uint32_t drain_bar = bar0 + 8u * (2 * S + 2 * C_::kNumAcc);
-    const uint32_t go_bar = drain_bar + 8u;       // cluster K split: rank 0's ring is free
+    const uint32_t go_bar = drain_bar + 8u;       // cluster K split: every other rank's ring is free
     const uint32_t red_bar = drain_bar + 16u;     // cluster K split: the other ranks' partials are in
     volatile uint32_t *s_tmem = reinterpret_cast<volatile uint32_t *>(smem + C_::kOffMisc);
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + C_::kOffMisc + 4);
@@ -635,7 +641,7 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
             mbar_init(acce_bar(a), 4);
         }
         mbar_init(drain_bar, NM);
-        mbar_init(go_bar, 1);
+        mbar_init(go_bar, kp.ksplit > 1 ? kp.ksplit - 1 : 1);
         mbar_init(red_bar, 1);
         *s_abort = 0;
         *s_last = 0;
@@ -1136,30 +1142,59 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                         emit(v, tc, tc.qcol + c);
                     }
                 } else if (kp.ksplit > 1) {
-                    // Cluster K split: one work unit per CTA, the tile's ranks
-                    // in one cluster.  Every rank's ring is drained once its
-                    // accumulator is complete.  The other ranks stage their
-                    // FP32 partial tiles in their own rings; rank 0 arms its
-                    // reduction barrier for their bytes and tells them its
-                    // ring is free; each then pushes its partial into rank
-                    // 0's ring with one bulk copy that counts its bytes on
-                    // that barrier; rank 0 adds them in rank order to its own
-                    // accumulator and writes the tile.
+                    // Cluster K split, reduced by scatter: one work unit per
+                    // CTA, the tile's ranks in one cluster.  A rank's ring is
+                    // drained once its accumulator is complete; it then arms
+                    // its reduction barrier for the partials of its rows and
+                    // tells the other ranks.  Each warp quarter whose rows
+                    // another rank owns stages its FP32 partial in its own
+                    // ring and pushes it there with one bulk copy that counts
+                    // its bytes on the owner's barrier.  The owner's quarters
+                    // add the partials in rank order and write their rows.
+                    const uint32_t S = static_cast<uint32_t>(kp.ksplit);
                     const uint32_t rank = w - g_first;
-                    // the plan puts exactly one cluster on each tile; anything
-                    // else would address partial slots that do not exist
-                    const bool shape_ok = g_first % static_cast<uint32_t>(kp.ksplit) == 0 &&
-                                          g_last - g_first + 1 == static_cast<uint32_t>(kp.ksplit) &&
-                                          kp.ksplit <= C_::kMaxKsplit;
+                    const uint32_t qpr = 4u / (S == 4u ? 4u : 2u);      // lane quarters per rank
+                    const uint32_t owner = static_cast<uint32_t>(quad) / qpr;
+                    // the plan puts exactly one cluster of 2 or 4 on each tile;
+                    // anything else would address buffers that do not exist
+                    const bool shape_ok = C_::kCanKsplit && (S == 2u || S == 4u) && g_first % S == 0 &&
+                                          g_last - g_first + 1 == S;
                     if (!shape_ok) {
-                        if (etid == 0)
+                        if (lane == 0)
                             record_error(kp.error, kErrReduce, s_abort);
-                    } else if (rank == 0) {
-                        if (etid == 0) {
+                    } else if (owner != rank) {
+                        float4 *out = reinterpret_cast<float4 *>(smem + C_::kRedOut + quad * C_::kQuadBytes);
+#pragma unroll 1
+                        for (int c = 0; c < BN; c += CW) {
+                            float v[CW];
+                            load_acc(t_acc, c, v);
+#pragma unroll
+                            for (int j = 0; j < CW / 4; ++j)
+                                out[(c / 4 + j) * 32 + lane] =
+                                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                        }
+                        fence_proxy_async_smem();       // the copy engine reads what the lanes wrote
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (mbar_wait_cluster_bounded(go_bar, 0, s_abort, kp.limit_ns)) {
+                                const uint32_t slot = rank < owner ? rank : rank - 1;
+                                const uint32_t dst =
+                                    sbase + C_::kRedOff + (slot * qpr + (quad - owner * qpr)) * C_::kQuadBytes;
+                                bulk_copy_to_cluster(cluster_addr(dst, owner),
+                                                     sbase + C_::kRedOut + quad * C_::kQuadBytes,
+                                                     static_cast<uint32_t>(C_::kQuadBytes),
+                                                     cluster_addr(red_bar, owner));
+                            } else {
+                                record_error(kp.error, kErrReduce, s_abort);
+                            }
+                        }
+                    } else {
+                        if (lane == 0 && static_cast<uint32_t>(quad) == rank * qpr) {
                             mbar_arrive_expect_tx(red_bar,
-                                                  static_cast<uint32_t>((kp.ksplit - 1) * C_::kRedSlot));
-                            for (int r = 1; r < kp.ksplit; ++r)
-                                mbar_arrive_remote(go_bar, static_cast<uint32_t>(r));
+                                                  static_cast<uint32_t>((S - 1) * qpr * C_::kQuadBytes));
+                            for (uint32_t o = 0; o < S; ++o)
+                                if (o != rank)
+                                    mbar_arrive_remote(go_bar, o);
                         }
                         // the CTA's other roles are done: spin rather than park
                         // (a parked wait wakes late on a remote completion)
@@ -1172,48 +1207,62 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                         // nothing more arrives here: the cluster may finish
                         cluster_arrive();
                         cl_arrived = true;
-                        if (!named_bar_or(1, 128, got ? 0 : 1)) {
+                        if (got) {
+                            const uint32_t qj = static_cast<uint32_t>(quad) - rank * qpr;
+                            uint32_t nchunk = 0;
 #pragma unroll 1
                             for (int c = 0; c < BN; c += CW) {
-                                float v[CW];
-                                load_acc(t_acc, c, v);
-                                for (int r = 1; r < kp.ksplit; ++r) {
+                                float own[CW], v[CW];
+                                load_acc(t_acc, c, own);
+                                for (uint32_t s = 0; s < S; ++s) {
+                                    if (s == rank) {
+#pragma unroll
+                                        for (int j = 0; j < CW; ++j)
+                                            v[j] = s == 0 ? own[j] : v[j] + own[j];
+                                        continue;
+                                    }
+                                    const uint32_t slot = s < rank ? s : s - 1;
                                     const float4 *src = reinterpret_cast<const float4 *>(
-                                        smem + C_::kRedOff + (r - 1) * C_::kRedSlot);
+                                        smem + C_::kRedOff + (slot * qpr + qj) * C_::kQuadBytes);
 #pragma unroll
                                     for (int j = 0; j < CW / 4; ++j) {
-                                        const float4 x = src[(c / 4 + j) * 128 + row];
-                                        v[4 * j + 0] += x.x;
-                                        v[4 * j + 1] += x.y;
-                                        v[4 * j + 2] += x.z;
-                                        v[4 * j + 3] += x.w;
+                                        const float4 x = src[(c / 4 + j) * 32 + lane];
+                                        v[4 * j + 0] = s == 0 ? x.x : v[4 * j + 0] + x.x;
+                                        v[4 * j + 1] = s == 0 ? x.y : v[4 * j + 1] + x.y;
+                                        v[4 * j + 2] = s == 0 ? x.z : v[4 * j + 2] + x.z;
+                                        v[4 * j + 3] = s == 0 ? x.w : v[4 * j + 3] + x.w;
                                     }
                                 }
                                 if (kp.has_ops)
                                     apply_ops(v, p, tc.plim, tc.qcol + c);
-                                emit(v, tc, tc.qcol + c);
-                            }
-                        }
-                    } else {
-                        float4 *mine = reinterpret_cast<float4 *>(smem + C_::kRedOff);
-#pragma unroll 1
-                        for (int c = 0; c < BN; c += CW) {
-                            float v[CW];
-                            load_acc(t_acc, c, v);
+                                if (kp.qfmt >= 0) {
+                                    emit_q(v, p, tc.plim, tc.qcol + c);
+                                } else if (!tma_tile) {
+                                    const OutView o{kp.C, kp.ldc, tc.plim, kp.Q, kp.swap};
+                                    store_bf16<CW>(o, p, tc.qcol + c, v);
+                                } else {
+                                    // this quarter's 32 output columns: a [CW][32]
+                                    // BF16 block and a TMA store (the map's box)
+                                    uint8_t *buf = smem + C_::kRedStage + (quad * 2 + (nchunk & 1u)) * C_::kQStageBytes;
+                                    if (lane == 0)
+                                        bulk_wait_group_read<1>();
+                                    __syncwarp();
+                                    __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(buf) + lane;
 #pragma unroll
-                            for (int j = 0; j < CW / 4; ++j)
-                                mine[(c / 4 + j) * 128 + row] =
-                                    make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                        }
-                        fence_proxy_async_smem();       // the copy engine reads what the threads wrote
-                        named_bar_sync(1, 128);
-                        if (etid == 0) {
-                            if (mbar_wait_cluster_bounded(go_bar, 0, s_abort, kp.limit_ns))
-                                bulk_copy_to_cluster(cluster_addr(sbase + C_::kRedOff + (rank - 1) * C_::kRedSlot, 0),
-                                                     sbase + C_::kRedOff, static_cast<uint32_t>(C_::kRedSlot),
-                                                     cluster_addr(red_bar, 0));
-                            else
-                                record_error(kp.error, kErrReduce, s_abort);
+                                    for (int j = 0; j < CW; ++j)
+                                        dst[j * 32] = __float2bfloat16_rn(v[j]);
+                                    fence_proxy_async_smem();
+                                    __syncwarp();
+                                    if (lane == 0) {
+                                        tma_store_2d(&tmC, smem_u32(buf), static_cast<int32_t>(tc.prow + quad * 32),
+                                                     static_cast<int32_t>(tc.qcol + c));
+                                        bulk_commit_group();
+                                    }
+                                    ++nchunk;
+                                }
+                            }
+                            if (lane == 0)
+                                bulk_wait_group<0>();
                         }
                     }
                 } else {
@@ -1348,8 +1397,10 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     const bool quantised = b.epi.qfmt >= 0;
     const int tma_store = (pl.N % 8 == 0 && !quantised) ? 1 : 0;
     void *Cbase = quantised ? static_cast<void *>(b.epi.Cq) : b.C;
-    const bool okC = tma_store ? (pl.swap ? make_output_map(&tmC, Cbase, pl.M, pl.N, 128, C_::kCW)
-                                          : make_output_map(&tmC, Cbase, pl.M, pl.N, C_::kCW, 128))
+    // (a cluster K split stores each 32-row lane quarter of a tile on its own)
+    const int box_p = pl.ksplit > 1 ? 32 : 128;
+    const bool okC = tma_store ? (pl.swap ? make_output_map(&tmC, Cbase, pl.M, pl.N, box_p, C_::kCW)
+                                          : make_output_map(&tmC, Cbase, pl.M, pl.N, C_::kCW, box_p))
                                : make_output_map(&tmC, Cbase, 1, 8, 8, 1);
     if (!okC)
         return cudaErrorInvalidValue;
@@ -1408,7 +1459,8 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     kp.tail_first = 0;
     kp.tail_split = 1;
     kp.ksplit = static_cast<int>(pl.ksplit);
-    if (pl.ksplit > 1 && (pl.ksplit > C_::kMaxKsplit || pl.grid != pl.workers || pl.grid % pl.ksplit != 0))
+    if (pl.ksplit > 1 && (!C_::kCanKsplit || !pl.swap || (pl.ksplit != 2 && pl.ksplit != 4) ||
+                          pl.grid != pl.workers || pl.grid % pl.ksplit != 0))
         return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));

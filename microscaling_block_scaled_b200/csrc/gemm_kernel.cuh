@@ -1189,12 +1189,20 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                             }
                         }
                     } else {
-                        if (lane == 0 && static_cast<uint32_t>(quad) == rank * qpr) {
-                            mbar_arrive_expect_tx(red_bar,
-                                                  static_cast<uint32_t>((S - 1) * qpr * C_::kQuadBytes));
-                            for (uint32_t o = 0; o < S; ++o)
-                                if (o != rank)
-                                    mbar_arrive_remote(go_bar, o);
+                        if (static_cast<uint32_t>(quad) == rank * qpr) {
+                            // lane 0 arms for the incoming bytes (a copy that
+                            // lands first only drives the byte count below
+                            // zero until then); lanes 1.. each tell one other
+                            // rank.  The go-ahead carries no data: this ring
+                            // was last touched by the TMA and the MMAs, both
+                            // complete, so a relaxed arrive suffices.
+                            if (lane == 0)
+                                mbar_arrive_expect_tx(red_bar,
+                                                      static_cast<uint32_t>((S - 1) * qpr * C_::kQuadBytes));
+                            else if (static_cast<uint32_t>(lane) < S)
+                                mbar_arrive_remote_relaxed(go_bar, static_cast<uint32_t>(lane) - 1 < rank
+                                                                       ? static_cast<uint32_t>(lane) - 1
+                                                                       : static_cast<uint32_t>(lane));
                         }
                         // the CTA's other roles are done: spin rather than park
                         // (a parked wait wakes late on a remote completion)

@@ -523,6 +523,20 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar, uint32_t rank)
         : "memory");
 }
 
+// A relaxed arrive on the mbarrier at shared offset `bar` of CTA `rank`: a
+// signal that orders none of the thread's memory operations, so it does not
+// wait for them to drain (a release arrive to another CTA costs ~0.5-1 us
+// after the epilogue's memory traffic).
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar, uint32_t rank)
+{
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(bar),
+        "r"(rank)
+        : "memory");
+}
+
 // Non-blocking test with cluster-scope acquire (for phases completed by
 // arrivals from the other CTA of the pair).
 __device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity)

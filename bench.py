@@ -61,7 +61,8 @@ def parse():
     ap.add_argument("--reps", type=int, default=20, help="extra replays of the step graph for the spread")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--schedule", default="auto",
-                    help="planner override: auto, dp, splitk:S (S K ranges per tile) or streamk:W (W workers)")
+                    help="planner override: auto, dp, splitk:S (S K ranges per tile), streamk:W (W workers) "
+                         "or ksplit:2|4 (each tile's K range over a cluster of 2 or 4 CTAs)")
     ap.add_argument("--kchunks", type=int, default=0, choices=[0, 1, 2, 4],
                     help="128-byte K chunks per ring stage (0: the planner's choice)")
     return ap.parse_args()
@@ -79,7 +80,9 @@ def parse_schedule(text):
         return mxgemm.SCHED_SPLITK, int(arg), 0
     if kind == "streamk" and arg.isdigit() and int(arg) >= 1:
         return mxgemm.SCHED_STREAMK, 1, int(arg)
-    raise SystemExit("--schedule: auto, dp, splitk:S or streamk:W, not %r" % text)
+    if kind == "ksplit" and arg in ("2", "4"):
+        return mxgemm.SCHED_KSPLIT, int(arg), 0
+    raise SystemExit("--schedule: auto, dp, splitk:S, streamk:W or ksplit:2|4, not %r" % text)
 
 
 def override_label(args):

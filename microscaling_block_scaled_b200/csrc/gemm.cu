@@ -150,14 +150,16 @@ GemmPlan make_plan(int fmt, int64_t M, int64_t N, int64_t K, int num_sms, int sc
     if (s == 0) {
         // auto: decode tiles (swapped, at most 64 columns) that fill at most
         // half the GPU split each tile's K range over a cluster of 4 or 2
-        // CTAs, every CTA with at least two K steps; the partial tiles are
-        // summed through distributed shared memory, so the split costs no
-        // global round trip.  (MXFP8 64x4096x4096 runs 32 tiles: whole tiles
-        // leave 116 SMs idle and take 15 us per chained step, a split with
-        // the partials summed through global memory 15.7 us.)
+        // CTAs, every CTA with at least four K steps (the hand-off of the
+        // partial tiles costs ~3 us, which fewer steps do not repay); the
+        // partials are summed through distributed shared memory, so the
+        // split costs no global round trip.  Chained steps, 64x4096x4096:
+        // MXFP8 (16 K steps) 14.7 us whole, 12.4 us in clusters of 2 or 4;
+        // MXFP4 (8 K steps) 11.9 us whole, 10.2 us in 2, 11.7 us in 4; BF16
+        // (32 K steps) 20.2 us whole, 14.3 us in 2, 13.7 us in 4.
         if (pl.swap)
             for (int64_t c = 4; c >= 2; c /= 2)
-                if (pl.tiles * c <= sms && pl.kt >= 2 * c) {
+                if (pl.tiles * c <= sms && pl.kt >= 4 * c) {
                     ks = c;
                     break;
                 }

@@ -80,7 +80,8 @@ def test_schedule_overrides_parse_and_key_the_traffic():
     assert bench.parse_schedule("dp") == (mxgemm.SCHED_DP, 1, 0)
     assert bench.parse_schedule("splitk:3") == (mxgemm.SCHED_SPLITK, 3, 0)
     assert bench.parse_schedule("streamk:148") == (mxgemm.SCHED_STREAMK, 1, 148)
-    for bad in ("splitk", "splitk:0", "streamk:x", "dp:2", "fast"):
+    assert bench.parse_schedule("ksplit:4") == (mxgemm.SCHED_KSPLIT, 4, 0)
+    for bad in ("splitk", "splitk:0", "streamk:x", "dp:2", "fast", "ksplit:3", "ksplit"):
         with pytest.raises(SystemExit):
             bench.parse_schedule(bad)
 

@@ -53,7 +53,7 @@ def test_profiling_reports_repack_and_gemm_times():
 
 
 @pytest.mark.parametrize("fmt,M,N,K", [
-    (F4, 32, 1024, 2048),       # swapped decode tiles, K split over clusters of two
+    (F4, 32, 1024, 4096),       # swapped decode tiles, K split over clusters of two
     (F8, 64, 1024, 4096),       # swapped decode tiles, K split over clusters of four
     (F8, 200, 640, 1536),       # 128-column tiles
     (F8, 512, 8192, 256),       # CTA-pair tiles

@@ -128,21 +128,22 @@ def test_k_chunks_per_stage(fmt, M, K, kc):
 
 
 def test_cluster_split_for_decode_tiles_that_fill_at_most_half_the_gpu():
-    # the 64x4096x4096 decode shapes: 32 tiles, each K range over a cluster of
-    # four CTAs (every CTA >= 2 K steps), no global partials
-    for fmt in (F8, F4, mxgemm.FMT_BF16):
+    # the 64x4096x4096 decode shapes: 32 tiles, each K range over a cluster
+    # of CTAs with at least four K steps each, no global partials
+    for fmt, kt, ks in ((F8, 16, 4), (F4, 8, 2), (mxgemm.FMT_BF16, 32, 4)):
         p = plan(fmt, 64, 4096, 4096)
-        assert (p["sched"], p["ksplit"], p["tiles"], p["workers"], p["grid"]) == ("ksplit", 4, 32, 128, 128), p
-        assert p["partial_bytes"] == 0
+        assert (p["sched"], p["ksplit"], p["tiles"], p["kt"]) == ("ksplit", ks, 32, kt), p
+        assert p["workers"] == p["grid"] == 32 * ks and p["partial_bytes"] == 0
     # 2 tiles, 32 K steps: four-way
     p = plan(F8, 32, 256, 8192)
     assert (p["sched"], p["ksplit"], p["workers"]) == ("ksplit", 4, 8)
-    # 37..74 tiles: two-way; 2 K steps per CTA at least
-    p = plan(F8, 16, 128 * 60, 1024)
-    assert (p["sched"], p["ksplit"], p["workers"]) == ("ksplit", 2, 120) and p["kt"] == 4
-    # too few K steps: whole tiles
-    q = plan(F8, 32, 256, 512)
-    assert q["sched"] == "dp" and "ksplit" not in q
+    # 37..74 tiles: two-way
+    p = plan(F8, 16, 128 * 60, 2048)
+    assert (p["sched"], p["ksplit"], p["workers"]) == ("ksplit", 2, 120) and p["kt"] == 8
+    # fewer than four K steps per CTA: whole tiles
+    for M, N, K in [(32, 256, 512), (16, 128 * 60, 1024), (32, 1024, 1024)]:
+        q = plan(F8, M, N, K)
+        assert q["sched"] == "dp" and "ksplit" not in q, q
     # more than half the GPU: whole tiles
     for M, N, K in [(32, 14336, 4096), (16, 14336, 4096), (32, 4096 * 8, 8192)]:
         r = plan(F8, M, N, K)
@@ -201,7 +202,7 @@ def test_plan_invariants_over_random_shapes():
             # one wave of clusters, each CTA of a cluster with >= 2 K steps
             ks = p["ksplit"]
             assert p["swap"] == 1 and p["BN"] <= 64 and ks in (2, 4)
-            assert p["workers"] == p["grid"] == p["tiles"] * ks <= sms and p["kt"] >= 2 * ks
+            assert p["workers"] == p["grid"] == p["tiles"] * ks <= sms and p["kt"] >= 4 * ks
             assert p["partial_bytes"] == 0
         else:
             assert p["partial_bytes"] == 2 * p["workers"] * 128 * p["BN"] * 4

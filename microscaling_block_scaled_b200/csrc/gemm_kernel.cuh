@@ -143,7 +143,7 @@ struct Cfg {
     static constexpr int kQuadBytes = 32 * BN * 4;
     static constexpr int kRedOut = kRedOff + 3 * kQuadBytes;
     static constexpr int kRedStage = kRedOut + 4 * kQuadBytes;
-    static constexpr int kQStageBytes = kCW * 32 * 2;
+    static constexpr int kQStageBytes = BN * 32 * 2;          // a lane quarter's [BN][32] BF16 output
     static constexpr bool kCanKsplit = BN <= 64;
     static constexpr int kNumBars = 2 * kStages + 2 * kNumAcc + 3;   // + drain, go-ahead, reduction
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -156,7 +156,7 @@ struct Cfg {
     static_assert(kBChunk % 1024 == 0, "tiles must keep 1024-byte alignment");
     static_assert(kStaged || 2 * kChunkOutBytes <= kABytes, "ring stage 0 holds two output chunks");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-    static_assert(!kCanKsplit || kRedStage + 8 * kQStageBytes <= kOffOut, "cluster split buffers fit the ring");
+    static_assert(!kCanKsplit || kRedStage + 4 * kQStageBytes <= kOffOut, "cluster split buffers fit the ring");
 };
 
 // Instruction descriptor of the block-scaled MMA (PTX ISA, instruction
@@ -1217,7 +1217,9 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                         cl_arrived = true;
                         if (got) {
                             const uint32_t qj = static_cast<uint32_t>(quad) - rank * qpr;
-                            uint32_t nchunk = 0;
+                            // BF16 output through this quarter's [BN][32] staging
+                            // block and one TMA store (the map's box)
+                            uint8_t *stage = smem + C_::kRedStage + quad * C_::kQStageBytes;
 #pragma unroll 1
                             for (int c = 0; c < BN; c += CW) {
                                 float own[CW], v[CW];
@@ -1249,28 +1251,22 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                                     const OutView o{kp.C, kp.ldc, tc.plim, kp.Q, kp.swap};
                                     store_bf16<CW>(o, p, tc.qcol + c, v);
                                 } else {
-                                    // this quarter's 32 output columns: a [CW][32]
-                                    // BF16 block and a TMA store (the map's box)
-                                    uint8_t *buf = smem + C_::kRedStage + (quad * 2 + (nchunk & 1u)) * C_::kQStageBytes;
-                                    if (lane == 0)
-                                        bulk_wait_group_read<1>();
-                                    __syncwarp();
-                                    __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(buf) + lane;
+                                    __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(stage) + c * 32 + lane;
 #pragma unroll
                                     for (int j = 0; j < CW; ++j)
                                         dst[j * 32] = __float2bfloat16_rn(v[j]);
-                                    fence_proxy_async_smem();
-                                    __syncwarp();
-                                    if (lane == 0) {
-                                        tma_store_2d(&tmC, smem_u32(buf), static_cast<int32_t>(tc.prow + quad * 32),
-                                                     static_cast<int32_t>(tc.qcol + c));
-                                        bulk_commit_group();
-                                    }
-                                    ++nchunk;
                                 }
                             }
-                            if (lane == 0)
-                                bulk_wait_group<0>();
+                            if (kp.qfmt < 0 && tma_tile) {
+                                fence_proxy_async_smem();
+                                __syncwarp();
+                                if (lane == 0) {
+                                    tma_store_2d(&tmC, smem_u32(stage), static_cast<int32_t>(tc.prow + quad * 32),
+                                                 static_cast<int32_t>(tc.qcol));
+                                    bulk_commit_group();
+                                    bulk_wait_group_read<0>();
+                                }
+                            }
                         }
                     }
                 } else {
@@ -1346,9 +1342,10 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                 it += ke - kb;
             }
         }
-        // Output stores must finish reading shared memory before the CTA exits.
+        // Output stores must finish reading shared memory before the CTA
+        // exits; the kernel's completion covers their writes.
         if (etid == 0)
-            bulk_wait_group<0>();
+            bulk_wait_group_read<0>();
     }
 
     if (kp.ksplit > 1 && !cl_arrived)
@@ -1405,10 +1402,11 @@ cudaError_t launch_t(const GemmPlan &pl, const GemmBuffers &b, uint64_t limit_ns
     const bool quantised = b.epi.qfmt >= 0;
     const int tma_store = (pl.N % 8 == 0 && !quantised) ? 1 : 0;
     void *Cbase = quantised ? static_cast<void *>(b.epi.Cq) : b.C;
-    // (a cluster K split stores each 32-row lane quarter of a tile on its own)
-    const int box_p = pl.ksplit > 1 ? 32 : 128;
-    const bool okC = tma_store ? (pl.swap ? make_output_map(&tmC, Cbase, pl.M, pl.N, box_p, C_::kCW)
-                                          : make_output_map(&tmC, Cbase, pl.M, pl.N, C_::kCW, box_p))
+    // (a cluster K split stores each 32-row lane quarter of a tile, all its
+    // BN columns, with one box)
+    const bool okC = tma_store ? (pl.ksplit > 1 ? make_output_map(&tmC, Cbase, pl.M, pl.N, 32, BN)
+                                  : pl.swap    ? make_output_map(&tmC, Cbase, pl.M, pl.N, 128, C_::kCW)
+                                               : make_output_map(&tmC, Cbase, pl.M, pl.N, C_::kCW, 128))
                                : make_output_map(&tmC, Cbase, 1, 8, 8, 1);
     if (!okC)
         return cudaErrorInvalidValue;

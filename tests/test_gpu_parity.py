@@ -99,13 +99,13 @@ def test_gemm_forced_schedules(fmt, sched, M, N, K):
 @pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
 @pytest.mark.parametrize("M,N,K", [
     (1, 4096, 4096), (9, 640, 4096), (33, 300, 4096), (64, 4104, 4096), (48, 1000, 8192),
-    (16, 128 * 60, 4096), (64, 4096, 4096), (17, 256, 4608), (17, 256, 4160),
+    (16, 128 * 60, 4096), (64, 4096, 4096), (17, 256, 4608), (17, 256, 4224),
 ])
 def test_gemm_cluster_k_split(fmt, M, N, K):
     """Decode tiles that fill at most half the GPU split each tile's K range
     over a cluster of CTAs; the other ranks write their FP32 partial tiles
     into rank 0's drained ring through distributed shared memory and rank 0
-    adds them.  Ragged N, K tails (K = 4160: 32.5 MXFP8 chunks, 16.25 MXFP4
+    adds them.  Ragged N, K tails (K = 4224: 33 MXFP8 chunks, two per stage; 16.5 MXFP4
     chunks per row) and one tile column of 1 to 64 rows."""
     h = handle()
     plan = h.describe(fmt, M, N, K)

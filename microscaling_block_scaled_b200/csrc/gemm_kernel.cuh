@@ -1150,7 +1150,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                     // another rank owns stages its FP32 partial in its own
                     // ring and pushes it there with one bulk copy that counts
                     // its bytes on the owner's barrier.  The owner's quarters
-                    // add the partials in rank order and write their rows.
+                    // add the others' partials to their own in rank order and
+                    // write their rows.
                     const uint32_t S = static_cast<uint32_t>(kp.ksplit);
                     const uint32_t rank = w - g_first;
                     const uint32_t qpr = 4u / (S == 4u ? 4u : 2u);      // lane quarters per rank
@@ -1220,27 +1221,24 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                             // BF16 output through this quarter's [BN][32] staging
                             // block and one TMA store (the map's box)
                             uint8_t *stage = smem + C_::kRedStage + quad * C_::kQStageBytes;
+                            // own partial first, then the others in rank order
+                            // (a fixed order: the result does not depend on
+                            // which copy lands first)
 #pragma unroll 1
                             for (int c = 0; c < BN; c += CW) {
-                                float own[CW], v[CW];
-                                load_acc(t_acc, c, own);
-                                for (uint32_t s = 0; s < S; ++s) {
-                                    if (s == rank) {
-#pragma unroll
-                                        for (int j = 0; j < CW; ++j)
-                                            v[j] = s == 0 ? own[j] : v[j] + own[j];
-                                        continue;
-                                    }
-                                    const uint32_t slot = s < rank ? s : s - 1;
+                                float v[CW];
+                                load_acc(t_acc, c, v);
+#pragma unroll 1
+                                for (uint32_t slot = 0; slot + 1 < S; ++slot) {
                                     const float4 *src = reinterpret_cast<const float4 *>(
                                         smem + C_::kRedOff + (slot * qpr + qj) * C_::kQuadBytes);
 #pragma unroll
                                     for (int j = 0; j < CW / 4; ++j) {
                                         const float4 x = src[(c / 4 + j) * 32 + lane];
-                                        v[4 * j + 0] = s == 0 ? x.x : v[4 * j + 0] + x.x;
-                                        v[4 * j + 1] = s == 0 ? x.y : v[4 * j + 1] + x.y;
-                                        v[4 * j + 2] = s == 0 ? x.z : v[4 * j + 2] + x.z;
-                                        v[4 * j + 3] = s == 0 ? x.w : v[4 * j + 3] + x.w;
+                                        v[4 * j + 0] += x.x;
+                                        v[4 * j + 1] += x.y;
+                                        v[4 * j + 2] += x.z;
+                                        v[4 * j + 3] += x.w;
                                     }
                                 }
                                 if (kp.has_ops)

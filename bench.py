@@ -550,7 +550,7 @@ def run_extra(args, w):
                 "l2": "inputs rotate over %d copies (%.1f MB each)" % (nsets, abytes / 1e6),
                 "timing": "CUDA graph of K steps, CUDA events on the launch stream", "step_us": us,
                 "plan": (mxgemm.mxgemm_describe_grouped_plan(sms, fmt, len(w["groups"]), M, N, K) if op == "grouped"
-                         else mxgemm.mxgemm_describe_plan_for(sms, fmt, M, N, K) if op == "bf16"
+                         else h.describe(mxgemm.FMT_BF16, M, N, K) if op == "bf16"
                          else h.describe(fmt, M, N, K))}),
             "clocks": clocks, "roofline": roof, "cpu_baseline": None,
             "e2e": {"value": job_tflops(fl, world, args.e2e_steps, e2e_ms), "unit": "TFLOPS",

@@ -294,7 +294,8 @@ MXGEMM_API int mxgemm_set_kchunks(mxgemm_handle h, int kc);
  * range of each tile split over a cluster of `ksplit` CTAs, field appended),
  * or for CTA-pair plans dptail: whole tiles, except that the tiles of the
  * last, partial wave (from tail_first on, fields appended) are split into
- * tail_split K ranges over the pairs that wave would leave idle. */
+ * tail_split K ranges over the pairs that wave would leave idle.  fmt
+ * MXGEMM_FMT_BF16 describes the plan of mxgemm_run_bf16 (K % 8 == 0). */
 MXGEMM_API int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
                          char *buf, size_t cap);
 

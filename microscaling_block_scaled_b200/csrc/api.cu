@@ -653,6 +653,13 @@ int mxgemm_describe_plan(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t
 {
     if (!h || !buf || cap == 0)
         return MXGEMM_ERR_INVALID_ARG;
+    if (fmt == MXGEMM_FMT_BF16) {           // the plan of mxgemm_run_bf16
+        if (M < 1 || N < 1 || K < 8 || K % 8 != 0 || M > kMaxDim || N > kMaxDim || K > kMaxDim)
+            return MXGEMM_ERR_INVALID_ARG;
+        format_plan(mxg::make_plan(fmt, M, N, K, h->num_sms, h->sched, h->splits, h->workers, h->kchunks, false),
+                    buf, cap);
+        return MXGEMM_OK;
+    }
     int rc = check_shape(fmt, M, N, K);
     if (rc != MXGEMM_OK)
         return rc;

@@ -297,6 +297,11 @@ def test_bf16_gemm_forced_schedules(sched, M, N, K):
     _no_device_error(h)
     ref, _, mag = oracle.gemm_bf16(ab, bb)
     assert_parity(bits(C), ref, mag, "bf16 forced %s" % (sched,))
+    # the handle describes the BF16 plan under its schedule
+    plan = _with_schedule(h, sched, lambda: h.describe(mxgemm.FMT_BF16, M, N, K))
+    want = {mxgemm.SCHED_SPLITK: "splitk", mxgemm.SCHED_STREAMK: "streamk", mxgemm.SCHED_KSPLIT: "ksplit"}[sched[0]]
+    if not (want == "ksplit" and M > 64):        # the cluster split takes decode tiles only
+        assert "fmt=2" in plan and "sched=" + want in plan, plan
 
 
 def test_bf16_gemm_integer_exact_and_specials():

@@ -428,16 +428,14 @@ struct EpiOps {
     int64_t P, Q, ldc;
 };
 
-// v[j] = act(v[j] + b[j]) + r[j] for the first nv of 32 values, four at a
-// time: four independent chains overlap (one warp per sub-partition runs the
-// epilogue: nothing else hides a long dependency chain), while the code a
-// CTA runs once stays small -- fully unrolled, every CTA fetched ~20 KB of
-// cold instructions for it (a ReLU alone cost ~5 us per decode GEMM).
+// v[j] = act(v[j] + b[j]) + r[j] for the first nv of 32 values, unrolled so
+// the values' independent arithmetic overlaps (one warp per sub-partition
+// runs the epilogue: nothing else hides a long dependency chain).
 template <int ACT>
 __device__ __forceinline__ void ops_run(float (&v)[32], const float (&b)[32], const float (&r)[32], int64_t nv,
                                         bool has_bias, bool has_res)
 {
-#pragma unroll 4
+#pragma unroll
     for (int j = 0; j < 32; ++j) {
         if (j < nv) {
             float x = has_bias ? __fadd_rn(v[j], b[j]) : v[j];
@@ -464,7 +462,7 @@ static __device__ __noinline__ void apply_epilogue_ops(float *vio, int cw, const
             return;
         nv = e.Q - q0 < cw ? e.Q - q0 : cw;
         const uint16_t *res = e.residual ? e.residual + p * e.ldc + q0 : nullptr;
-#pragma unroll 8
+#pragma unroll
         for (int j = 0; j < 32; ++j) {
             b[j] = (e.bias && j < nv) ? bf16_bits_to_float(e.bias[q0 + j]) : 0.0f;
             r[j] = (res && j < nv) ? bf16_bits_to_float(res[j]) : 0.0f;
@@ -474,13 +472,13 @@ static __device__ __noinline__ void apply_epilogue_ops(float *vio, int cw, const
             return;
         nv = e.Q - q0 < cw ? e.Q - q0 : cw;
         const float bp = e.bias ? bf16_bits_to_float(e.bias[p]) : 0.0f;
-#pragma unroll 8
+#pragma unroll
         for (int j = 0; j < 32; ++j) {
             b[j] = bp;
             r[j] = (e.residual && j < nv) ? bf16_bits_to_float(e.residual[(q0 + j) * e.ldc + p]) : 0.0f;
         }
     }
-#pragma unroll 8
+#pragma unroll
     for (int j = 0; j < 32; ++j)
         v[j] = j < nv ? vio[j] : 0.0f;
     const bool hb = e.bias != nullptr, hr = e.residual != nullptr;
@@ -490,7 +488,7 @@ static __device__ __noinline__ void apply_epilogue_ops(float *vio, int cw, const
     case 3: ops_run<3>(v, b, r, nv, hb, hr); break;
     default: ops_run<0>(v, b, r, nv, hb, hr); break;
     }
-#pragma unroll 8
+#pragma unroll
     for (int j = 0; j < 32; ++j)
         if (j < nv)
             vio[j] = v[j];
@@ -539,20 +537,19 @@ static __device__ __noinline__ void quantise_store_plain(const float *vin, const
 // C[m][n] for 32 consecutive n (n = p of each lane, the first a multiple of
 // 32) and rows m = m0 .. m0 + nm - 1 (values vin[j], nm <= 32); for each row
 // the 32 lanes form one run.  All 32 lanes must call with the same m0 and
-// nm.  Four rows at a time, so their reductions and conversions overlap
-// while the code a CTA runs once stays small (see ops_run).
+// nm.  Unrolled over the rows so their reductions and conversions overlap.
 static __device__ __noinline__ void quantise_store_swapped(const float *vin, int nm, const QOut kp, int64_t p,
                                                            int64_t m0, int lane)
 {
     float v[32];
-#pragma unroll 8
+#pragma unroll
     for (int j = 0; j < 32; ++j)
         v[j] = j < nm ? __bfloat162float(__float2bfloat16_rn(vin[j])) : 0.0f;
     uint32_t amax[32];
-#pragma unroll 4
+#pragma unroll
     for (int j = 0; j < 32; ++j)
         amax[j] = __reduce_max_sync(0xffffffffu, __float_as_uint(v[j]) & 0x7FFFFFFFu);
-#pragma unroll 4
+#pragma unroll
     for (int j = 0; j < 32; ++j) {
         if (j < nm) {
             const int64_t m = m0 + j;

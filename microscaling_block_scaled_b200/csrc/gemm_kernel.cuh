@@ -450,9 +450,11 @@ __device__ __forceinline__ void ops_run(float (&v)[32], const float (&b)[32], co
 // layout: the thread holds row m = p, columns n = q0 + j (valid below Q);
 // swapped: column n = p (valid below P), rows m = q0 + j (valid below Q).
 // Values outside C are left alone.  All bias and residual loads are issued
-// before any arithmetic.  Out of line (one copy per translation unit, not
-// per kernel instance); the arithmetic inside is unrolled.
-static __device__ __noinline__ void apply_epilogue_ops(float *vio, int cw, const EpiOps e, int64_t p, int64_t plim,
+// before any arithmetic, and the arithmetic is unrolled.  Inlined into each
+// kernel instance (the build takes minutes longer): as an out-of-line call
+// the kernel's ~170 live registers were saved around it and the fused decode
+// step took 18.8 us against 16.7 us inline.
+static __device__ __forceinline__ void apply_epilogue_ops(float *vio, int cw, const EpiOps e, int64_t p, int64_t plim,
                                                        int64_t q0)
 {
     float v[32], b[32], r[32];
@@ -500,7 +502,7 @@ struct QOut {
     int qfmt;
 };
 
-static __device__ __noinline__ void quantise_store_plain(const float *vin, const QOut kp, int64_t p, int64_t q0)
+static __device__ __forceinline__ void quantise_store_plain(const float *vin, const QOut kp, int64_t p, int64_t q0)
 {
     float v[32];
     uint32_t amax = 0;
@@ -537,8 +539,9 @@ static __device__ __noinline__ void quantise_store_plain(const float *vin, const
 // C[m][n] for 32 consecutive n (n = p of each lane, the first a multiple of
 // 32) and rows m = m0 .. m0 + nm - 1 (values vin[j], nm <= 32); for each row
 // the 32 lanes form one run.  All 32 lanes must call with the same m0 and
-// nm.  Unrolled over the rows so their reductions and conversions overlap.
-static __device__ __noinline__ void quantise_store_swapped(const float *vin, int nm, const QOut kp, int64_t p,
+// nm.  Unrolled over the rows so their reductions and conversions overlap;
+// inlined like apply_epilogue_ops (quantised decode step 18.4 -> 16.1 us).
+static __device__ __forceinline__ void quantise_store_swapped(const float *vin, int nm, const QOut kp, int64_t p,
                                                            int64_t m0, int lane)
 {
     float v[32];

@@ -157,6 +157,7 @@ struct Cfg {
     static_assert(kStaged || 2 * kChunkOutBytes <= kABytes, "ring stage 0 holds two output chunks");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
     static_assert(!kCanKsplit || kRedStage + 4 * kQStageBytes <= kOffOut, "cluster split buffers fit the ring");
+    static_assert(!kCanKsplit || kRedOff + BN * 128 * 4 <= kOffOut, "a staged FP32 decode tile fits the ring");
 };
 
 // Instruction descriptor of the block-scaled MMA (PTX ISA, instruction
@@ -587,6 +588,30 @@ static __device__ __forceinline__ void quantise_store_swapped(const float *vin, 
     }
 }
 
+// One row of quantised output, swapped layout: the 32 lanes of the calling
+// warp hold C[m][n] for 32 consecutive n (n = p, the first a multiple of 32);
+// all lanes call with the same m (lanes with n past N pass valid = false and
+// a zero value).  The same rule as quantise_store_swapped.
+__device__ __forceinline__ void quantise_row_swapped(float vin, const QOut &kp, int64_t m, int64_t p, int lane,
+                                                     bool valid)
+{
+    const float v = __bfloat162float(__float2bfloat16_rn(vin));
+    const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(v) & 0x7FFFFFFFu);
+    float inv;
+    const uint32_t sb = kp.qfmt == kFmtMXFP8 ? mx_block_scale<8>(amax, &inv) : mx_block_scale<2>(amax, &inv);
+    const float q = sb == 0xFFu ? 0.0f : __fmul_rn(v, inv);
+    if (kp.qfmt == kFmtMXFP8) {
+        if (valid)
+            kp.Cq[m * kp.ldc + p] = static_cast<uint8_t>(cvt_e4m3(q));
+    } else {
+        const float hi = __shfl_down_sync(0xffffffffu, q, 1);
+        if ((lane & 1) == 0 && valid)
+            kp.Cq[m * (kp.ldc / 2) + p / 2] = static_cast<uint8_t>(cvt_e2m1x2(hi, q));
+    }
+    if (lane == 0)
+        kp.Cs[m * (kp.ldc / 32) + p / 32] = static_cast<uint8_t>(sb);
+}
+
 template <int FMT, int BN, int KC>
 __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
@@ -684,6 +709,13 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
     // Grouped plans walk their tiles through the group offsets (each role its
     // own walk, all in the same order); plain plans compute them directly.
     const bool grouped = kp.goff != nullptr;
+    // Decode tiles with fused operations or quantised output, one tile per
+    // CTA: on that tile the epilogue warps only stage the FP32 accumulator in
+    // the drained ring, and every warp of the CTA -- the producers and MMA
+    // warps are idle by then -- shares the operations and the stores (the
+    // same decision in every warp, from the parameters alone).
+    const bool spread = C_::kCanKsplit && kp.swap && sc.dp && W <= gridDim.x && !grouped && kp.ksplit <= 1 &&
+                        (kp.has_ops || kp.qfmt >= 0);
     GroupWalk walk;
     if (grouped)
         walk.init(kp.goff, kp.P, kp.Q, kp.groups, kp.tilesQ, BN);
@@ -1128,7 +1160,23 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
                 const uint32_t g_last = sc.dp ? tile : sc.owner(tile * sc.KT + sc.KT - 1);
                 const int64_t p = tc.prow + row;
                 bool released = false;
-                if (g_first == g_last) {
+                if (g_first == g_last && spread) {
+                    // the CTA's only tile: FP32 [BN][128] into the drained ring
+                    float *stage = reinterpret_cast<float *>(smem + C_::kRedOff);
+#pragma unroll
+                    for (int c = 0; c < BN; c += CW) {
+                        float v[CW];
+                        load_acc(t_acc, c, v);
+#pragma unroll
+                        for (int j = 0; j < CW; ++j)
+                            stage[(c + j) * 128 + row] = v[j];
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(acce_bar(acc));
+                    released = true;
+                } else if (g_first == g_last) {
                     // Drain the accumulator row into registers as BF16 pairs and
                     // hand the accumulator back before any store, so the next
                     // tile's MMAs overlap this tile's output traffic.
@@ -1363,6 +1411,76 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
             bulk_wait_group_read<0>();
     }
 
+    if (spread) {
+        // Every warp takes units of the staged tile: unit u is 32 consecutive
+        // rows of the row operand (32 consecutive n of C, one per lane) of
+        // output row m.  Residual and bias loads for all of a warp's units go
+        // out first; the operations run four units per call of ops4.
+        named_bar_sync(2, C_::kThreads);
+        if (!*s_abort) {
+            constexpr int kU = 4 * BN;
+            constexpr int kW = C_::kWarps;
+            constexpr int kMaxU = (kU + kW - 1) / kW;
+            const TileCoord tc = plain_coord(kp, blockIdx.x, BN);
+            const float *stage = reinterpret_cast<const float *>(smem + C_::kRedOff);
+            float sv[kMaxU], bv[kMaxU], rv[kMaxU];
+#pragma unroll
+            for (int i = 0; i < kMaxU; ++i) {
+                const int u = warp + i * kW;
+                const int pb = u & 3, ml = u >> 2;
+                const int64_t p = tc.prow + pb * 32 + lane;
+                const int64_t m = tc.qcol + ml;
+                const bool ok = u < kU && p < kp.P && m < kp.Q;
+                sv[i] = u < kU ? stage[ml * 128 + pb * 32 + lane] : 0.0f;
+                bv[i] = (ok && kp.bias) ? bf16_bits_to_float(kp.bias[p]) : 0.0f;
+                rv[i] = (ok && kp.residual) ? bf16_bits_to_float(kp.residual[m * kp.ldc + p]) : 0.0f;
+            }
+            if (kp.has_ops) {
+                const int hb = kp.bias != nullptr, hr = kp.residual != nullptr;
+#pragma unroll
+                for (int i = 0; i < kMaxU; i += 4) {
+                    const Val4 in{sv[i], i + 1 < kMaxU ? sv[i + 1] : 0.0f, i + 2 < kMaxU ? sv[i + 2] : 0.0f,
+                                  i + 3 < kMaxU ? sv[i + 3] : 0.0f};
+                    const Val4 b4{bv[i], i + 1 < kMaxU ? bv[i + 1] : 0.0f, i + 2 < kMaxU ? bv[i + 2] : 0.0f,
+                                  i + 3 < kMaxU ? bv[i + 3] : 0.0f};
+                    const Val4 r4{rv[i], i + 1 < kMaxU ? rv[i + 1] : 0.0f, i + 2 < kMaxU ? rv[i + 2] : 0.0f,
+                                  i + 3 < kMaxU ? rv[i + 3] : 0.0f};
+                    Val4 o;
+                    switch (kp.act) {
+                    case 1: o = ops4<1>(in, 0.0f, b4, r4, hb, hr); break;
+                    case 2: o = ops4<2>(in, 0.0f, b4, r4, hb, hr); break;
+                    case 3: o = ops4<3>(in, 0.0f, b4, r4, hb, hr); break;
+                    default: o = ops4<0>(in, 0.0f, b4, r4, hb, hr); break;
+                    }
+                    sv[i] = o.a;
+                    if (i + 1 < kMaxU)
+                        sv[i + 1] = o.b;
+                    if (i + 2 < kMaxU)
+                        sv[i + 2] = o.c;
+                    if (i + 3 < kMaxU)
+                        sv[i + 3] = o.d;
+                }
+            }
+            const QOut qo{kp.Cq, kp.Cs, kp.ldc, kp.qfmt};
+#pragma unroll
+            for (int i = 0; i < kMaxU; ++i) {
+                const int u = warp + i * kW;
+                const int pb = u & 3, ml = u >> 2;
+                const int64_t p = tc.prow + pb * 32 + lane;
+                const int64_t m = tc.qcol + ml;
+                // rows past P hold zeros (the loads zero-fill them): valid lanes
+                // and the block's scale depend only on the warp-uniform start
+                if (u < kU && m < kp.Q && tc.prow + pb * 32 < kp.P) {
+                    if (kp.qfmt < 0) {
+                        if (p < kp.P)
+                            kp.C[m * kp.ldc + p] = __float2bfloat16_rn(sv[i]);
+                    } else {
+                        quantise_row_swapped(sv[i], qo, m, p, lane, p < kp.P);
+                    }
+                }
+            }
+        }
+    }
     if (kp.ksplit > 1 && !cl_arrived)
         cluster_arrive();
     tc_fence_before();

@@ -99,6 +99,10 @@ FUSED_PATHS = {
     "swap-splitk3": ((48, 512, 2048), (mxgemm.SCHED_SPLITK, 3, 0)),
     "swap-ksplit4": ((48, 512, 2048), (mxgemm.SCHED_KSPLIT, 4, 0)),
     "swap-dp": ((48, 512, 2048), (mxgemm.SCHED_DP, 1, 0)),
+    # 200 decode tiles on 148 CTAs: some CTAs run two tiles, so the epilogue
+    # warps apply the operations themselves (the all-warps form is for a
+    # CTA's only tile)
+    "swap-multitile": ((24, 128 * 200, 256), None),
 }
 
 
@@ -174,6 +178,7 @@ QPATHS = {
     "splitk3": ((100, 640, 2048), (mxgemm.SCHED_SPLITK, 3, 0)),
     "swap-streamk": ((40, 512, 2048), (mxgemm.SCHED_STREAMK, 1, 37)),
     "swap-ksplit2": ((32, 512, 2048), (mxgemm.SCHED_KSPLIT, 2, 0)),
+    "swap-multitile": ((24, 128 * 200, 256), None),
 }
 
 

@@ -690,6 +690,13 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         fence_mbar_init();
         fence_proxy_async_smem();
     }
+    if (C_::kScaled && BN < 128 && kp.fused_sf) {
+        // rows of the column operand's scale atoms that no stage writes (see
+        // the gather): zero once, by every thread, before the setup barrier
+        uint32_t *z = reinterpret_cast<uint32_t *>(smem + C_::kOffSFB);
+        for (int i = threadIdx.x; i < S * C_::kSFBBytes / 4; i += C_::kThreads)
+            z[i] = 0u;
+    }
     if (warp == 1) {
         tmem_alloc(sbase + C_::kOffMisc, C_::kTmemCols);
         tmem_relinquish();
@@ -733,6 +740,10 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
         // blocks past K are zero-filled) and arrives on the stage's full
         // barrier once its copies have landed.
         const bool sideP = warp == 7;
+        // the column operand of a tile narrower than 128 rows has scales in
+        // only its first BN rows of the atom: 32-row groups past them stay
+        // zero from setup instead of being zero-filled on every stage
+        constexpr int kGatherQ = BN >= 128 ? 4 : (BN + 31) / 32;
         const uint8_t *raw = sideP ? kp.rawP : kp.rawQ;
         const uint32_t bytes = sideP ? C_::kSFABytes : C_::kSFBBytes;
         const uint32_t off = sideP ? C_::kOffSFA : C_::kOffSFB;
@@ -773,6 +784,8 @@ __global__ void __launch_bounds__(Cfg<FMT, BN, KC>::kThreads, 1)
             for (int rb = 0; rb < nrb; ++rb) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
+                    if (!sideP && i >= kGatherQ)
+                        break;          // rows of the atom past the tile: zero since setup
                     const int64_t row = row0 + rb * 128 + i * 32 + lane;
                     const bool rv = row < nrows;
 #pragma unroll

@@ -95,3 +95,17 @@ def test_schedule_overrides_parse_and_key_the_traffic():
     a.schedule, a.kchunks = "splitk:2", 1
     assert bench.traffic_key(a) == "mxfp4_32x14336x4096@splitk2_kc1"
     assert bench.override_config(a) == {"planner_override": "splitk2_kc1"}
+
+
+def test_committed_traffic_matches_the_kernel_sources():
+    """Every recorded DRAM-traffic figure under profiles/ was captured on the
+    current source of its kernel (and planner), so the default workload's
+    roofline.traffic is filled in."""
+    with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+        d = json.load(f)
+    for name, e in d.items():
+        if name == "_about":
+            continue
+        kind = "pair" if "pair" in e["kernel"] else "one_cta"
+        assert bench.recorded_traffic(name, kind) == e["dram_bytes_per_launch"], name
+    assert bench.recorded_traffic(bench.DEFAULT_WORKLOAD, "pair") is not None

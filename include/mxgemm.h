@@ -221,8 +221,17 @@ MXGEMM_API int mxgemm_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64
 
 /* mxgemm_run with HOST buffers (pinned or pageable): copies the operands and
  * scales to device staging buffers owned by the handle, runs the hot path and
- * copies C back to the host buffer C_host, all on `stream`, then synchronises
- * the stream.  Host buffers use the canonical layouts above. */
+ * copies C back to the host buffer C_host, after the work already queued on
+ * `stream`, then synchronises the stream.  Host buffers use the canonical
+ * layouts above.  A product with 32 MB or more of copies runs in blocks of C
+ * (an addition; the pages have no counterpart): row bands of A and of B go
+ * up on a copy stream of the handle, each block's GEMM runs on `stream` once
+ * its two bands have landed, and the block goes down on a second copy stream
+ * of the handle while later bands still go up.  Blocks are multiples of 256
+ * rows and columns with at most 4 parts of M and of N, each at least 2^22
+ * elements.  With profiling on, or while `stream` is capturing, the product
+ * runs as one block.  On return (success or error) no copy of this call is
+ * still in flight. */
 MXGEMM_API int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K,
                     const void *A_host, const uint8_t *A_scales_host,
                     const void *B_host, const uint8_t *B_scales_host,

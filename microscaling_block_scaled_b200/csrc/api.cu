@@ -9,12 +9,18 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <new>
 
 #include "../../include/mxgemm.h"
 #include "mx_internal.h"
+
+// Events of one blocked mxgemm_run_host: entry, exit, one per uploaded band
+// (at most 8 + 8) and one per block of C (at most 64).
+constexpr int kHostParts = 8;
+constexpr int kHostEvents = 2 + 2 * kHostParts + kHostParts * kHostParts;
 
 struct mxgemm_ctx {
     int device = 0;
@@ -29,9 +35,12 @@ struct mxgemm_ctx {
     uint32_t *counters = nullptr;
     size_t counters_cap = 0;
     int *err = nullptr;
-    // device staging of mxgemm_run_host
+    // device staging of mxgemm_run_host, its upload and download streams and
+    // the events that order them against the GEMMs on the caller's stream
     uint8_t *stage = nullptr;
     size_t stage_cap = 0;
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t hev[kHostEvents] = {};
     // schedule override
     int sched = MXGEMM_SCHED_AUTO;
     int splits = 1;
@@ -210,11 +219,14 @@ int do_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const voi
 // middle event keeps the GEMM from starting before the repack ends; with
 // the conversion fused it records no repack time).  A fused epilogue
 // (epi) keeps the plan on one-CTA tiles, whose epilogue implements it.
+// chain = false launches the GEMM without the programmatic dependency, so it
+// starts only once everything before it on the stream has completed.
 int repack_and_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const void *A, const uint8_t *SA,
                     const void *B, const uint8_t *SB, void *C, cudaStream_t st,
-                    const mxg::Epilogue &epi = mxg::Epilogue(), bool allow_pair = true)
+                    const mxg::Epilogue &epi = mxg::Epilogue(), bool allow_pair = true, bool chain = true)
 {
     const bool prof = h->profiling != 0;
+    const int pdl = (prof || !chain) ? 0 : 1;
     h->ev_valid = 0;
     const mxg::GemmPlan pl = plan_for(h, fmt, M, N, K, allow_pair);
     if (!pl.valid)
@@ -230,8 +242,8 @@ int repack_and_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
     }
     if (prof && cudaEventRecord(h->ev[1], st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
-    rc = fused ? launch_plan(h, pl, A, B, C, st, prof ? 0 : 1, h->prefetch_b ? 2 : 0, SA, SB, epi)
-               : launch_plan(h, pl, A, B, C, st, prof ? 0 : 1, 3, nullptr, nullptr, epi);
+    rc = fused ? launch_plan(h, pl, A, B, C, st, pdl, h->prefetch_b ? 2 : 0, SA, SB, epi)
+               : launch_plan(h, pl, A, B, C, st, pdl, 3, nullptr, nullptr, epi);
     if (rc != MXGEMM_OK)
         return rc;
     if (prof) {
@@ -243,6 +255,156 @@ int repack_and_gemm(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
 }
 
 bool optional_aligned16(const void *p) { return p == nullptr || aligned16(p); }
+
+// How mxgemm_run_host cuts a large product into blocks of C.  Over PCIe the
+// copies dominate such a product (8192^3 MXFP8: 132 MB up and 128 MB down
+// against a 0.45 ms GEMM), so the operands go up in row bands of A and of
+// B, each block of C is computed once its two bands have landed, and goes
+// down while later bands still go up.  Parts are multiples of 256 rows (the
+// CTA pair's tile); a block keeps at least 2^22 elements (64 tiles of
+// 256 x 256) so that its GEMM still fills the GPU; under 32 MB of copies the
+// product stays one block.  MXGEMM_HOST_BLOCKS (a measurement knob): "0"
+// keeps every product in one block, "PxQ" cuts products of 32 MB or more
+// into P parts of M and Q of N (1 to 8 each, parts still multiples of 256).
+struct HostBlocks {
+    int64_t mb, nb;  // rows of a full part of M and of N
+    int pm, pn;      // parts
+};
+
+HostBlocks host_blocks(int64_t M, int64_t N, size_t copy_bytes)
+{
+    HostBlocks b{M, N, 1, 1};
+    const char *e = getenv("MXGEMM_HOST_BLOCKS");
+    if (copy_bytes < (size_t(32) << 20) || (e && e[0] == '0' && e[1] == 0))
+        return b;
+    int pm = M >= 4096 ? 4 : (M >= 2048 ? 2 : 1);
+    int pn = N >= 4096 ? 4 : (N >= 2048 ? 2 : 1);
+    auto part = [](int64_t d, int p) { return ((d + p - 1) / p + 255) / 256 * 256; };
+    int fm = 0, fn = 0;
+    if (e && sscanf(e, "%dx%d", &fm, &fn) == 2 && fm >= 1 && fm <= kHostParts && fn >= 1 && fn <= kHostParts) {
+        pm = fm;
+        pn = fn;
+    } else {
+        while ((pm > 1 || pn > 1) && part(M, pm) * part(N, pn) < (int64_t(1) << 22)) {
+            if (pm >= pn)
+                pm /= 2;
+            else
+                pn /= 2;
+        }
+    }
+    if (pm == 1 && pn == 1)
+        return b;
+    b.mb = part(M, pm);
+    b.nb = part(N, pn);
+    b.pm = static_cast<int>((M + b.mb - 1) / b.mb);
+    b.pn = static_cast<int>((N + b.nb - 1) / b.nb);
+    return b;
+}
+
+// The blocked form of mxgemm_run_host.  Three streams: the uploads on
+// h->up, the GEMMs on the caller's stream, the downloads on h->down, ordered
+// by events.  The bands go up as A_0, B_0, A_1, B_1, ...; each block's GEMM
+// waits for the later of its two bands and runs unchained (its operands come
+// from a copy, not from the kernel before it); each block goes down into its
+// rows and columns of C_host once its GEMM is done.  Everything is queued
+// before the first download (one into pageable memory may hold the host
+// thread until it is done), and every stream is drained before returning,
+// on error too, so no copy still touches the caller's buffers.
+int run_host_blocked(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, const uint8_t *A_host,
+                     const uint8_t *SA_host, const uint8_t *B_host, const uint8_t *SB_host, uint8_t *C_host,
+                     uint8_t *dA, uint8_t *dSA, uint8_t *dB, uint8_t *dSB, uint8_t *dC, const HostBlocks &hb,
+                     cudaStream_t st)
+{
+    if (!h->up && cudaStreamCreateWithFlags(&h->up, cudaStreamNonBlocking) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    if (!h->down && cudaStreamCreateWithFlags(&h->down, cudaStreamNonBlocking) != cudaSuccess)
+        return MXGEMM_ERR_CUDA;
+    for (cudaEvent_t &e : h->hev)
+        if (!e && cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess)
+            return MXGEMM_ERR_CUDA;
+    const size_t rb = static_cast<size_t>(mxg::row_bytes(fmt, K));   // bytes of an operand row
+    const size_t sb = static_cast<size_t>(K / 32);                    // bytes of a row's scales
+    auto part_rows = [](int64_t total, int64_t part, int i) {
+        return static_cast<size_t>(total - part * i < part ? total - part * i : part);
+    };
+    cudaEvent_t *ev = h->hev;  // 0 entry, 1 exit, then the bands, then the blocks
+    int next = 2;
+    int a_ev[kHostParts] = {}, b_ev[kHostParts] = {};
+    int blk[kHostParts * kHostParts][2];
+    int nblk = 0, na = 0, nb = 0;
+    auto drain = [&](int rc) {
+        cudaStreamSynchronize(h->up);
+        cudaStreamSynchronize(h->down);
+        cudaStreamSynchronize(st);
+        cudaGetLastError();
+        return rc;
+    };
+    if (cudaEventRecord(ev[0], st) != cudaSuccess || cudaStreamWaitEvent(h->up, ev[0], 0) != cudaSuccess ||
+        cudaStreamWaitEvent(h->down, ev[0], 0) != cudaSuccess)
+        return drain(MXGEMM_ERR_CUDA);
+    for (int t = 0; t < hb.pm || t < hb.pn; ++t) {
+        if (t < hb.pm) {
+            const size_t r0 = static_cast<size_t>(hb.mb) * t, r = part_rows(M, hb.mb, t);
+            if (cudaMemcpyAsync(dA + r0 * rb, A_host + r0 * rb, r * rb, cudaMemcpyHostToDevice, h->up) !=
+                    cudaSuccess ||
+                cudaMemcpyAsync(dSA + r0 * sb, SA_host + r0 * sb, r * sb, cudaMemcpyHostToDevice, h->up) !=
+                    cudaSuccess ||
+                cudaEventRecord(ev[next], h->up) != cudaSuccess)
+                return drain(MXGEMM_ERR_CUDA);
+            a_ev[t] = next++;
+            for (int j = 0; j < nb; ++j) {
+                blk[nblk][0] = t;
+                blk[nblk++][1] = j;
+            }
+            ++na;
+        }
+        if (t < hb.pn) {
+            const size_t r0 = static_cast<size_t>(hb.nb) * t, r = part_rows(N, hb.nb, t);
+            if (cudaMemcpyAsync(dB + r0 * rb, B_host + r0 * rb, r * rb, cudaMemcpyHostToDevice, h->up) !=
+                    cudaSuccess ||
+                cudaMemcpyAsync(dSB + r0 * sb, SB_host + r0 * sb, r * sb, cudaMemcpyHostToDevice, h->up) !=
+                    cudaSuccess ||
+                cudaEventRecord(ev[next], h->up) != cudaSuccess)
+                return drain(MXGEMM_ERR_CUDA);
+            b_ev[t] = next++;
+            for (int i = 0; i < na; ++i) {
+                blk[nblk][0] = i;
+                blk[nblk++][1] = t;
+            }
+            ++nb;
+        }
+    }
+    const int gemm_ev = next;
+    for (int k = 0; k < nblk; ++k) {
+        const int i = blk[k][0], j = blk[k][1];
+        const size_t mi = part_rows(M, hb.mb, i), nj = part_rows(N, hb.nb, j);
+        const size_t m0 = static_cast<size_t>(hb.mb) * i, n0 = static_cast<size_t>(hb.nb) * j;
+        uint8_t *c = dC + (m0 * static_cast<size_t>(N) + mi * n0) * 2;
+        if (cudaStreamWaitEvent(st, ev[a_ev[i] > b_ev[j] ? a_ev[i] : b_ev[j]], 0) != cudaSuccess)
+            return drain(MXGEMM_ERR_CUDA);
+        int rc = repack_and_gemm(h, fmt, static_cast<int64_t>(mi), static_cast<int64_t>(nj), K, dA + m0 * rb,
+                                 dSA + m0 * sb, dB + n0 * rb, dSB + n0 * sb, c, st, mxg::Epilogue(), true, false);
+        if (rc != MXGEMM_OK)
+            return drain(rc);
+        if (cudaEventRecord(ev[gemm_ev + k], st) != cudaSuccess)
+            return drain(MXGEMM_ERR_CUDA);
+    }
+    for (int k = 0; k < nblk; ++k) {
+        const int i = blk[k][0], j = blk[k][1];
+        const size_t mi = part_rows(M, hb.mb, i), nj = part_rows(N, hb.nb, j);
+        const size_t m0 = static_cast<size_t>(hb.mb) * i, n0 = static_cast<size_t>(hb.nb) * j;
+        const uint8_t *c = dC + (m0 * static_cast<size_t>(N) + mi * n0) * 2;
+        if (cudaStreamWaitEvent(h->down, ev[gemm_ev + k], 0) != cudaSuccess ||
+            cudaMemcpy2DAsync(C_host + (m0 * static_cast<size_t>(N) + n0) * 2, static_cast<size_t>(N) * 2, c,
+                              nj * 2, nj * 2, mi, cudaMemcpyDeviceToHost, h->down) != cudaSuccess)
+            return drain(MXGEMM_ERR_CUDA);
+    }
+    if (cudaEventRecord(ev[1], h->down) != cudaSuccess || cudaStreamWaitEvent(st, ev[1], 0) != cudaSuccess)
+        return drain(MXGEMM_ERR_CUDA);
+    if (cudaStreamSynchronize(st) != cudaSuccess)
+        return drain(MXGEMM_ERR_CUDA);
+    return MXGEMM_OK;
+}
 
 void format_plan(const mxg::GemmPlan &pl, char *buf, size_t cap)
 {
@@ -338,6 +500,13 @@ int mxgemm_destroy(mxgemm_handle h)
     for (cudaEvent_t &e : h->ev)
         if (e)
             cudaEventDestroy(e);
+    for (cudaEvent_t &e : h->hev)
+        if (e)
+            cudaEventDestroy(e);
+    if (h->up)
+        cudaStreamDestroy(h->up);
+    if (h->down)
+        cudaStreamDestroy(h->down);
     delete h;
     return rc;
 }
@@ -413,6 +582,16 @@ int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
     if (rc != MXGEMM_OK)
         return rc;
     uint8_t *d = h->stage;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+        cudaGetLastError();
+        return MXGEMM_ERR_CUDA;
+    }
+    const HostBlocks hb = host_blocks(M, N, nA + nSA + nB + nSB + nC);
+    if ((hb.pm > 1 || hb.pn > 1) && !h->profiling && cs == cudaStreamCaptureStatusNone)
+        return run_host_blocked(h, fmt, M, N, K, static_cast<const uint8_t *>(A_host), A_scales_host,
+                                static_cast<const uint8_t *>(B_host), B_scales_host, static_cast<uint8_t *>(C_host),
+                                d + oA, d + oSA, d + oB, d + oSB, d + oC, hb, st);
     if (cudaMemcpyAsync(d + oA, A_host, nA, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(d + oSA, A_scales_host, nSA, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(d + oB, B_host, nB, cudaMemcpyHostToDevice, st) != cudaSuccess ||

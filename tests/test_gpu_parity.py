@@ -11,7 +11,8 @@ import torch
 import oracle
 from microscaling_block_scaled_b200 import mxgemm, synth
 
-from gpu_util import assert_parity, bits, full_case, handle, rows_case, rows_cols_points_case, sampled_case
+from gpu_util import (assert_parity, bits, full_case, gpu_quantize, handle, rows_case, rows_cols_points_case,
+                      sampled_case)
 
 pytestmark = pytest.mark.gpu
 
@@ -415,6 +416,48 @@ def test_repack_then_gemm_equals_run_and_host_path(fmt, M, N, K):
     torch.cuda.synchronize()
     assert torch.equal(C1.view(torch.int16), C2.view(torch.int16))
     assert torch.equal(C1.view(torch.int16).cpu(), C3.view(torch.int16))
+
+
+@pytest.mark.parametrize("fmt,M,N,K,same_plans", [(F8, 4096, 4096, 1024, True), (F4, 3000, 6004, 1024, False)],
+                         ids=["mxfp8-2x2-blocks", "mxfp4-ragged-blocks"])
+def test_host_path_in_blocks(fmt, M, N, K, same_plans):
+    """With 32 MB or more of copies, mxgemm_run_host uploads row bands of A
+    and B, computes each block of C once its bands have landed and
+    downloads it while later bands upload (three streams).  4096 x 4096 runs
+    as 2 x 2 blocks of 2048 x 2048; 3000 x 6004 as 2 x 2 ragged blocks
+    (1536 / 1464 rows by 3072 / 2932 columns).  Two calls with different
+    inputs on one handle, so a GEMM that started before its bands landed
+    would read the first call's operands: each call matches the oracle on
+    whole rows and whole columns on both sides of every block boundary, and
+    where each block runs the same kind of plan as the whole product (CTA
+    pairs), mxgemm_run bit for bit."""
+    h = handle()
+    rows = sorted({0, 1, 1535, 1536, 2047, 2048, M - 2, M - 1})
+    cols = sorted({0, 3, 2047, 2048, 3071, 3072, N - 2, N - 1})
+    for seed in (61, 62):
+        A32, B32 = synth.operands(M, N, K, seed=seed, kind="normal", device="cpu")
+        qa, sa = gpu_quantize(fmt, A32)
+        qb, sb = gpu_quantize(fmt, B32)
+        oa, osa = oracle.quantize(fmt, A32.numpy())
+        ob, osb = oracle.quantize(fmt, B32.numpy())
+        assert np.array_equal(qa.cpu().numpy(), oa) and np.array_equal(sa.cpu().numpy(), osa)
+        assert np.array_equal(qb.cpu().numpy(), ob) and np.array_equal(sb.cpu().numpy(), osb)
+        C = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        C.fill_(float("nan"))
+        h.run_host(fmt, M, N, K, qa.cpu().pin_memory(), sa.cpu().pin_memory(), qb.cpu().pin_memory(),
+                   sb.cpu().pin_memory(), C)
+        st, code = h.check_device_error()
+        assert st == mxgemm.OK and code == 0, ("device error word", code)
+        got = C.view(torch.int16).numpy().view(np.uint16)
+        ref, _, mag = oracle.gemm(fmt, K, oa[rows], osa[rows], ob, osb)
+        assert_parity(got[rows], ref, mag, "host path whole rows, seed %d" % seed)
+        ref, _, mag = oracle.gemm(fmt, K, oa, osa, ob[cols], osb[cols])
+        assert_parity(got[:, cols], ref, mag, "host path whole columns, seed %d" % seed)
+        assert bool(torch.isfinite(C.float()).all())
+        if same_plans:
+            C1 = h.run(fmt, qa, sa, qb, sb, K=K)
+            torch.cuda.synchronize()
+            assert np.array_equal(bits(C1), got)
 
 
 @pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])

@@ -26,38 +26,116 @@ namespace mxg {
 
 namespace {
 
-// Input element as FP32: FP32 as is, BF16 bit patterns widened exactly.
-__device__ __forceinline__ float widen(float x) { return x; }
-__device__ __forceinline__ float widen(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+// The input viewed as one flat sequence of 32-element blocks: K is a
+// multiple of 32, so a block never straddles two rows, and codes and scales
+// are row-major and contiguous too (block b's codes start at byte 32 b for
+// E4M3 and 16 b for E2M1, its scale is byte b).
+//
+// Each lane converts E = 8 consecutive values (32 bytes of FP32 input or 16
+// of BF16); the L = 4 lanes of a block reduce its amax with two shuffles, so
+// a warp tile covers 8 blocks with contiguous loads and stores.  A warp
+// loads U tiles (128 input bytes per lane) before converting any.  The
+// kernel streams from DRAM, but with one value per lane it also ran out of
+// issue slots at the power-capped SM clock: eight values per lane share one
+// amax reduction and scale, and the E4M3 codes are converted in pairs.
+constexpr int kQuantE = 8;
+constexpr int kQuantThreads = 256;
+constexpr int kQuantCtasPerSm = 4;   // 64 registers a thread at most
 
-// One warp per 32-element block; T = float (FP32 input) or uint16_t (BF16
-// bit patterns, widened exactly to FP32 before the rule applies).
+template <typename T>
+struct QuantShape {
+    static constexpr int V = kQuantE * static_cast<int>(sizeof(T)) / 16;   // 16-byte loads a lane: 2 FP32, 1 BF16
+    static constexpr int U = 128 / (16 * V);                              // tiles a warp pass: 4 FP32, 8 BF16
+};
+
+// Two E4M3 codes (RNE, saturating at +-448): `lo` in bits 0..7, `hi` in 8..15.
+__device__ __forceinline__ uint32_t cvt_e4m3_pair(float hi, float lo)
+{
+    uint16_t h;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(hi), "f"(lo));
+    return h;
+}
+
+// The E values of one lane from its 16-byte loads: FP32 as they are, BF16
+// bit patterns widened exactly (element 2i in the low half of word i).
+template <typename T>
+__device__ __forceinline__ void widen(const uint4 (&v)[QuantShape<T>::V], float (&x)[kQuantE])
+{
+#pragma unroll
+    for (int w = 0; w < QuantShape<T>::V; ++w) {
+        const uint32_t wd[4] = {v[w].x, v[w].y, v[w].z, v[w].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if constexpr (sizeof(T) == 4) {
+                x[4 * w + i] = __uint_as_float(wd[i]);
+            } else {
+                x[8 * w + 2 * i] = __uint_as_float(wd[i] << 16);
+                x[8 * w + 2 * i + 1] = __uint_as_float(wd[i] & 0xFFFF0000u);
+            }
+        }
+    }
+}
+
 template <int FMT, typename T>
-__global__ void __launch_bounds__(256) mx_quantize_kernel(const T *__restrict__ X, uint8_t *__restrict__ Q,
-                                                          uint8_t *__restrict__ S, int64_t R, int64_t K)
+__global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm)
+    mx_quantize_kernel(const T *__restrict__ X, uint8_t *__restrict__ Q, uint8_t *__restrict__ S, int64_t total)
 {
     constexpr int kEmax = FMT == kFmtMXFP8 ? 8 : 2;
+    constexpr int E = kQuantE, L = 32 / kQuantE;
+    constexpr int V = QuantShape<T>::V, U = QuantShape<T>::U;
     const int lane = threadIdx.x & 31;
-    const int64_t nb = K / 32;
-    const int64_t nblocks = R * nb;
-    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
-    for (int64_t blk = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + threadIdx.x / 32; blk < nblocks;
-         blk += warps) {
-        const int64_t r = blk / nb, j = blk - r * nb;
-        const float x = widen(X[r * K + j * 32 + lane]);
-        const uint32_t mag = __float_as_uint(x) & 0x7FFFFFFFu;
-        const uint32_t amax = __reduce_max_sync(0xffffffffu, mag);   // NaN > Inf > finite as integers
-        float inv;
-        const uint32_t sbyte = mx_block_scale<kEmax>(amax, &inv);
-        const float q = sbyte == 0xFFu ? 0.0f : __fmul_rn(x, inv);
-        if (lane == 0)
-            S[r * nb + j] = static_cast<uint8_t>(sbyte);
-        if (FMT == kFmtMXFP8) {
-            Q[r * K + j * 32 + lane] = static_cast<uint8_t>(cvt_e4m3(q));
-        } else {
-            const float hi = __shfl_down_sync(0xffffffffu, q, 1);
-            if ((lane & 1) == 0)
-                Q[r * (K / 2) + j * 16 + lane / 2] = static_cast<uint8_t>(cvt_e2m1x2(hi, q));
+    const int64_t chunks = total / E;                 // lane chunks: a multiple of L
+    const int64_t tiles = (chunks + 31) / 32;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    for (int64_t t0 = warp * U; t0 < tiles; t0 += nwarps * U) {   // warp-uniform
+        const int64_t c0 = t0 * 32;
+        const int rem = chunks - c0 < 32 * U ? static_cast<int>(chunks - c0) : 32 * U;
+        const uint4 *src = reinterpret_cast<const uint4 *>(X) + c0 * V;
+        uint4 v[U][V];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = u * 32 + lane;
+#pragma unroll
+            for (int w = 0; w < V; ++w)
+                v[u][w] = c < rem ? __ldcs(src + c * V + w) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = u * 32 + lane;
+            float x[E];
+            widen<T>(v[u], x);
+            uint32_t m = 0;
+#pragma unroll
+            for (int k = 0; k < E; ++k) {
+                const uint32_t mag = __float_as_uint(x[k]) & 0x7FFFFFFFu;   // NaN > Inf > finite
+                m = mag > m ? mag : m;
+            }
+#pragma unroll
+            for (int off = L / 2; off >= 1; off /= 2) {
+                const uint32_t o = __shfl_xor_sync(0xffffffffu, m, off);
+                m = o > m ? o : m;
+            }
+            float inv;
+            const uint32_t sbyte = mx_block_scale<kEmax>(m, &inv);
+            if (c >= rem)
+                continue;
+            float q[E];
+#pragma unroll
+            for (int k = 0; k < E; ++k)
+                q[k] = sbyte == 0xFFu ? 0.0f : __fmul_rn(x[k], inv);
+            const int64_t gc = c0 + c;
+            if (lane % L == 0)
+                S[gc / L] = static_cast<uint8_t>(sbyte);
+            if constexpr (FMT == kFmtMXFP8) {
+                const uint32_t w0 = cvt_e4m3_pair(q[1], q[0]) | (cvt_e4m3_pair(q[3], q[2]) << 16);
+                const uint32_t w1 = cvt_e4m3_pair(q[5], q[4]) | (cvt_e4m3_pair(q[7], q[6]) << 16);
+                *reinterpret_cast<uint2 *>(Q + gc * E) = make_uint2(w0, w1);
+            } else {
+                *reinterpret_cast<uint32_t *>(Q + gc * (E / 2)) =
+                    cvt_e2m1x2(q[1], q[0]) | (cvt_e2m1x2(q[3], q[2]) << 8) | (cvt_e2m1x2(q[5], q[4]) << 16) |
+                    (cvt_e2m1x2(q[7], q[6]) << 24);
+            }
         }
     }
 }
@@ -67,24 +145,28 @@ __global__ void __launch_bounds__(256) mx_quantize_kernel(const T *__restrict__ 
 cudaError_t launch_quantize(int fmt, int64_t R, int64_t K, const float *X, uint8_t *Q, uint8_t *S,
                             cudaStream_t stream, const uint16_t *X_bf16)
 {
-    const int64_t nblocks = R * (K / 32);
-    if (nblocks == 0)
+    const int64_t total = R * K;
+    if (total == 0)
         return cudaSuccess;
-    const int threads = 256;
-    int64_t grid = (nblocks + 7) / 8;
-    if (grid > 148 * 64)
-        grid = 148 * 64;
+    // lane chunks of kQuantE values, 32 per warp tile, U tiles per warp and
+    // pass; one wave of kQuantCtasPerSm CTAs on each of 148 SMs at most
+    const int U = X_bf16 ? QuantShape<uint16_t>::U : QuantShape<float>::U;
+    const int64_t chunks = total / kQuantE;
+    const int64_t per_cta = 32LL * U * (kQuantThreads / 32);
+    int64_t grid = (chunks + per_cta - 1) / per_cta;
+    if (grid > 148 * kQuantCtasPerSm)
+        grid = 148 * kQuantCtasPerSm;
     const unsigned g = static_cast<unsigned>(grid);
     if (X_bf16) {
         if (fmt == kFmtMXFP8)
-            mx_quantize_kernel<kFmtMXFP8, uint16_t><<<g, threads, 0, stream>>>(X_bf16, Q, S, R, K);
+            mx_quantize_kernel<kFmtMXFP8, uint16_t><<<g, kQuantThreads, 0, stream>>>(X_bf16, Q, S, total);
         else
-            mx_quantize_kernel<kFmtMXFP4, uint16_t><<<g, threads, 0, stream>>>(X_bf16, Q, S, R, K);
+            mx_quantize_kernel<kFmtMXFP4, uint16_t><<<g, kQuantThreads, 0, stream>>>(X_bf16, Q, S, total);
     } else {
         if (fmt == kFmtMXFP8)
-            mx_quantize_kernel<kFmtMXFP8, float><<<g, threads, 0, stream>>>(X, Q, S, R, K);
+            mx_quantize_kernel<kFmtMXFP8, float><<<g, kQuantThreads, 0, stream>>>(X, Q, S, total);
         else
-            mx_quantize_kernel<kFmtMXFP4, float><<<g, threads, 0, stream>>>(X, Q, S, R, K);
+            mx_quantize_kernel<kFmtMXFP4, float><<<g, kQuantThreads, 0, stream>>>(X, Q, S, total);
     }
     return cudaGetLastError();
 }

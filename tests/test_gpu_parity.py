@@ -4,6 +4,7 @@ Pass rule per element: |C_gpu - C_ref| <= 1 BF16 ulp(C_ref) + 2^-18 * sum_k |a_k
 with identical NaN / +-Inf positions; quantised codes and scales must agree
 bit for bit.
 """
+import ml_dtypes
 import numpy as np
 import pytest
 import torch
@@ -29,6 +30,32 @@ def test_quantiser_bit_exact(fmt, kind):
     oq, os_ = oracle.quantize(fmt, A32.numpy())
     assert np.array_equal(s.cpu().numpy(), os_)
     assert np.array_equal(q.cpu().numpy(), oq)
+
+
+@pytest.mark.parametrize("fmt", [F8, F4], ids=["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("bf16_input", [False, True], ids=["fp32", "bf16"])
+@pytest.mark.parametrize("R,K", [(1, 32), (3, 96), (5, 160), (7, 4128), (33, 2080)])
+def test_quantiser_ragged_sizes_bit_exact(fmt, bf16_input, R, K):
+    """The quantiser covers the input in warp tiles of 32 chunks of 16 bytes,
+    four tiles per warp and pass.  Sizes that end inside a tile or inside a
+    warp's group of four match the oracle bit for bit, with FP32 and BF16
+    input, and leave the bytes past the codes and scales untouched."""
+    X32, _ = synth.operands(R, 1, K, seed=R + K, kind="heavy")
+    qw = K if fmt == F8 else K // 2
+    Qp = torch.full((R * qw + 64,), 0xA5, dtype=torch.uint8, device="cuda")
+    Sp = torch.full((R * (K // 32) + 64,), 0x5A, dtype=torch.uint8, device="cuda")
+    out = (Qp[:R * qw].view(R, qw), Sp[:R * (K // 32)].view(R, K // 32))
+    if bf16_input:
+        xb = np.ascontiguousarray(X32.numpy().astype(ml_dtypes.bfloat16).view(np.uint16))
+        mxgemm.quantize_bf16(fmt, torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16), out=out)
+        oq, os_ = oracle.quantize_bf16(fmt, xb)
+    else:
+        mxgemm.quantize(fmt, X32.cuda().contiguous(), out=out)
+        oq, os_ = oracle.quantize(fmt, X32.numpy())
+    torch.cuda.synchronize()
+    assert np.array_equal(out[1].cpu().numpy(), os_)
+    assert np.array_equal(out[0].cpu().numpy(), oq)
+    assert bool((Qp[R * qw:] == 0xA5).all()) and bool((Sp[R * (K // 32):] == 0x5A).all())
 
 
 @pytest.mark.parametrize("fmt", [F8, F4])

@@ -31,21 +31,22 @@ namespace {
 // are row-major and contiguous too (block b's codes start at byte 32 b for
 // E4M3 and 16 b for E2M1, its scale is byte b).
 //
-// Each lane converts E = 8 consecutive values (32 bytes of FP32 input or 16
-// of BF16); the L = 4 lanes of a block reduce its amax with two shuffles, so
-// a warp tile covers 8 blocks with contiguous loads and stores.  A warp
-// loads U tiles (128 input bytes per lane) before converting any.  The
-// kernel streams from DRAM, but with one value per lane it also ran out of
-// issue slots at the power-capped SM clock: eight values per lane share one
-// amax reduction and scale, and the E4M3 codes are converted in pairs.
-constexpr int kQuantE = 8;
+// Each lane converts the E values of 32 input bytes (8 FP32 or 16 BF16,
+// two 16-byte loads); the L = 32 / E lanes of a block reduce its amax with
+// shuffles, so a warp tile covers 1 KB of input with contiguous loads and
+// stores.  A warp loads U = 4 tiles (128 input bytes per lane) before
+// converting any.  The kernel streams from DRAM, but with one value per lane
+// it also ran out of issue slots at the power-capped SM clock: the values of
+// a lane share one amax reduction and scale, and the E4M3 codes are
+// converted in pairs.
 constexpr int kQuantThreads = 256;
 constexpr int kQuantCtasPerSm = 4;   // 64 registers a thread at most
 
 template <typename T>
 struct QuantShape {
-    static constexpr int V = kQuantE * static_cast<int>(sizeof(T)) / 16;   // 16-byte loads a lane: 2 FP32, 1 BF16
-    static constexpr int U = 128 / (16 * V);                              // tiles a warp pass: 4 FP32, 8 BF16
+    static constexpr int E = 32 / static_cast<int>(sizeof(T));   // values a lane: 8 FP32, 16 BF16
+    static constexpr int V = 2;                                  // 16-byte loads a lane and tile
+    static constexpr int U = 4;                                  // tiles a warp pass
 };
 
 // Two E4M3 codes (RNE, saturating at +-448): `lo` in bits 0..7, `hi` in 8..15.
@@ -59,7 +60,7 @@ __device__ __forceinline__ uint32_t cvt_e4m3_pair(float hi, float lo)
 // The E values of one lane from its 16-byte loads: FP32 as they are, BF16
 // bit patterns widened exactly (element 2i in the low half of word i).
 template <typename T>
-__device__ __forceinline__ void widen(const uint4 (&v)[QuantShape<T>::V], float (&x)[kQuantE])
+__device__ __forceinline__ void widen(const uint4 (&v)[QuantShape<T>::V], float (&x)[QuantShape<T>::E])
 {
 #pragma unroll
     for (int w = 0; w < QuantShape<T>::V; ++w) {
@@ -81,7 +82,7 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm)
     mx_quantize_kernel(const T *__restrict__ X, uint8_t *__restrict__ Q, uint8_t *__restrict__ S, int64_t total)
 {
     constexpr int kEmax = FMT == kFmtMXFP8 ? 8 : 2;
-    constexpr int E = kQuantE, L = 32 / kQuantE;
+    constexpr int E = QuantShape<T>::E, L = 32 / E;
     constexpr int V = QuantShape<T>::V, U = QuantShape<T>::U;
     const int lane = threadIdx.x & 31;
     const int64_t chunks = total / E;                 // lane chunks: a multiple of L
@@ -128,13 +129,24 @@ __global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm)
             if (lane % L == 0)
                 S[gc / L] = static_cast<uint8_t>(sbyte);
             if constexpr (FMT == kFmtMXFP8) {
-                const uint32_t w0 = cvt_e4m3_pair(q[1], q[0]) | (cvt_e4m3_pair(q[3], q[2]) << 16);
-                const uint32_t w1 = cvt_e4m3_pair(q[5], q[4]) | (cvt_e4m3_pair(q[7], q[6]) << 16);
-                *reinterpret_cast<uint2 *>(Q + gc * E) = make_uint2(w0, w1);
+                uint32_t w[E / 4];   // 4 codes a word
+#pragma unroll
+                for (int i = 0; i < E / 4; ++i)
+                    w[i] = cvt_e4m3_pair(q[4 * i + 1], q[4 * i]) | (cvt_e4m3_pair(q[4 * i + 3], q[4 * i + 2]) << 16);
+                if constexpr (E == 8)
+                    *reinterpret_cast<uint2 *>(Q + gc * E) = make_uint2(w[0], w[1]);
+                else
+                    *reinterpret_cast<uint4 *>(Q + gc * E) = make_uint4(w[0], w[1], w[2], w[3]);
             } else {
-                *reinterpret_cast<uint32_t *>(Q + gc * (E / 2)) =
-                    cvt_e2m1x2(q[1], q[0]) | (cvt_e2m1x2(q[3], q[2]) << 8) | (cvt_e2m1x2(q[5], q[4]) << 16) |
-                    (cvt_e2m1x2(q[7], q[6]) << 24);
+                uint32_t w[E / 8];   // 8 codes a word
+#pragma unroll
+                for (int i = 0; i < E / 8; ++i)
+                    w[i] = cvt_e2m1x2(q[8 * i + 1], q[8 * i]) | (cvt_e2m1x2(q[8 * i + 3], q[8 * i + 2]) << 8) |
+                           (cvt_e2m1x2(q[8 * i + 5], q[8 * i + 4]) << 16) | (cvt_e2m1x2(q[8 * i + 7], q[8 * i + 6]) << 24);
+                if constexpr (E == 8)
+                    *reinterpret_cast<uint32_t *>(Q + gc * (E / 2)) = w[0];
+                else
+                    *reinterpret_cast<uint2 *>(Q + gc * (E / 2)) = make_uint2(w[0], w[1]);
             }
         }
     }
@@ -148,10 +160,10 @@ cudaError_t launch_quantize(int fmt, int64_t R, int64_t K, const float *X, uint8
     const int64_t total = R * K;
     if (total == 0)
         return cudaSuccess;
-    // lane chunks of kQuantE values, 32 per warp tile, U tiles per warp and
+    // lane chunks of 32 input bytes, 32 per warp tile, U tiles per warp and
     // pass; one wave of kQuantCtasPerSm CTAs on each of 148 SMs at most
     const int U = X_bf16 ? QuantShape<uint16_t>::U : QuantShape<float>::U;
-    const int64_t chunks = total / kQuantE;
+    const int64_t chunks = total / (X_bf16 ? QuantShape<uint16_t>::E : QuantShape<float>::E);
     const int64_t per_cta = 32LL * U * (kQuantThreads / 32);
     int64_t grid = (chunks + per_cta - 1) / per_cta;
     if (grid > 148 * kQuantCtasPerSm)

@@ -36,7 +36,7 @@ def test_quantiser_bit_exact(fmt, kind):
 @pytest.mark.parametrize("bf16_input", [False, True], ids=["fp32", "bf16"])
 @pytest.mark.parametrize("R,K", [(1, 32), (3, 96), (5, 160), (7, 4128), (33, 2080)])
 def test_quantiser_ragged_sizes_bit_exact(fmt, bf16_input, R, K):
-    """The quantiser covers the input in warp tiles of 32 chunks of 16 bytes,
+    """The quantiser covers the input in warp tiles of 32 lanes x 32 bytes,
     four tiles per warp and pass.  Sizes that end inside a tile or inside a
     warp's group of four match the oracle bit for bit, with FP32 and BF16
     input, and leave the bytes past the codes and scales untouched."""

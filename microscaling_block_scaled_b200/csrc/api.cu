@@ -592,16 +592,24 @@ int mxgemm_run_host(mxgemm_handle h, int fmt, int64_t M, int64_t N, int64_t K, c
         return run_host_blocked(h, fmt, M, N, K, static_cast<const uint8_t *>(A_host), A_scales_host,
                                 static_cast<const uint8_t *>(B_host), B_scales_host, static_cast<uint8_t *>(C_host),
                                 d + oA, d + oSA, d + oB, d + oSB, d + oC, hb, st);
+    // on error, wait for the copies already queued (a capturing stream holds
+    // none: its work has not run)
+    auto drain = [&](int code) {
+        if (cs == cudaStreamCaptureStatusNone)
+            cudaStreamSynchronize(st);
+        cudaGetLastError();
+        return code;
+    };
     if (cudaMemcpyAsync(d + oA, A_host, nA, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(d + oSA, A_scales_host, nSA, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(d + oB, B_host, nB, cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(d + oSB, B_scales_host, nSB, cudaMemcpyHostToDevice, st) != cudaSuccess)
-        return MXGEMM_ERR_CUDA;
+        return drain(MXGEMM_ERR_CUDA);
     rc = repack_and_gemm(h, fmt, M, N, K, d + oA, d + oSA, d + oB, d + oSB, d + oC, st);
     if (rc != MXGEMM_OK)
-        return rc;
+        return drain(rc);
     if (cudaMemcpyAsync(C_host, d + oC, nC, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        return MXGEMM_ERR_CUDA;
+        return drain(MXGEMM_ERR_CUDA);
     if (cudaStreamSynchronize(st) != cudaSuccess)
         return MXGEMM_ERR_CUDA;
     return MXGEMM_OK;
